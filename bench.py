@@ -1,0 +1,444 @@
+#!/usr/bin/env python
+"""Benchmark of the two-level sparse-attention path on B200.
+
+One step = one pass of the whole path (block pooling, block scoring + top-m,
+token scoring + top-k, sparse attention) over one batch of synthetic input
+already resident in HBM.  The default workload is the 64K-token prefill
+(1 sequence, B=128, m=64, k=2048, 16 heads of 128); the metric is queries per
+second, with the attention kernel's fraction of the HBM roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own independent
+copy of the workload (a different seed); there is no collective on the data
+path, so scaling is weak and the value is all ranks' queries over the slowest
+rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "hierarchical indexer+sparse-attn queries/s at 64K prefill; % of HBM roofline"
+UNIT = "queries/s"
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="prefill_64k")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
+    return ap.parse_args()
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def closed_form_counts(w):
+    """Per-query candidate counts and kept tokens from the closed forms of the path."""
+    import numpy as np
+
+    i = np.arange(w.n_q, dtype=np.int64)
+    p = w.n_kv - w.n_q + i
+    c = p // w.block
+    s = np.minimum(w.top_m, c + 1)
+    n_cand = np.where(s == c + 1, p + 1, (s - 1) * w.block + p % w.block + 1)
+    k_eff = np.minimum(w.top_k, n_cand)
+    return {"n_cand": int(n_cand.sum()) * w.batch, "k_eff": int(k_eff.sum()) * w.batch,
+            "n_vis": int((c + 1).sum()) * w.batch}
+
+
+def attention_bytes(w, counts):
+    """Algorithmic bytes of one sparse-attention launch: every kept (token, head) K and V row
+    once per query, plus the query rows, output rows, LSE and index lists."""
+    nq = w.batch * w.n_q
+    gather = counts["k_eff"] * w.n_heads * w.d_head * 2 * 2
+    return gather + nq * w.n_heads * w.d_head * 2 * 2 + nq * w.n_heads * 4 + nq * w.top_k * 4
+
+
+def indexer_bytes(w, counts):
+    nq = w.batch * w.n_q
+    return (counts["n_cand"] * w.d_idx * 2            # token gather
+            + w.batch * w.n_kv * w.d_idx * 2            # pooling read
+            + nq * w.d_idx * 2 + nq * (w.top_m + w.top_k) * 4)
+
+
+def _profile_traffic(kernel_file: str, summary_name: str):
+    """DRAM bytes per launch from the committed ncu summary, or None when the kernel changed since."""
+    path = os.path.join(ROOT, "profiles", summary_name)
+    src = os.path.join(ROOT, "hierarchical_sparse_attention_block_b200", "csrc", kernel_file)
+    try:
+        with open(path) as f:
+            j = json.load(f)
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if j.get("source_sha256_16") != sha:
+            return None
+        return j.get("dram_bytes_per_launch_full_workload")
+    except Exception:
+        return None
+
+
+def run_ours(a, rank, world, local_rank):
+    import numpy as np
+    import torch
+
+    import hierarchical_sparse_attention_block_b200 as hs
+    import synth.device as sd
+    from synth.workloads import WORKLOADS
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = WORKLOADS[a.workload].with_(seed=WORKLOADS[a.workload].seed + rank)
+    p = hs.params_of(w)
+    inp = sd.device_inputs(w, device=dev)
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+
+    nq = w.batch * w.n_q
+    bk = torch.empty((w.batch, w.n_blk, w.d_idx), dtype=torch.float32, device=dev)
+    blk = torch.empty((w.batch, w.n_q, w.top_m), dtype=torch.int32, device=dev)
+    tok = torch.empty((w.batch, w.n_q, w.top_k), dtype=torch.int32, device=dev)
+    o = torch.empty((w.batch, w.n_q, w.n_heads, w.d_head), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.batch, w.n_q, w.n_heads), dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    ws_topm = torch.empty(hs.hisa_block_topm_workspace_size(p), dtype=torch.uint8, device=dev)
+    ws_tok = torch.empty(hs.hisa_token_topk_workspace_size(p)[1], dtype=torch.uint8, device=dev)
+    n_attn_ws = hs.hisa_sparse_attn_workspace_size(p)
+    ws_attn = torch.empty(max(n_attn_ws, 16), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    stages = ["pool", "block_topm", "token_topk", "sparse_attn"]
+
+    def step(ev):
+        ev[0].record(st)
+        hs.hisa_block_pool(p, inp["k_idx"], bk, stream=st)
+        ev[1].record(st)
+        hs.hisa_block_topm(p, inp["q_idx"], bk, blk, None, status, ws_topm, stream=st)
+        ev[2].record(st)
+        hs.hisa_token_topk(p, inp["q_idx"], inp["k_idx"], blk, tok, None, status, ws_tok, stream=st)
+        ev[3].record(st)
+        hs.sparse_attn_fwd(p, inp["q"], inp["k"], inp["v"], tok, o, lse, status, ws_attn, stream=st)
+        ev[4].record(st)
+
+    def new_events():
+        return [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+
+    for _ in range(a.warmup):
+        flush.zero_()
+        step(new_events())
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} after warm-up")
+
+    # the indexer alone and the flat comparator, for the speedup figure (outside the timed steps)
+    comp = {}
+    if world == 1:
+        flat_tok = torch.empty_like(tok)
+        fmin, fpref = hs.hisa_flat_topk_workspace_size(p)
+        ws_flat = torch.empty(fpref, dtype=torch.uint8, device=dev)
+        for _ in range(2):
+            hs.hisa_flat_topk(p, inp["q_idx"], inp["k_idx"], flat_tok, None, ws_flat, stream=st)
+        reps = max(2, min(a.steps, 5))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        tt = []
+        for _ in range(reps):
+            flush.zero_()
+            e0.record(st)
+            hs.hisa_flat_topk(p, inp["q_idx"], inp["k_idx"], flat_tok, None, ws_flat, stream=st)
+            e1.record(st)
+            e1.synchronize()
+            tt.append(e0.elapsed_time(e1))
+        comp["flat_indexer_ms"] = statistics.median(tt)
+        del ws_flat, flat_tok
+
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    evs = [new_events() for _ in range(a.steps)]
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else 0) as clk:
+        g0.record(st)
+        for s in range(a.steps):
+            flush.zero_()
+            step(evs[s])
+        g1.record(st)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    stage_ms = {n: [] for n in stages}
+    step_ms = []
+    for ev in evs:
+        for j, n in enumerate(stages):
+            stage_ms[n].append(ev[j].elapsed_time(ev[j + 1]))
+        step_ms.append(ev[0].elapsed_time(ev[4]))
+    ms = sum(step_ms) / len(step_ms)
+    region_ms = g0.elapsed_time(g1)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} in the timed steps")
+
+    counts = closed_form_counts(w)
+    hbm_gbs, peak_kind = _peaks()
+    attn_ms = statistics.mean(stage_ms["sparse_attn"])
+    a_bytes = attention_bytes(w, counts)
+    achieved = a_bytes / (attn_ms * 1e-3) / 1e9
+    idx_ms = sum(statistics.mean(stage_ms[n]) for n in stages[:3])
+
+    # launches per step: pool, block score, top-m, 2 per token chunk, attention (+ merge)
+    per_q_keys = w.top_m * w.block * 4
+    chunk = max(1, ws_tok.numel() // per_q_keys)
+    n_chunks = math.ceil(nq / chunk)
+    splits = 1 if n_attn_ws == 0 else 2
+    launches = 3 + 2 * n_chunks + (1 if splits == 1 else 2)
+
+    result = {
+        "metric": METRIC, "value": nq * world / (ms * 1e-3), "unit": UNIT, "n_gpus": world, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded SplitMix64; integer indexer q/k in [-4,4], unit-variance "
+                                  "Irwin-Hall Q/K/V, planted needle blocks)",
+        "config": {"workload": w.name, "batch": w.batch, "n_q": w.n_q, "n_kv": w.n_kv, "d_idx": w.d_idx,
+                   "block": w.block, "top_m": w.top_m, "top_k": w.top_k, "n_heads": w.n_heads, "d_head": w.d_head,
+                   "needles": w.needles, "parallelism": f"dp{world} (independent copies)",
+                   "l2": f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write)"},
+        "roofline": {"bound": "hbm", "kernel": "sparse_attn", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
+                     "frac": achieved / hbm_gbs, "peak_kind": peak_kind,
+                     "frac_of_nominal_8tbs": achieved / 8000.0,
+                     "algorithmic_bytes_per_launch": a_bytes,
+                     "traffic": _profile_traffic("sparse_attn.cu", "sparse_attn_prefill_64k.json")},
+        "stages_ms": {n: statistics.mean(v) for n, v in stage_ms.items()},
+        "indexer_ms": idx_ms, "indexer_queries_per_s": nq / (idx_ms * 1e-3),
+        "tokens_per_s": counts["k_eff"] / (ms * 1e-3),
+        "end_to_end_hbm_roofline_frac_8tbs": ((a_bytes + indexer_bytes(w, counts)) / 8e12) / (ms * 1e-3),
+        "region_ms_incl_l2_flush": region_ms,
+        "gpu_launches": launches * a.steps,
+        "clocks": clk.summary(),
+    }
+    if comp:
+        result["flat_indexer_ms"] = comp["flat_indexer_ms"]
+        result["speedup_vs_flat_indexer"] = comp["flat_indexer_ms"] / idx_ms
+
+    if not a.no_e2e:
+        result["e2e"] = run_e2e(a, hs, w, p, inp, dev, st, world)
+    del inp
+    torch.cuda.empty_cache()
+    return result
+
+
+def run_e2e(a, hs, w, p, inp, dev, st, world):
+    """The same metric through hisa_forward with host-resident inputs: every step copies its
+    inputs from pinned host memory and reads the outputs back."""
+    import torch
+
+    host = {k: v.cpu().pin_memory() for k, v in inp.items() if not k.startswith("_")}
+    d_in = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+    o = torch.empty((w.batch, w.n_q, w.n_heads, w.d_head), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.batch, w.n_q, w.n_heads), dtype=torch.float32, device=dev)
+    h_o = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    h_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    ws = torch.empty(hs.hisa_forward_workspace_size(p), dtype=torch.uint8, device=dev)
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = o.numel() * 2 + lse.numel() * 4
+
+    def one():
+        for k in host:
+            d_in[k].copy_(host[k], non_blocking=True)
+        hs.hisa_forward(p, d_in["q_idx"], d_in["k_idx"], d_in["q"], d_in["k"], d_in["v"], o, lse, None, None, None,
+                        ws, stream=st)
+        h_o.copy_(o, non_blocking=True)
+        h_lse.copy_(lse, non_blocking=True)
+
+    for _ in range(max(1, a.warmup)):
+        one()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    steps = max(1, min(a.steps, 5))
+    e0.record(st)
+    for _ in range(steps):
+        one()
+    e1.record(st)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    del host, d_in, ws
+    return {"value": w.batch * w.n_q * world / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
+
+
+def oracle_sample(w, seconds: float, device_inputs=None):
+    """Time the CPU oracle (as it stands) on a position-stratified sample of queries, scaled to
+    queries/s.  Inputs come from the seeded generator (device half, bit-identical to the host half)."""
+    import numpy as np
+
+    import oracle
+    from synth.workloads import full_inputs
+
+    O = oracle.Oracle()
+    threads = O.threads()
+    if device_inputs is not None:
+        inp = {k: v.view(__import__("torch").int16).cpu().numpy().view(np.uint16)
+               for k, v in device_inputs.items() if not k.startswith("_")}
+    else:
+        inp = full_inputs(w)
+    t0 = time.perf_counter()
+    bkeys = np.stack([O.block_pool(inp["k_idx"][s], w.block) for s in range(w.batch)])
+    pool_s = time.perf_counter() - t0
+    nq = w.batch * w.n_q
+    n = 8
+    done, elapsed = 0, 0.0
+    rng = np.random.default_rng(0)
+    while elapsed < seconds and done < nq:
+        ids = np.sort(rng.choice(nq, size=min(n, nq), replace=False)).astype(np.int64)
+        t0 = time.perf_counter()
+        O.run(w, inp, query_ids=ids, block_keys=bkeys)
+        elapsed += time.perf_counter() - t0
+        done += len(ids)
+        n = min(n * 2, 4096)
+    per_q = elapsed / done
+    total_s = pool_s + per_q * nq
+    return {"value": nq / total_s, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{done} of {nq} queries drawn uniformly over positions, full path (pooling, top-m, top-k, "
+                      f"attention in fp64), plus pooling of every block; {elapsed + pool_s:.1f} s of CPU time, "
+                      f"scaled to the whole workload"}
+
+
+def main():
+    a = _args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+
+    if a.impl == "reference":
+        if rank == 0:
+            from synth.workloads import WORKLOADS
+
+            w = WORKLOADS[a.workload]
+            cpu = oracle_sample(w, a.cpu_seconds * max(1, a.steps) / 10.0)
+            line = {"impl": "reference", "metric": METRIC, "value": cpu["value"], "unit": UNIT, "n_gpus": world,
+                    "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * w.batch * w.n_q / cpu["value"],
+                    "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                    "data": "synthetic", "config": {"workload": w.name},
+                    "cpu_baseline": {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")},
+                    "e2e": {"value": cpu["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            print(json.dumps(line), flush=True)
+        if world > 1:
+            import torch
+
+            torch.distributed.destroy_process_group()
+        return
+
+    import torch
+
+    res = run_ours(a, rank, world, local_rank)
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        import synth.device as sd
+        from synth.workloads import WORKLOADS
+
+        w = WORKLOADS[a.workload]
+        small = w.batch * w.n_q <= 8192
+        dev_inp = None if small else sd.device_inputs(w, device=torch.device("cuda", local_rank))
+        res["cpu_baseline"] = oracle_sample(w, a.cpu_seconds, dev_inp)
+        del dev_inp
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

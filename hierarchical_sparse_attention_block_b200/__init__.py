@@ -1,0 +1,227 @@
+"""Python binding of the two-level sparse-attention library (include/hisa.h).
+
+Argument marshalling only: every step of the path runs in the CUDA kernels of
+``libhisa.so``.  PyTorch supplies device memory and the current stream.  The
+library must be built (``hierarchical_sparse_attention_block_b200.build``);
+importing this package without it raises ImportError -- there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libhisa.so")
+
+HISA_OK, HISA_ERR_INVALID_ARG, HISA_ERR_UNSUPPORTED, HISA_ERR_WORKSPACE, HISA_ERR_CUDA = range(5)
+STATUS_BAD_INDEX = 1
+STATUS_TIMEOUT = 2
+
+# Every exported symbol of include/hisa.h.
+EXPORTS = (
+    "hisa_block_pool", "hisa_block_topm_workspace_size", "hisa_block_topm", "hisa_token_topk_workspace_size",
+    "hisa_token_topk", "hisa_sparse_attn_workspace_size", "sparse_attn_fwd", "hisa_forward_workspace_size",
+    "hisa_forward", "hisa_flat_topk_workspace_size", "hisa_flat_topk", "hisa_status_string",
+    "hisa_last_cuda_error", "hisa_version",
+)
+
+
+class HisaParams(ctypes.Structure):
+    """Mirror of hisa_params_t."""
+
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("d_idx", ctypes.c_int32), ("n_q", ctypes.c_int64), ("n_kv", ctypes.c_int64),
+        ("block", ctypes.c_int32), ("top_m", ctypes.c_int32), ("top_k", ctypes.c_int32),
+        ("n_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32), ("d_head", ctypes.c_int32),
+        ("scale", ctypes.c_float), ("flags", ctypes.c_int32),
+    ]
+
+
+class HisaError(RuntimeError):
+    def __init__(self, call: str, status: int):
+        detail = _lib.hisa_status_string(status).decode()
+        if status == HISA_ERR_CUDA:
+            detail += f" (cudaError {_lib.hisa_last_cuda_error()})"
+        super().__init__(f"{call}: {detail}")
+        self.status = status
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m hierarchical_sparse_attention_block_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i64, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.POINTER(ctypes.c_size_t)
+    pp = ctypes.POINTER(HisaParams)
+    sig = {
+        "hisa_block_pool": [pp, vp, i64, i64, vp, vp],
+        "hisa_block_topm_workspace_size": [pp, sz],
+        "hisa_block_topm": [pp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
+        "hisa_token_topk_workspace_size": [pp, sz, sz],
+        "hisa_token_topk": [pp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
+        "hisa_sparse_attn_workspace_size": [pp, sz],
+        "sparse_attn_fwd": [pp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
+        "hisa_forward_workspace_size": [pp, sz],
+        "hisa_forward": [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
+        "hisa_flat_topk_workspace_size": [pp, sz, sz],
+        "hisa_flat_topk": [pp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
+    }
+    for name, args in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = ctypes.c_int
+    lib.hisa_status_string.argtypes = [ctypes.c_int]
+    lib.hisa_status_string.restype = ctypes.c_char_p
+    lib.hisa_last_cuda_error.restype = ctypes.c_int32
+    lib.hisa_version.restype = ctypes.c_char_p
+    return lib
+
+
+_lib = _load()
+
+
+def lib():
+    return _lib
+
+
+def params(batch, n_q, n_kv, d_idx, block, top_m, top_k, n_heads=1, n_kv_heads=None, d_head=64,
+           scale=0.0) -> HisaParams:
+    return HisaParams(batch=batch, d_idx=d_idx, n_q=n_q, n_kv=n_kv, block=block, top_m=top_m, top_k=top_k,
+                      n_heads=n_heads, n_kv_heads=n_kv_heads if n_kv_heads else n_heads, d_head=d_head,
+                      scale=scale, flags=0)
+
+
+def params_of(w) -> HisaParams:
+    """hisa_params_t of a workload description (synth.workloads.Workload or alike)."""
+    return params(w.batch, w.n_q, w.n_kv, w.d_idx, w.block, w.top_m, w.top_k, w.n_heads, w.n_kv_heads, w.d_head)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(name, rc):
+    if rc != HISA_OK:
+        raise HisaError(name, rc)
+
+
+def _size(fn, p, two=False):
+    a = ctypes.c_size_t(0)
+    if two:
+        b = ctypes.c_size_t(0)
+        _check(fn.__name__, fn(ctypes.byref(p), ctypes.byref(a), ctypes.byref(b)))
+        return a.value, b.value
+    _check(fn.__name__, fn(ctypes.byref(p), ctypes.byref(a)))
+    return a.value
+
+
+def _workspace(nbytes, device):
+    import torch
+
+    return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+
+
+# ---------------------------------------------------------------- calls of include/hisa.h
+
+def hisa_block_pool(p, k_idx, block_keys, blk_begin=0, blk_end=-1, stream=None):
+    _check("hisa_block_pool", _lib.hisa_block_pool(ctypes.byref(p), _ptr(k_idx), blk_begin, blk_end,
+                                                   _ptr(block_keys), _stream(stream)))
+
+
+def hisa_block_topm_workspace_size(p) -> int:
+    return _size(_lib.hisa_block_topm_workspace_size, p)
+
+
+def hisa_block_topm(p, q_idx, block_keys, block_idx, block_scores=None, dev_status=None, workspace=None,
+                    stream=None):
+    if workspace is None:
+        workspace = _workspace(hisa_block_topm_workspace_size(p), q_idx.device)
+    _check("hisa_block_topm", _lib.hisa_block_topm(ctypes.byref(p), _ptr(q_idx), _ptr(block_keys), _ptr(block_idx),
+                                                   _ptr(block_scores), _ptr(dev_status), _ptr(workspace),
+                                                   workspace.numel(), _stream(stream)))
+
+
+def hisa_token_topk_workspace_size(p):
+    """(minimum, preferred) bytes."""
+    return _size(_lib.hisa_token_topk_workspace_size, p, two=True)
+
+
+def hisa_token_topk(p, q_idx, k_idx, block_idx, token_idx, token_scores=None, dev_status=None, workspace=None,
+                    stream=None):
+    if workspace is None:
+        workspace = _workspace(hisa_token_topk_workspace_size(p)[1], q_idx.device)
+    _check("hisa_token_topk", _lib.hisa_token_topk(ctypes.byref(p), _ptr(q_idx), _ptr(k_idx), _ptr(block_idx),
+                                                   _ptr(token_idx), _ptr(token_scores), _ptr(dev_status),
+                                                   _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def hisa_sparse_attn_workspace_size(p) -> int:
+    return _size(_lib.hisa_sparse_attn_workspace_size, p)
+
+
+def sparse_attn_fwd(p, q, k, v, token_idx, o, lse=None, dev_status=None, workspace=None, stream=None):
+    if workspace is None:
+        n = hisa_sparse_attn_workspace_size(p)
+        workspace = _workspace(n, q.device) if n else None
+    _check("sparse_attn_fwd", _lib.sparse_attn_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(token_idx),
+                                                   _ptr(o), _ptr(lse), _ptr(dev_status), _ptr(workspace),
+                                                   0 if workspace is None else workspace.numel(), _stream(stream)))
+
+
+def hisa_forward_workspace_size(p) -> int:
+    return _size(_lib.hisa_forward_workspace_size, p)
+
+
+def hisa_forward(p, q_idx, k_idx, q, k, v, o, lse=None, block_idx_out=None, token_idx_out=None, dev_status=None,
+                 workspace=None, stream=None):
+    if workspace is None:
+        workspace = _workspace(hisa_forward_workspace_size(p), q_idx.device)
+    _check("hisa_forward", _lib.hisa_forward(ctypes.byref(p), _ptr(q_idx), _ptr(k_idx), _ptr(q), _ptr(k), _ptr(v),
+                                             _ptr(o), _ptr(lse), _ptr(block_idx_out), _ptr(token_idx_out),
+                                             _ptr(dev_status), _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def hisa_flat_topk_workspace_size(p):
+    return _size(_lib.hisa_flat_topk_workspace_size, p, two=True)
+
+
+def hisa_flat_topk(p, q_idx, k_idx, token_idx, token_scores=None, workspace=None, stream=None):
+    if workspace is None:
+        workspace = _workspace(hisa_flat_topk_workspace_size(p)[1], q_idx.device)
+    _check("hisa_flat_topk", _lib.hisa_flat_topk(ctypes.byref(p), _ptr(q_idx), _ptr(k_idx), _ptr(token_idx),
+                                                 _ptr(token_scores), _ptr(workspace), workspace.numel(),
+                                                 _stream(stream)))
+
+
+def hisa_version() -> str:
+    return _lib.hisa_version().decode()
+
+
+# ---------------------------------------------------------------- convenience front end
+
+def forward(p, q_idx, k_idx, q, k, v, return_indices=False, stream=None):
+    """Allocate the outputs with torch and run hisa_forward; returns (o, lse[, block_idx, token_idx])."""
+    import torch
+
+    dev = q_idx.device
+    o = torch.empty((p.batch, p.n_q, p.n_heads, p.d_head), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((p.batch, p.n_q, p.n_heads), dtype=torch.float32, device=dev)
+    blk = tok = None
+    if return_indices:
+        blk = torch.empty((p.batch, p.n_q, p.top_m), dtype=torch.int32, device=dev)
+        tok = torch.empty((p.batch, p.n_q, p.top_k), dtype=torch.int32, device=dev)
+    hisa_forward(p, q_idx, k_idx, q, k, v, o, lse, blk, tok, stream=stream)
+    return (o, lse, blk, tok) if return_indices else (o, lse)
+
+
+def n_blocks(p) -> int:
+    return math.ceil(p.n_kv / p.block)

@@ -1,0 +1,339 @@
+// C ABI (include/hisa.h): argument validation, workspace sizing and the
+// order of launches.  Every step of the path runs in the kernels of this
+// library; this file only checks arguments and enqueues them.
+#include <math.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "hisa.h"
+#include "internal.h"
+
+namespace hisa {
+
+namespace {
+
+thread_local int32_t g_last_cuda_error = 0;
+
+hisa_status_t cuda_fail(cudaError_t e) {
+  if (e == cudaSuccess) return HISA_OK;
+  g_last_cuda_error = (int32_t)e;
+  return HISA_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+bool pow2(int64_t x) { return x > 0 && (x & (x - 1)) == 0; }
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// Validation shared by every call.  need_attn: the attention fields matter.
+hisa_status_t make_shape(const hisa_params_t* p, bool need_indexer, bool need_attn, Shape* s) {
+  if (!p) return HISA_ERR_INVALID_ARG;
+  if (p->flags != 0) return HISA_ERR_INVALID_ARG;
+  if (p->batch < 1 || p->batch > 65535) return HISA_ERR_INVALID_ARG;
+  if (p->n_kv < 1 || p->n_kv > 0x7FFFFFFFLL) return HISA_ERR_INVALID_ARG;
+  if (p->n_q < 1 || p->n_q > p->n_kv) return HISA_ERR_INVALID_ARG;
+  if (p->top_k < 1) return HISA_ERR_INVALID_ARG;
+  s->batch = p->batch;
+  s->n_q = p->n_q;
+  s->n_kv = p->n_kv;
+  s->d_idx = p->d_idx;
+  s->B = p->block;
+  s->m = p->top_m;
+  s->k = p->top_k;
+  s->H = p->n_heads;
+  s->Hkv = p->n_kv_heads;
+  s->d = p->d_head;
+  s->n_query = (int64_t)p->batch * p->n_q;
+  if (need_indexer) {
+    if (p->block < 1 || !pow2(p->block) || p->block > 4096) return p->block < 1 ? HISA_ERR_INVALID_ARG : HISA_ERR_UNSUPPORTED;
+    if (p->top_m < 2) return HISA_ERR_INVALID_ARG;
+    if (p->d_idx != 64 && p->d_idx != 128 && p->d_idx != 256) return p->d_idx < 1 ? HISA_ERR_INVALID_ARG : HISA_ERR_UNSUPPORTED;
+    s->n_blk = (p->n_kv + p->block - 1) / p->block;
+    if ((int64_t)p->top_m * p->block > (int64_t)1 << 24) return HISA_ERR_UNSUPPORTED;
+  } else {
+    s->n_blk = p->block >= 1 ? (p->n_kv + p->block - 1) / p->block : 0;
+  }
+  if (need_attn) {
+    if (p->n_heads < 1 || p->n_kv_heads < 1 || p->n_heads % p->n_kv_heads != 0) return HISA_ERR_INVALID_ARG;
+    if (p->d_head != 64 && p->d_head != 128) return p->d_head < 1 ? HISA_ERR_INVALID_ARG : HISA_ERR_UNSUPPORTED;
+    if (!(p->scale == p->scale) || isinf(p->scale)) return HISA_ERR_INVALID_ARG;
+    s->scale = p->scale > 0.f ? p->scale : (float)(1.0 / sqrt((double)p->d_head));
+  } else {
+    s->scale = 0.f;
+  }
+  return HISA_OK;
+}
+
+size_t topm_ws(const Shape& s) {
+  size_t b = align_up((size_t)s.n_query * s.n_blk * sizeof(float));
+  if (block_score_tc_eligible(s)) b += align_up(block_score_tc_scratch_bytes(s));
+  return b;
+}
+
+size_t token_keys_per_query(const Shape& s, int slots) { return (size_t)slots * s.B * sizeof(uint32_t); }
+
+constexpr size_t kKeysCap = (size_t)4 << 30;  // preferred key buffer cap: 4 GiB
+
+size_t keys_preferred(const Shape& s, int slots) {
+  const size_t per = token_keys_per_query(s, slots);
+  const size_t all = per * (size_t)s.n_query;
+  if (all <= kKeysCap) return all;
+  size_t nq = kKeysCap / per;
+  if (nq < 1) nq = 1;
+  return nq * per;
+}
+
+// Token stage over all queries, in as few chunks as the key buffer allows.
+hisa_status_t run_token_stage(const Shape& s, const void* q_idx, const void* k_idx, const int32_t* block_idx,
+                              int slots, int32_t* token_idx, float* token_scores, int32_t* status, void* keys_buf,
+                              size_t keys_bytes, cudaStream_t st) {
+  const size_t per = token_keys_per_query(s, slots);
+  const int64_t chunk = (int64_t)(keys_bytes / per);
+  if (chunk < 1) return HISA_ERR_WORKSPACE;
+  uint32_t* keys = static_cast<uint32_t*>(keys_buf);
+  for (int64_t q0 = 0; q0 < s.n_query; q0 += chunk) {
+    const int64_t nq = s.n_query - q0 < chunk ? s.n_query - q0 : chunk;
+    cudaError_t e = launch_token_score(s, q_idx, k_idx, block_idx, slots, keys, status, q0, nq, st);
+    if (e == cudaSuccess) e = launch_token_select(s, keys, block_idx, slots, token_idx, token_scores, q0, nq, st);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  return HISA_OK;
+}
+
+hisa_status_t run_block_stage(const Shape& s, const void* q_idx, const float* block_keys, int32_t* block_idx,
+                              float* block_scores, int32_t* status, void* ws, cudaStream_t st) {
+  float* scores = static_cast<float*>(ws);
+  cudaError_t e = cudaErrorNotSupported;
+  if (block_score_tc_eligible(s)) e = launch_block_score_tc(s, q_idx, block_keys, scores, status, st);
+  if (e == cudaErrorNotSupported) e = launch_block_score(s, q_idx, block_keys, scores, st);
+  if (e == cudaSuccess) e = launch_block_topm(s, scores, block_idx, block_scores, st);
+  return cuda_fail(e);
+}
+
+}  // namespace
+
+cudaError_t ensure_smem(const void* func, int bytes) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  static std::mutex mu;
+  static const void* done_f[64][16];
+  static int done_b[64][16];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev >= 0 && dev < 64) {
+    for (int i = 0; i < 16; ++i)
+      if (done_f[dev][i] == func && done_b[dev][i] >= bytes) return cudaSuccess;
+  }
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64) {
+    for (int i = 0; i < 16; ++i) {
+      if (done_f[dev][i] == nullptr || done_f[dev][i] == func) {
+        done_f[dev][i] = func;
+        done_b[dev][i] = bytes;
+        break;
+      }
+    }
+  }
+  return cudaSuccess;
+}
+
+}  // namespace hisa
+
+using hisa::Shape;
+
+extern "C" {
+
+const char* hisa_status_string(hisa_status_t status) {
+  switch (status) {
+    case HISA_OK: return "ok";
+    case HISA_ERR_INVALID_ARG: return "invalid argument";
+    case HISA_ERR_UNSUPPORTED: return "unsupported size";
+    case HISA_ERR_WORKSPACE: return "workspace missing or too small";
+    case HISA_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+int32_t hisa_last_cuda_error(void) { return hisa::g_last_cuda_error; }
+
+const char* hisa_version(void) { return "hisa-b200 0.1.0"; }
+
+hisa_status_t hisa_block_pool(const hisa_params_t* params, const void* k_idx, int64_t blk_begin, int64_t blk_end,
+                              float* block_keys, cudaStream_t stream) {
+  Shape s;
+  hisa_status_t rc = hisa::make_shape(params, true, false, &s);
+  if (rc != HISA_OK) return rc;
+  if (!k_idx || !block_keys || !hisa::aligned16(k_idx) || !hisa::aligned16(block_keys)) return HISA_ERR_INVALID_ARG;
+  if (blk_end < 0) blk_end = s.n_blk;
+  if (blk_begin < 0 || blk_begin > blk_end || blk_end > s.n_blk) return HISA_ERR_INVALID_ARG;
+  return hisa::cuda_fail(hisa::launch_block_pool(s, k_idx, blk_begin, blk_end, block_keys, stream));
+}
+
+hisa_status_t hisa_block_topm_workspace_size(const hisa_params_t* params, size_t* bytes) {
+  Shape s;
+  hisa_status_t rc = hisa::make_shape(params, true, false, &s);
+  if (rc != HISA_OK) return rc;
+  if (!bytes) return HISA_ERR_INVALID_ARG;
+  *bytes = hisa::topm_ws(s);
+  return HISA_OK;
+}
+
+hisa_status_t hisa_block_topm(const hisa_params_t* params, const void* q_idx, const float* block_keys,
+                              int32_t* block_idx, float* block_scores, int32_t* dev_status, void* workspace,
+                              size_t workspace_bytes, cudaStream_t stream) {
+  Shape s;
+  hisa_status_t rc = hisa::make_shape(params, true, false, &s);
+  if (rc != HISA_OK) return rc;
+  if (!q_idx || !block_keys || !block_idx) return HISA_ERR_INVALID_ARG;
+  if (!hisa::aligned16(q_idx) || !hisa::aligned16(block_keys) || !hisa::aligned16(block_idx)) return HISA_ERR_INVALID_ARG;
+  if (block_scores && !hisa::aligned16(block_scores)) return HISA_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < hisa::topm_ws(s) || !hisa::aligned16(workspace)) return HISA_ERR_WORKSPACE;
+  return hisa::run_block_stage(s, q_idx, block_keys, block_idx, block_scores, dev_status, workspace, stream);
+}
+
+hisa_status_t hisa_token_topk_workspace_size(const hisa_params_t* params, size_t* min_bytes, size_t* preferred_bytes) {
+  Shape s;
+  hisa_status_t rc = hisa::make_shape(params, true, false, &s);
+  if (rc != HISA_OK) return rc;
+  if (!min_bytes && !preferred_bytes) return HISA_ERR_INVALID_ARG;
+  if (min_bytes) *min_bytes = hisa::token_keys_per_query(s, s.m);
+  if (preferred_bytes) *preferred_bytes = hisa::keys_preferred(s, s.m);
+  return HISA_OK;
+}
+
+hisa_status_t hisa_token_topk(const hisa_params_t* params, const void* q_idx, const void* k_idx,
+                              const int32_t* block_idx, int32_t* token_idx, float* token_scores, int32_t* dev_status,
+                              void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  Shape s;
+  hisa_status_t rc = hisa::make_shape(params, true, false, &s);
+  if (rc != HISA_OK) return rc;
+  if (!q_idx || !k_idx || !block_idx || !token_idx) return HISA_ERR_INVALID_ARG;
+  if (!hisa::aligned16(q_idx) || !hisa::aligned16(k_idx) || !hisa::aligned16(block_idx) || !hisa::aligned16(token_idx))
+    return HISA_ERR_INVALID_ARG;
+  if (token_scores && !hisa::aligned16(token_scores)) return HISA_ERR_INVALID_ARG;
+  if (!workspace || !hisa::aligned16(workspace)) return HISA_ERR_WORKSPACE;
+  return hisa::run_token_stage(s, q_idx, k_idx, block_idx, s.m, token_idx, token_scores, dev_status, workspace,
+                               workspace_bytes, stream);
+}
+
+hisa_status_t hisa_sparse_attn_workspace_size(const hisa_params_t* params, size_t* bytes) {
+  Shape s;
+  hisa_status_t rc = hisa::make_shape(params, false, true, &s);
+  if (rc != HISA_OK) return rc;
+  if (!bytes) return HISA_ERR_INVALID_ARG;
+  *bytes = hisa::attn_partial_bytes(s, hisa::attn_pick_splits(s));
+  return HISA_OK;
+}
+
+hisa_status_t sparse_attn_fwd(const hisa_params_t* params, const void* q, const void* k, const void* v,
+                              const int32_t* token_idx, void* o, float* lse, int32_t* dev_status, void* workspace,
+                              size_t workspace_bytes, cudaStream_t stream) {
+  Shape s;
+  hisa_status_t rc = hisa::make_shape(params, false, true, &s);
+  if (rc != HISA_OK) return rc;
+  if (!q || !k || !v || !token_idx || !o) return HISA_ERR_INVALID_ARG;
+  if (!hisa::aligned16(q) || !hisa::aligned16(k) || !hisa::aligned16(v) || !hisa::aligned16(token_idx) ||
+      !hisa::aligned16(o))
+    return HISA_ERR_INVALID_ARG;
+  if (lse && !hisa::aligned16(lse)) return HISA_ERR_INVALID_ARG;
+  int splits = hisa::attn_pick_splits(s);
+  if (splits > 1 && (!workspace || !hisa::aligned16(workspace) || workspace_bytes < hisa::attn_partial_bytes(s, splits)))
+    splits = 1;
+  return hisa::cuda_fail(hisa::launch_sparse_attn(s, q, k, v, token_idx, o, lse, dev_status, splits, workspace, stream));
+}
+
+// Workspace of hisa_forward: block keys | block stage | block_idx | token_idx | attention partials | token keys.
+namespace {
+struct FwdLayout {
+  size_t bk, blk_stage, block_idx, token_idx, attn, keys, total;
+};
+FwdLayout fwd_layout(const Shape& s) {
+  FwdLayout L;
+  size_t off = 0;
+  L.bk = off;
+  off += hisa::align_up((size_t)s.batch * s.n_blk * s.d_idx * sizeof(float));
+  L.blk_stage = off;
+  off += hisa::topm_ws(s);
+  L.block_idx = off;
+  off += hisa::align_up((size_t)s.n_query * s.m * sizeof(int32_t));
+  L.token_idx = off;
+  off += hisa::align_up((size_t)s.n_query * s.k * sizeof(int32_t));
+  L.attn = off;
+  off += hisa::align_up(hisa::attn_partial_bytes(s, hisa::attn_pick_splits(s)));
+  L.keys = off;
+  off += hisa::align_up(hisa::keys_preferred(s, s.m));
+  L.total = off;
+  return L;
+}
+}  // namespace
+
+hisa_status_t hisa_forward_workspace_size(const hisa_params_t* params, size_t* bytes) {
+  Shape s;
+  hisa_status_t rc = hisa::make_shape(params, true, true, &s);
+  if (rc != HISA_OK) return rc;
+  if (!bytes) return HISA_ERR_INVALID_ARG;
+  *bytes = fwd_layout(s).total;
+  return HISA_OK;
+}
+
+hisa_status_t hisa_forward(const hisa_params_t* params, const void* q_idx, const void* k_idx, const void* q,
+                           const void* k, const void* v, void* o, float* lse, int32_t* block_idx_out,
+                           int32_t* token_idx_out, int32_t* dev_status, void* workspace, size_t workspace_bytes,
+                           cudaStream_t stream) {
+  Shape s;
+  hisa_status_t rc = hisa::make_shape(params, true, true, &s);
+  if (rc != HISA_OK) return rc;
+  const void* ptrs[] = {q_idx, k_idx, q, k, v, o};
+  for (const void* p : ptrs)
+    if (!p || !hisa::aligned16(p)) return HISA_ERR_INVALID_ARG;
+  if ((lse && !hisa::aligned16(lse)) || (block_idx_out && !hisa::aligned16(block_idx_out)) ||
+      (token_idx_out && !hisa::aligned16(token_idx_out)))
+    return HISA_ERR_INVALID_ARG;
+  const FwdLayout L = fwd_layout(s);
+  if (!workspace || !hisa::aligned16(workspace) || workspace_bytes < L.total) return HISA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* bk = reinterpret_cast<float*>(ws + L.bk);
+  int32_t* blk = block_idx_out ? block_idx_out : reinterpret_cast<int32_t*>(ws + L.block_idx);
+  int32_t* tok = token_idx_out ? token_idx_out : reinterpret_cast<int32_t*>(ws + L.token_idx);
+
+  cudaError_t e = hisa::launch_block_pool(s, k_idx, 0, s.n_blk, bk, stream);
+  if (e != cudaSuccess) return hisa::cuda_fail(e);
+  rc = hisa::run_block_stage(s, q_idx, bk, blk, nullptr, dev_status, ws + L.blk_stage, stream);
+  if (rc != HISA_OK) return rc;
+  rc = hisa::run_token_stage(s, q_idx, k_idx, blk, s.m, tok, nullptr, dev_status, ws + L.keys,
+                             workspace_bytes - L.keys, stream);
+  if (rc != HISA_OK) return rc;
+  const int splits = hisa::attn_pick_splits(s);
+  return hisa::cuda_fail(hisa::launch_sparse_attn(s, q, k, v, tok, o, lse, dev_status, splits, ws + L.attn, stream));
+}
+
+hisa_status_t hisa_flat_topk_workspace_size(const hisa_params_t* params, size_t* min_bytes, size_t* preferred_bytes) {
+  Shape s;
+  hisa_status_t rc = hisa::make_shape(params, true, false, &s);
+  if (rc != HISA_OK) return rc;
+  if (!min_bytes && !preferred_bytes) return HISA_ERR_INVALID_ARG;
+  if (s.n_blk > 50000 || s.n_blk * (int64_t)s.B > ((int64_t)1 << 30)) return HISA_ERR_UNSUPPORTED;
+  if (min_bytes) *min_bytes = hisa::token_keys_per_query(s, (int)s.n_blk);
+  if (preferred_bytes) *preferred_bytes = hisa::keys_preferred(s, (int)s.n_blk);
+  return HISA_OK;
+}
+
+hisa_status_t hisa_flat_topk(const hisa_params_t* params, const void* q_idx, const void* k_idx, int32_t* token_idx,
+                             float* token_scores, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  Shape s;
+  hisa_status_t rc = hisa::make_shape(params, true, false, &s);
+  if (rc != HISA_OK) return rc;
+  if (!q_idx || !k_idx || !token_idx) return HISA_ERR_INVALID_ARG;
+  if (!hisa::aligned16(q_idx) || !hisa::aligned16(k_idx) || !hisa::aligned16(token_idx)) return HISA_ERR_INVALID_ARG;
+  if (token_scores && !hisa::aligned16(token_scores)) return HISA_ERR_INVALID_ARG;
+  if (!workspace || !hisa::aligned16(workspace)) return HISA_ERR_WORKSPACE;
+  if (s.n_blk > 50000 || s.n_blk * (int64_t)s.B > ((int64_t)1 << 30)) return HISA_ERR_UNSUPPORTED;
+  return hisa::run_token_stage(s, q_idx, k_idx, nullptr, (int)s.n_blk, token_idx, token_scores, nullptr, workspace,
+                               workspace_bytes, stream);
+}
+
+}  // extern "C"

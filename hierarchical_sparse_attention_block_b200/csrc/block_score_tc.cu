@@ -1,0 +1,340 @@
+// Step 2 on the 5th-generation tensor cores (prefill): scores = Q_idx x BKᵀ.
+// "北大HISA稀疏注意力机制" section 1.2.1 item 2 (block scores with the
+// indexer's dot product); QbitAI HISA article, "塊級粗過濾".
+//
+// One CTA (one warpgroup) per tile of 128 queries x 128 blocks of one
+// sequence; tiles entirely above the causal diagonal exit at once.
+//   * TMA brings the 128 query rows (bf16, 128-byte swizzle: already the
+//     K-major UMMA operand layout) and the 128 fp32 block keys (unswizzled
+//     staging) into shared memory, completing on an mbarrier.
+//   * The fp32 block keys are split into three bf16 terms,
+//     x = hi + mid + lo (each term the bf16 rounding of what is left), and
+//     written as three K-major swizzled B operands.  Every product of a bf16
+//     query with a bf16 term is exact, so the fp32 accumulation gives the same
+//     score as an fp32 dot product up to summation order -- and exactly the
+//     same score on integer-valued inputs.
+//   * One thread issues 3 x (d_idx / 16) tcgen05.mma (kind::f16, M=N=128,
+//     fp32 accumulator in 128 TMEM columns) and commits them to an mbarrier.
+//   * Each warp reads its 32 TMEM lanes (= query rows) back with tcgen05.ld
+//     and stores the causally visible scores.
+// Every wait is bounded (1 s of %globaltimer); a timeout sets status bit 1
+// and the CTA skips to releasing its TMEM.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace hisa {
+namespace {
+
+constexpr int kTcThreads = 128;
+constexpr int kTileM = 128;  // queries per tile
+constexpr int kTileN = 128;  // blocks per tile
+constexpr int kStatusTimeout = 2;
+constexpr uint64_t kWaitNs = 1000000000ull;
+
+template <int D>
+struct TcLayout {
+  static constexpr int HALVES = D / 64;                // 128-byte K slices
+  static constexpr int A_BYTES = HALVES * kTileM * 128;
+  static constexpr int B_PLANE = HALVES * kTileN * 128;
+  static constexpr int B_BYTES = 3 * B_PLANE;
+  static constexpr int S_BYTES = kTileN * D * 4;       // fp32 block-key staging
+  static constexpr int A_OFF = 0;
+  static constexpr int B_OFF = A_OFF + A_BYTES;
+  static constexpr int S_OFF = B_OFF + B_BYTES;
+  static constexpr int BAR_OFF = S_OFF + S_BYTES;      // 2 mbarriers + TMEM address
+  static constexpr int SMEM = BAR_OFF + 64 + 1024;     // + slack for 1024-byte alignment
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase) {
+  const uint64_t t0 = global_ns();
+  while (true) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(phase)
+        : "memory");
+    if (ok) return true;
+    if (global_ns() - t0 > kWaitNs) return false;
+  }
+}
+
+// K-major operand, 128-byte swizzle: rows of 128 B, 8-row groups 1024 B apart.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1 << 16;           // leading byte offset (unused for this layout): 16 B
+  d |= (uint64_t)(1024 >> 4) << 32; // stride byte offset: 1024 B between 8-row groups
+  d |= (uint64_t)1 << 46;           // descriptor version (sm_100)
+  d |= (uint64_t)2 << 61;           // swizzle: 128 B
+  return d;
+}
+
+// kind::f16 instruction descriptor: bf16 x bf16 -> fp32, both K-major, M = 128, N = 128.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kTileN >> 3) << 17) |
+                            ((uint32_t)(kTileM >> 4) << 24);
+
+__device__ __forceinline__ uint32_t bf16_bits(float x) {
+  __nv_bfloat16 h = __float2bfloat16_rn(x);
+  return (uint32_t)(*reinterpret_cast<uint16_t*>(&h));
+}
+
+template <int D>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    block_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_bk,
+                          float* __restrict__ scores, int32_t* __restrict__ status, int64_t n_q, int64_t n_kv,
+                          int B, int64_t n_blk, int q_tiles, int n_tiles) {
+  using L = TcLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+
+  const int nt = blockIdx.x % n_tiles;
+  const int qt_all = blockIdx.x / n_tiles;
+  const int seq = qt_all / q_tiles;
+  const int qt = qt_all % q_tiles;
+  const int64_t q0 = (int64_t)qt * kTileM;
+  const int64_t q_last = min(q0 + kTileM, n_q) - 1;
+  const int64_t c_max = (n_kv - n_q + q_last) / B;
+  const int64_t j0 = (int64_t)nt * kTileN;
+  if (j0 > c_max) return;  // whole tile above the causal diagonal
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint8_t* sA = smem + L::A_OFF;
+  uint8_t* sB = smem + L::B_OFF;
+  const float* sS = reinterpret_cast<const float*>(smem + L::S_OFF);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::BAR_OFF + 16);
+  const uint32_t bar_tma = smem_u32(&bars[0]), bar_mma = smem_u32(&bars[1]);
+
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"((uint32_t)kTileN));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  if (tid == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_tma));
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar_mma));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = *tmem_slot;
+
+  if (tid == 0) {
+    const uint32_t tx = (uint32_t)(L::A_BYTES + L::S_BYTES);
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar_tma), "r"(tx) : "memory");
+    const int32_t qrow = (int32_t)((int64_t)seq * n_q + q0);
+#pragma unroll
+    for (int h = 0; h < L::HALVES; ++h) {
+      asm volatile(
+          "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+              "r"(smem_u32(sA + h * kTileM * 128)),
+          "l"(reinterpret_cast<uint64_t>(&tmap_q)), "r"(h * 64), "r"(qrow), "r"(bar_tma)
+          : "memory");
+    }
+    const int32_t brow = (int32_t)((int64_t)seq * n_blk + j0);
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            smem_u32(sS)),
+        "l"(reinterpret_cast<uint64_t>(&tmap_bk)), "r"(0), "r"(brow), "r"(bar_tma)
+        : "memory");
+  }
+  bool ok = mbar_wait(bar_tma, 0);
+  ok = __syncthreads_and(ok) != 0;
+
+  if (ok) {
+    // Split the fp32 block keys into three bf16 terms, each a K-major 128B-swizzled operand.
+    // Warp w converts rows w, w+4, ...; lane l handles dimensions 4l..4l+3 of each 128-wide slice.
+    for (int r = warp; r < kTileN; r += kTcThreads / 32) {
+#pragma unroll
+      for (int e0 = 0; e0 < D; e0 += 128) {
+        const int e = e0 + 4 * lane;
+        if (e >= D) break;
+        const float4 x = *reinterpret_cast<const float4*>(sS + r * D + e);
+        const float xs[4] = {x.x, x.y, x.z, x.w};
+        uint32_t t[3][2];
+#pragma unroll
+        for (int pr = 0; pr < 2; ++pr) {
+          uint32_t hb[2], mb[2], lb[2];
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const float v = xs[2 * pr + q];
+            hb[q] = bf16_bits(v);
+            const float r1 = v - __uint_as_float(hb[q] << 16);
+            mb[q] = bf16_bits(r1);
+            const float r2 = r1 - __uint_as_float(mb[q] << 16);
+            lb[q] = bf16_bits(r2);
+          }
+          t[0][pr] = hb[0] | (hb[1] << 16);
+          t[1][pr] = mb[0] | (mb[1] << 16);
+          t[2][pr] = lb[0] | (lb[1] << 16);
+        }
+        const int half = e / 64;
+        const int chunk = (e % 64) / 8;
+        const int within = (e % 8) * 2;  // bytes
+        const int off = half * kTileN * 128 + r * 128 + ((chunk ^ (r & 7)) * 16) + within;
+#pragma unroll
+        for (int pl = 0; pl < 3; ++pl)
+          *reinterpret_cast<uint2*>(sB + pl * L::B_PLANE + off) = make_uint2(t[pl][0], t[pl][1]);
+      }
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  __syncthreads();
+
+  if (ok && tid == 0) {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t a0 = smem_u32(sA), b0 = smem_u32(sB);
+    int first = 1;
+#pragma unroll
+    for (int pl = 0; pl < 3; ++pl) {
+#pragma unroll
+      for (int h = 0; h < L::HALVES; ++h) {
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+          const uint64_t ad = umma_desc_sw128(a0 + h * kTileM * 128 + s * 32);
+          const uint64_t bd = umma_desc_sw128(b0 + pl * L::B_PLANE + h * kTileN * 128 + s * 32);
+          const uint32_t acc = first ? 0u : 1u;
+          asm volatile(
+              "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+              " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem),
+              "l"(ad), "l"(bd), "r"(kIdesc), "r"(acc));
+          first = 0;
+        }
+      }
+    }
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar_mma)
+                 : "memory");
+  }
+  bool done = ok ? mbar_wait(bar_mma, 0) : false;
+  done = __syncthreads_and(done) != 0;
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  ok = done;
+
+  if (ok) {
+    const int64_t qi = q0 + warp * 32 + lane;  // this thread's query row within the sequence
+    const bool row_ok = qi < n_q;
+    const int64_t c = row_ok ? (n_kv - n_q + qi) / B : -1;
+    float* out = scores + ((int64_t)seq * n_q + qi) * n_blk;
+#pragma unroll
+    for (int cc = 0; cc < kTileN / 32; ++cc) {
+      uint32_t v[32];
+      const uint32_t addr = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(cc * 32);
+      asm volatile(
+          "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+          "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+          : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+            "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+            "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]),
+            "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]),
+            "=r"(v[30]), "=r"(v[31])
+          : "r"(addr));
+      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+      const int64_t jb = j0 + cc * 32;
+      if (row_ok && jb <= c) {
+        if (jb + 31 <= c) {
+#pragma unroll
+          for (int t = 0; t < 32; t += 4)
+            *reinterpret_cast<float4*>(out + jb + t) =
+                make_float4(__uint_as_float(v[t]), __uint_as_float(v[t + 1]), __uint_as_float(v[t + 2]),
+                            __uint_as_float(v[t + 3]));
+        } else {
+#pragma unroll
+          for (int t = 0; t < 32; ++t)
+            if (jb + t <= c) out[jb + t] = __uint_as_float(v[t]);
+        }
+      }
+    }
+  } else if (tid == 0 && status) {
+    atomicOr(status, kStatusTimeout);
+  }
+
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (warp == 0) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)kTileN));
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* base, uint64_t cols, uint64_t rows,
+                 uint32_t box_c, uint32_t box_r, CUtensorMapSwizzle sw) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * (uint64_t)esize};
+  cuuint32_t box[2] = {box_c, box_r};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D>
+cudaError_t launch_tc(const Shape& s, const void* q_idx, const float* bk, float* scores, int32_t* status,
+                      cudaStream_t st) {
+  using L = TcLayout<D>;
+  CUtensorMap mq, mb;
+  if (!make_map_2d(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q_idx, D, (uint64_t)s.n_query, 64, kTileM,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorNotSupported;
+  if (!make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, bk, D, (uint64_t)s.batch * s.n_blk, D, kTileN,
+                   CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorNotSupported;
+  auto kern = block_score_tc_kernel<D>;
+  cudaError_t e = ensure_smem((const void*)kern, L::SMEM);
+  if (e != cudaSuccess) return e;
+  const int q_tiles = (int)((s.n_q + kTileM - 1) / kTileM);
+  const int n_tiles = (int)((s.n_blk + kTileN - 1) / kTileN);
+  const int64_t grid = (int64_t)s.batch * q_tiles * n_tiles;
+  if (grid > 0x7FFFFFFFLL) return cudaErrorNotSupported;
+  kern<<<(unsigned)grid, kTcThreads, L::SMEM, st>>>(mq, mb, scores, status, s.n_q, s.n_kv, s.B, s.n_blk, q_tiles,
+                                                    n_tiles);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool block_score_tc_eligible(const Shape& s) {
+  if (true) return false;  // enabled once verified on the device
+  return (s.d_idx == 64 || s.d_idx == 128) && s.n_q >= 64 && s.n_query <= 0x7FFFFFFFLL &&
+         (int64_t)s.batch * s.n_blk <= 0x7FFFFFFFLL;
+}
+
+size_t block_score_tc_scratch_bytes(const Shape&) { return 0; }
+
+cudaError_t launch_block_score_tc(const Shape& s, const void* q_idx, const float* block_keys, float* scores,
+                                  int32_t* status, cudaStream_t st) {
+  if (!block_score_tc_eligible(s)) return cudaErrorNotSupported;
+  switch (s.d_idx) {
+    case 64: return launch_tc<64>(s, q_idx, block_keys, scores, status, st);
+    case 128: return launch_tc<128>(s, q_idx, block_keys, scores, status, st);
+    default: return cudaErrorNotSupported;
+  }
+}
+
+}  // namespace hisa

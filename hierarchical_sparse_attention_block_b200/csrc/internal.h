@@ -1,0 +1,56 @@
+// Launchers shared between the C-ABI layer (api.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace hisa {
+
+// Validated problem shape (see hisa_params_t in hisa.h).
+struct Shape {
+  int batch;
+  int64_t n_q, n_kv;
+  int d_idx, B, m, k, H, Hkv, d;
+  float scale;      // softmax scale, already resolved
+  int64_t n_blk;    // ceil(n_kv / B)
+  int64_t n_query;  // batch * n_q
+};
+
+// Step 1: block means for blocks [b0, b1) of every sequence.
+cudaError_t launch_block_pool(const Shape& s, const void* k_idx, int64_t b0, int64_t b1, float* block_keys,
+                              cudaStream_t st);
+
+// Step 2 (CUDA cores): scores[q][j] = q_idx[q] . block_keys[j] for j <= own block.
+cudaError_t launch_block_score(const Shape& s, const void* q_idx, const float* block_keys, float* scores,
+                               cudaStream_t st);
+
+// Step 2 on the tensor cores (prefill): same output as launch_block_score.
+// Returns cudaErrorNotSupported when the shape is outside the kernel's range.
+// status (nullable): bit 1 is set if a bounded wait timed out.
+cudaError_t launch_block_score_tc(const Shape& s, const void* q_idx, const float* block_keys, float* scores,
+                                  int32_t* status, cudaStream_t st);
+size_t block_score_tc_scratch_bytes(const Shape& s);
+bool block_score_tc_eligible(const Shape& s);
+
+// Step 3: block_idx from scores.
+cudaError_t launch_block_topm(const Shape& s, const float* scores, int32_t* block_idx, float* block_scores,
+                              cudaStream_t st);
+
+// Steps 4-5 over queries [q0, q0 + nq) (global query ids).  `slots` is the
+// number of block slots per query: m with a block list, n_blk for the flat
+// indexer (block_idx == nullptr: slot r is block r).  keys: [nq][slots * B].
+cudaError_t launch_token_score(const Shape& s, const void* q_idx, const void* k_idx, const int32_t* block_idx,
+                               int slots, uint32_t* keys, int32_t* status, int64_t q0, int64_t nq, cudaStream_t st);
+cudaError_t launch_token_select(const Shape& s, const uint32_t* keys, const int32_t* block_idx, int slots,
+                                int32_t* token_idx, float* token_scores, int64_t q0, int64_t nq, cudaStream_t st);
+
+// Step 6.  splits > 1 needs partial buffers of attn_partial_bytes(s, splits).
+int attn_pick_splits(const Shape& s);
+size_t attn_partial_bytes(const Shape& s, int splits);
+cudaError_t launch_sparse_attn(const Shape& s, const void* q, const void* k, const void* v, const int32_t* token_idx,
+                               void* o, float* lse, int32_t* status, int splits, void* partial, cudaStream_t st);
+
+// Dynamic shared memory opt-in, once per (kernel, device).
+cudaError_t ensure_smem(const void* func, int bytes);
+
+}  // namespace hisa

@@ -1,0 +1,223 @@
+// Steps 4-5: score the query against the tokens of its kept blocks and keep
+// the top k.  "北大HISA稀疏注意力机制" section 1.2.2 items 1-2; QbitAI HISA
+// article, "塊內精挑字符".  The flat indexer (every block is a slot) uses the
+// same two kernels, which keeps the speed comparison like for like.
+//
+// token_score_kernel: one CTA per (query, run of slots).  A kept block is one
+// contiguous B x d_idx tile of k_idx; 8 lanes share a token row (16-byte
+// loads, each lane 8*d_idx/64 dimensions), several rows in flight per lane,
+// fp32 FMA, 3-step shuffle reduction.  Each candidate's score is written as
+// an order-preserving u32 key at [slot * B + offset] of the query's row;
+// positions past the query or in unused slots get key 0 ("empty").
+//
+// token_select_kernel: one CTA per query; the row of keys is staged in shared
+// memory (when it fits) and a CTA radix selection takes the best
+// min(k, candidates), emitted in ascending token order.
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+#include "select.cuh"
+
+namespace hisa {
+namespace {
+
+constexpr int kScoreThreads = 256;
+constexpr int kMaxSlotsPerCta = 64;
+constexpr int kSelectThreads = 256;
+constexpr int kSelectSmemKeys = 49152;  // 192 KiB of keys
+
+template <int D>
+__global__ void __launch_bounds__(kScoreThreads)
+    token_score_kernel(const uint16_t* __restrict__ q_idx, const uint16_t* __restrict__ k_idx,
+                       const int32_t* __restrict__ block_idx, int slots, uint32_t* __restrict__ keys,
+                       int32_t* __restrict__ status, int64_t n_q, int64_t n_kv, int B, int spc, int chunks,
+                       int64_t q0) {
+  constexpr int CPL = D / 64;  // 16-byte chunks per lane
+  constexpr int U = 4;         // token rows in flight per lane group
+  __shared__ int s_blk[kMaxSlotsPerCta];
+  __shared__ int s_len[kMaxSlotsPerCta];
+
+  const int64_t lq = blockIdx.x / chunks;
+  const int chunk = blockIdx.x % chunks;
+  const int64_t qg = q0 + lq;
+  const int seq = (int)(qg / n_q);
+  const int64_t p = n_kv - n_q + qg % n_q;
+  const int64_t c = p / B;
+  const int r0 = chunk * spc;
+  const int nr = min(spc, slots - r0);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+
+  // Which slots are usable: an entry is used if it lies in [0, c] and is
+  // greater than every in-range entry before it (ascending, no repeats).
+  for (int rr = warp; rr < nr; rr += kScoreThreads / 32) {
+    const int r = r0 + rr;
+    int blk;
+    bool ok;
+    if (block_idx) {
+      const int32_t* row = block_idx + qg * slots;
+      blk = row[r];
+      int mx = -1;
+      for (int t = lane; t < r; t += 32) {
+        const int v = row[t];
+        if (v >= 0 && v <= c) mx = max(mx, v);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+      ok = blk >= 0 && blk <= c && blk > mx;
+      if (!ok && blk != -1 && lane == 0 && status) atomicOr(status, kStatusBadIndex);
+    } else {
+      blk = r;
+      ok = r <= c;
+    }
+    if (lane == 0) {
+      s_blk[rr] = ok ? blk : -1;
+      s_len[rr] = ok ? visible_len(blk, B, p) : 0;
+    }
+  }
+
+  // This thread's share of the query: chunks sub + 8u of the row.
+  const int grp = threadIdx.x >> 3, sub = threadIdx.x & 7;
+  const unsigned gmask = 0xFFu << (lane & ~7);
+  float qf[8 * CPL];
+  const uint16_t* qrow = q_idx + qg * D;
+#pragma unroll
+  for (int u = 0; u < CPL; ++u) {
+    const uint4 w = *reinterpret_cast<const uint4*>(qrow + (sub + 8 * u) * 8);
+    qf[8 * u + 0] = bf16_lo(w.x); qf[8 * u + 1] = bf16_hi(w.x);
+    qf[8 * u + 2] = bf16_lo(w.y); qf[8 * u + 3] = bf16_hi(w.y);
+    qf[8 * u + 4] = bf16_lo(w.z); qf[8 * u + 5] = bf16_hi(w.z);
+    qf[8 * u + 6] = bf16_lo(w.w); qf[8 * u + 7] = bf16_hi(w.w);
+  }
+  __syncthreads();
+
+  constexpr int NG = kScoreThreads / 8;  // token rows per CTA step
+  uint32_t* krow = keys + lq * (int64_t)slots * B;
+  for (int rr = 0; rr < nr; ++rr) {
+    const int blk = s_blk[rr], len = s_len[rr];
+    const uint16_t* kb = k_idx + ((int64_t)seq * n_kv + (int64_t)(blk < 0 ? 0 : blk) * B) * D + sub * 8;
+    uint32_t* dst = krow + (int64_t)(r0 + rr) * B;
+    for (int o0 = grp; o0 < B; o0 += NG * U) {
+      uint4 v[U][CPL];
+#pragma unroll
+      for (int j = 0; j < U; ++j) {
+        const int o = o0 + j * NG;
+#pragma unroll
+        for (int u = 0; u < CPL; ++u)
+          v[j][u] = o < len ? ld_nc_v4(kb + (int64_t)o * D + u * 64) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int j = 0; j < U; ++j) {
+        const int o = o0 + j * NG;
+        float dot = 0.f;
+#pragma unroll
+        for (int u = 0; u < CPL; ++u) {
+          const float* qq = qf + 8 * u;
+          dot = fmaf(qq[0], bf16_lo(v[j][u].x), dot); dot = fmaf(qq[1], bf16_hi(v[j][u].x), dot);
+          dot = fmaf(qq[2], bf16_lo(v[j][u].y), dot); dot = fmaf(qq[3], bf16_hi(v[j][u].y), dot);
+          dot = fmaf(qq[4], bf16_lo(v[j][u].z), dot); dot = fmaf(qq[5], bf16_hi(v[j][u].z), dot);
+          dot = fmaf(qq[6], bf16_lo(v[j][u].w), dot); dot = fmaf(qq[7], bf16_hi(v[j][u].w), dot);
+        }
+        dot += __shfl_xor_sync(gmask, dot, 4);
+        dot += __shfl_xor_sync(gmask, dot, 2);
+        dot += __shfl_xor_sync(gmask, dot, 1);
+        if (sub == 0 && o < B) dst[o] = o < len ? score_key(dot) : 0u;
+      }
+    }
+  }
+}
+
+template <int NT>
+__global__ void __launch_bounds__(NT)
+    token_select_kernel(const uint32_t* __restrict__ keys, const int32_t* __restrict__ block_idx, int slots,
+                        int32_t* __restrict__ token_idx, float* __restrict__ token_scores, int64_t n_q, int log2B,
+                        int k, int64_t q0, int keys_in_smem) {
+  __shared__ SelectShared<NT> sm;
+  extern __shared__ __align__(16) uint32_t dsm[];
+  const int B = 1 << log2B;
+  const int64_t lq = blockIdx.x;
+  const int64_t qg = q0 + lq;
+  const int n = slots * B;
+  const uint32_t* row = keys + lq * (int64_t)n;
+  uint32_t* skeys = dsm;
+  int32_t* sblk = reinterpret_cast<int32_t*>(dsm + (keys_in_smem ? n : 0));
+
+  for (int r = threadIdx.x; r < slots; r += NT) sblk[r] = block_idx ? block_idx[qg * slots + r] : r;
+  if (keys_in_smem) {
+    if ((n & 3) == 0) {
+      const uint4* src = reinterpret_cast<const uint4*>(row);
+      uint4* dst = reinterpret_cast<uint4*>(skeys);
+      for (int i = threadIdx.x; i < n / 4; i += NT) dst[i] = src[i];
+    } else {
+      for (int i = threadIdx.x; i < n; i += NT) skeys[i] = row[i];
+    }
+  }
+  __syncthreads();
+  auto key = [&](int i) -> uint32_t { return keys_in_smem ? skeys[i] : row[i]; };
+  const int nv = count_nonzero<NT>(key, n, sm);
+  const int K = min(k, nv);
+  int32_t* out = token_idx + qg * k;
+  float* osc = token_scores ? token_scores + qg * k : nullptr;
+  if (K > 0) {
+    const SelectResult r = (K == nv) ? select_all_nonzero() : radix_select<NT>(key, n, K, sm);
+    emit_selected<NT>(key, n, r, sm, [&](int i, int rank) {
+      const int slot = i >> log2B;
+      out[rank] = sblk[slot] * B + (i & (B - 1));
+      if (osc) osc[rank] = key_score(key(i));
+    });
+  }
+  for (int r = K + threadIdx.x; r < k; r += NT) {
+    out[r] = -1;
+    if (osc) osc[r] = __int_as_float(0x7FC00000);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_token_score(const Shape& s, const void* q_idx, const void* k_idx, const int32_t* block_idx,
+                               int slots, uint32_t* keys, int32_t* status, int64_t q0, int64_t nq, cudaStream_t st) {
+  if (nq <= 0) return cudaSuccess;
+  int spc = 1024 / s.B;
+  spc = spc < 1 ? 1 : (spc > kMaxSlotsPerCta ? kMaxSlotsPerCta : spc);
+  if (spc > slots) spc = slots;
+  const int chunks = (slots + spc - 1) / spc;
+  const int64_t grid = nq * chunks;
+  if (grid > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
+  const uint16_t* qp = static_cast<const uint16_t*>(q_idx);
+  const uint16_t* kp = static_cast<const uint16_t*>(k_idx);
+  switch (s.d_idx) {
+    case 64:
+      token_score_kernel<64><<<(unsigned)grid, kScoreThreads, 0, st>>>(qp, kp, block_idx, slots, keys, status, s.n_q,
+                                                                       s.n_kv, s.B, spc, chunks, q0);
+      break;
+    case 128:
+      token_score_kernel<128><<<(unsigned)grid, kScoreThreads, 0, st>>>(qp, kp, block_idx, slots, keys, status, s.n_q,
+                                                                        s.n_kv, s.B, spc, chunks, q0);
+      break;
+    case 256:
+      token_score_kernel<256><<<(unsigned)grid, kScoreThreads, 0, st>>>(qp, kp, block_idx, slots, keys, status, s.n_q,
+                                                                        s.n_kv, s.B, spc, chunks, q0);
+      break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_token_select(const Shape& s, const uint32_t* keys, const int32_t* block_idx, int slots,
+                                int32_t* token_idx, float* token_scores, int64_t q0, int64_t nq, cudaStream_t st) {
+  if (nq <= 0) return cudaSuccess;
+  const int64_t n = (int64_t)slots * s.B;
+  const int in_smem = n <= kSelectSmemKeys ? 1 : 0;
+  const int smem = (int)((in_smem ? n : 0) * 4 + (int64_t)slots * 4);
+  if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
+  int log2B = 0;
+  while ((1 << log2B) < s.B) ++log2B;
+  auto kern = token_select_kernel<kSelectThreads>;
+  cudaError_t e = ensure_smem((const void*)kern, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<(unsigned)nq, kSelectThreads, smem, st>>>(keys, block_idx, slots, token_idx, token_scores, s.n_q, log2B, s.k,
+                                                   q0, in_smem);
+  return cudaGetLastError();
+}
+
+}  // namespace hisa

@@ -1,0 +1,169 @@
+/*
+ * hisa.h -- C ABI of the two-level (block -> token) sparse-attention indexer
+ * and of the sparse attention that consumes its output, for NVIDIA B200
+ * (sm_100a).
+ *
+ * The method (sources cited by short key):
+ *   [IP] "北大HISA稀疏注意力机制：长文本处理效率提升3倍" (intelliparadigm.com):
+ *        section 1.2.1 "块级粗过滤" (coarse block filtering), section 1.2.2
+ *        "块内精筛选" (fine token selection), section 3.2 (block sizes 64/128/256).
+ *   [QB] QbitAI article on HISA (m.digipub.cc, KPSAJS2O0511DSSR): sections
+ *        "塊級粗過濾", "塊內精挑字符" and "HISA的關鍵優勢在於" (cost
+ *        O(L^2/B + L*m*B); output format and attention unchanged).
+ *
+ *   1. cut each sequence's indexer keys into blocks of B tokens and mean-pool
+ *      every block into one block key;
+ *   2. score each query against the block keys it can see (dot product);
+ *   3. keep m blocks: block 0, the query's own block c = floor(p/B), and the
+ *      m-2 best of blocks 1..c-1 (all visible blocks when c+1 <= m);
+ *   4. score the query against the tokens t <= p of those blocks;
+ *   5. keep the k best tokens (ties: lower index first);
+ *   6. softmax attention of every head over just those tokens.
+ *
+ * Conventions shared by every call
+ *   - Tensors are dense, row-major, in DEVICE memory, owned by the caller.
+ *     The library allocates nothing; calls that need scratch take a caller
+ *     workspace whose size the matching *_workspace_size call reports.
+ *   - bf16 tensors are passed as void* (__nv_bfloat16 elements).  Base
+ *     pointers must be 16-byte aligned.
+ *   - Shapes (b = batch, H = n_heads, Hk = n_kv_heads, d = d_head):
+ *       q_idx  [b][n_q][d_idx]  bf16     k_idx   [b][n_kv][d_idx] bf16
+ *       block_keys [b][ceil(n_kv/B)][d_idx] fp32
+ *       block_idx  [b][n_q][m]  int32    token_idx [b][n_q][k] int32
+ *       q [b][n_q][H][d] bf16   k, v [b][n_kv][Hk][d] bf16
+ *       o [b][n_q][H][d] bf16   lse [b][n_q][H] fp32 (natural log)
+ *     Query i of a sequence sits at position p_i = n_kv - n_q + i
+ *     (prefill: n_q = n_kv; decode: n_q = 1, p = n_kv - 1).
+ *   - Index lists are ascending with -1 padding at the tail.  Ties in a
+ *     selection go to the lower block / token index.
+ *   - Every call validates its arguments on the host before launching
+ *     anything (HISA_ERR_INVALID_ARG / HISA_ERR_UNSUPPORTED /
+ *     HISA_ERR_WORKSPACE) and then only enqueues work on `stream`; results
+ *     are ready when the stream reaches them.  A launch failure returns
+ *     HISA_ERR_CUDA; hisa_last_cuda_error() gives the cudaError_t value.
+ *   - Index lists given as INPUT are checked on the device: an entry that is
+ *     out of range (below -1, beyond the query's own block / position, or not
+ *     greater than every in-range entry before it) is skipped, never
+ *     dereferenced, and bit 0 of *dev_status is set (atomicOr).  No kernel
+ *     traps or waits unboundedly: a wait that runs out (1 s) sets bit 1 of
+ *     *dev_status and the results of that call are not valid.
+ *   - Supported sizes: d_idx in {64, 128, 256}; d_head in {64, 128}; B a
+ *     power of two in [1, 4096]; m >= 2; k >= 1; n_heads a multiple of
+ *     n_kv_heads; n_kv < 2^31.  Integer-valued indexer inputs (|x| <= 4)
+ *     make every block mean and score exact in fp32, so selections are exact.
+ */
+#ifndef HISA_H
+#define HISA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum hisa_status {
+  HISA_OK = 0,
+  HISA_ERR_INVALID_ARG = 1, /* null pointer, bad shape, misaligned pointer */
+  HISA_ERR_UNSUPPORTED = 2, /* valid request outside the sizes listed above */
+  HISA_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required */
+  HISA_ERR_CUDA = 4         /* a CUDA call failed; see hisa_last_cuda_error() */
+} hisa_status_t;
+
+/* Problem description.  scale <= 0 selects 1/sqrt(d_head).  flags must be 0. */
+typedef struct hisa_params {
+  int32_t batch;      /* b: independent sequences of equal length */
+  int32_t d_idx;      /* indexer head dimension */
+  int64_t n_q;        /* queries per sequence: the last n_q positions */
+  int64_t n_kv;       /* keys per sequence */
+  int32_t block;      /* B: tokens per block */
+  int32_t top_m;      /* m: blocks kept per query (forced blocks included) */
+  int32_t top_k;      /* k: tokens kept per query */
+  int32_t n_heads;    /* H: attention query heads */
+  int32_t n_kv_heads; /* Hk: attention key/value heads (H % Hk == 0) */
+  int32_t d_head;     /* d: attention head dimension */
+  float scale;        /* softmax scale tau */
+  int32_t flags;      /* reserved, 0 */
+} hisa_params_t;
+
+/* Step 1 -- [IP] 1.2.1 item 1; [QB] "塊級粗過濾" bullet 1.
+ * block_keys[s][j][:] = mean of k_idx[s][t][:] over the tokens t of block j
+ * (B of them, fewer in a final partial block), fp32, for blocks
+ * j in [blk_begin, blk_end) of every sequence; blk_end < 0 means the last
+ * block.  Other rows of block_keys are left untouched, so a decode loop can
+ * refresh only the newest block. */
+hisa_status_t hisa_block_pool(const hisa_params_t* params, const void* k_idx, int64_t blk_begin,
+                              int64_t blk_end, float* block_keys, cudaStream_t stream);
+
+/* Steps 2-3 -- [IP] 1.2.1 items 2-3; [QB] "塊級粗過濾" bullets 2-3 and the
+ * forced first/last block remark of "塊內精挑字符".
+ * block_idx[s][i][0..m): the min(m, c+1) kept blocks, ascending, -1 padded.
+ * block_scores (nullable) [b][n_q][m] fp32: q . block_key of each kept block
+ * (NaN for padding).  dev_status (nullable): see conventions.  Workspace:
+ * hisa_block_topm_workspace_size bytes.  With many queries per sequence the
+ * scores come from a tcgen05 tensor-core kernel that splits each fp32 block
+ * key into three bf16 terms (fp32-faithful; exact on integer inputs), with
+ * few queries from a CUDA-core kernel. */
+hisa_status_t hisa_block_topm_workspace_size(const hisa_params_t* params, size_t* bytes);
+hisa_status_t hisa_block_topm(const hisa_params_t* params, const void* q_idx, const float* block_keys,
+                              int32_t* block_idx, float* block_scores, int32_t* dev_status, void* workspace,
+                              size_t workspace_bytes, cudaStream_t stream);
+
+/* Steps 4-5 -- [IP] 1.2.2 items 1-2; [QB] "塊內精挑字符".
+ * token_idx[s][i][0..k): the min(k, candidates) best tokens t <= p_i of the
+ * blocks in block_idx[s][i], ascending, -1 padded.  token_scores (nullable)
+ * [b][n_q][k] fp32: their indexer scores (NaN for padding).  dev_status
+ * (nullable) int32 on the device, see conventions.  Any workspace of at least
+ * the reported minimum works; more lets more queries run per launch. */
+hisa_status_t hisa_token_topk_workspace_size(const hisa_params_t* params, size_t* min_bytes,
+                                             size_t* preferred_bytes);
+hisa_status_t hisa_token_topk(const hisa_params_t* params, const void* q_idx, const void* k_idx,
+                              const int32_t* block_idx, int32_t* token_idx, float* token_scores,
+                              int32_t* dev_status, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Step 6 -- [QB] "HISA的關鍵優勢在於" (the downstream attention is unchanged).
+ * For every query i and head h (kv head g = h / (H / Hk)):
+ *   o[s][i][h]   = sum_t softmax_t(scale * q[s][i][h] . k[s][t][g]) v[s][t][g]
+ *   lse[s][i][h] = ln sum_t exp(scale * q[s][i][h] . k[s][t][g])
+ * over the entries t of token_idx[s][i] (-1 skipped).  bf16 inputs, fp32
+ * accumulation, bf16 output.  An empty list gives o = 0, lse = -inf.
+ * lse and dev_status are nullable.  Workspace may be NULL (then every
+ * query/head is one work item); with hisa_sparse_attn_workspace_size bytes the
+ * token list is split across CTAs when there are few queries (decode). */
+hisa_status_t hisa_sparse_attn_workspace_size(const hisa_params_t* params, size_t* bytes);
+hisa_status_t sparse_attn_fwd(const hisa_params_t* params, const void* q, const void* k, const void* v,
+                              const int32_t* token_idx, void* o, float* lse, int32_t* dev_status, void* workspace,
+                              size_t workspace_bytes, cudaStream_t stream);
+
+/* Steps 1-6 in one call.  block_idx_out and token_idx_out (nullable) receive
+ * the intermediate selections.  Workspace: hisa_forward_workspace_size. */
+hisa_status_t hisa_forward_workspace_size(const hisa_params_t* params, size_t* bytes);
+hisa_status_t hisa_forward(const hisa_params_t* params, const void* q_idx, const void* k_idx, const void* q,
+                           const void* k, const void* v, void* o, float* lse, int32_t* block_idx_out,
+                           int32_t* token_idx_out, int32_t* dev_status, void* workspace, size_t workspace_bytes,
+                           cudaStream_t stream);
+
+/* The flat token indexer the two-level one replaces ([IP] 1.1 item 1; [QB]
+ * "兩步消除上下文索引瓶頸"): token_idx[s][i] = the min(k, p_i+1) best tokens
+ * t <= p_i of the whole sequence.  Same output format as hisa_token_topk;
+ * used as the speed comparator and for the degeneration check. */
+hisa_status_t hisa_flat_topk_workspace_size(const hisa_params_t* params, size_t* min_bytes,
+                                            size_t* preferred_bytes);
+hisa_status_t hisa_flat_topk(const hisa_params_t* params, const void* q_idx, const void* k_idx,
+                             int32_t* token_idx, float* token_scores, void* workspace, size_t workspace_bytes,
+                             cudaStream_t stream);
+
+/* Static text for a status code. */
+const char* hisa_status_string(hisa_status_t status);
+/* cudaError_t value of the last failed CUDA call on this host thread (0 if none). */
+int32_t hisa_last_cuda_error(void);
+/* Library version string. */
+const char* hisa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HISA_H */

@@ -1,0 +1,120 @@
+"""The C-ABI library without a GPU: every declared symbol is exported, and the host-side
+validation rejects bad arguments before anything is launched."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import hierarchical_sparse_attention_block_b200 as hs
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hisa.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:hisa_status_t|const char\*|int32_t)\s+(\w+)\s*\(", text, re.M)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert len(names) >= 14, names
+    lib = ctypes.CDLL(hs.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(hs.EXPORTS)
+
+
+def test_status_strings_and_version():
+    lib = hs.lib()
+    for code in range(5):
+        assert lib.hisa_status_string(code)
+    assert hs.hisa_version().startswith("hisa-b200")
+    assert lib.hisa_last_cuda_error() == 0
+
+
+def _p(**kw):
+    base = dict(batch=1, n_q=1024, n_kv=1024, d_idx=64, block=64, top_m=4, top_k=128, n_heads=1, d_head=64)
+    base.update(kw)
+    return hs.params(**base)
+
+
+def _ws(fn, p):
+    n = ctypes.c_size_t(0)
+    return fn(ctypes.byref(p), ctypes.byref(n)), n.value
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(n_q=2048), hs.HISA_ERR_INVALID_ARG),        # more queries than keys
+    (dict(n_q=0), hs.HISA_ERR_INVALID_ARG),
+    (dict(batch=0), hs.HISA_ERR_INVALID_ARG),
+    (dict(block=48), hs.HISA_ERR_UNSUPPORTED),        # not a power of two
+    (dict(block=0), hs.HISA_ERR_INVALID_ARG),
+    (dict(d_idx=96), hs.HISA_ERR_UNSUPPORTED),
+    (dict(top_m=1), hs.HISA_ERR_INVALID_ARG),         # the two forced blocks need m >= 2
+    (dict(top_k=0), hs.HISA_ERR_INVALID_ARG),
+])
+def test_indexer_validation(kw, code):
+    rc, _ = _ws(hs.lib().hisa_block_topm_workspace_size, _p(**kw))
+    assert rc == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(n_heads=3, n_kv_heads=2), hs.HISA_ERR_INVALID_ARG),
+    (dict(d_head=96), hs.HISA_ERR_UNSUPPORTED),
+    (dict(scale=float("nan")), hs.HISA_ERR_INVALID_ARG),
+])
+def test_attention_validation(kw, code):
+    rc, _ = _ws(hs.lib().hisa_sparse_attn_workspace_size, _p(**kw))
+    assert rc == code
+
+
+def test_flags_must_be_zero():
+    p = _p()
+    p.flags = 1
+    rc, _ = _ws(hs.lib().hisa_forward_workspace_size, p)
+    assert rc == hs.HISA_ERR_INVALID_ARG
+
+
+def test_null_and_misaligned_pointers_rejected_before_launch():
+    lib = hs.lib()
+    p = _p()
+    assert lib.hisa_block_pool(None, ctypes.c_void_p(256), 0, -1, ctypes.c_void_p(512), None) == hs.HISA_ERR_INVALID_ARG
+    assert lib.hisa_block_pool(ctypes.byref(p), None, 0, -1, ctypes.c_void_p(512), None) == hs.HISA_ERR_INVALID_ARG
+    assert lib.hisa_block_pool(ctypes.byref(p), ctypes.c_void_p(258), 0, -1, ctypes.c_void_p(512),
+                               None) == hs.HISA_ERR_INVALID_ARG
+    # block range outside [0, n_blk]
+    assert lib.hisa_block_pool(ctypes.byref(p), ctypes.c_void_p(256), 3, 2, ctypes.c_void_p(512),
+                               None) == hs.HISA_ERR_INVALID_ARG
+    assert lib.hisa_block_pool(ctypes.byref(p), ctypes.c_void_p(256), 0, 17, ctypes.c_void_p(512),
+                               None) == hs.HISA_ERR_INVALID_ARG
+
+
+def test_workspace_checks_before_launch():
+    lib = hs.lib()
+    p = _p()
+    a = ctypes.c_void_p(4096)
+    need = hs.hisa_block_topm_workspace_size(p)
+    assert need >= 1024 * 16 * 4
+    assert lib.hisa_block_topm(ctypes.byref(p), a, a, a, None, None, a, need - 1, None) == hs.HISA_ERR_WORKSPACE
+    assert lib.hisa_block_topm(ctypes.byref(p), a, a, a, None, None, None, need, None) == hs.HISA_ERR_WORKSPACE
+    mn, pref = hs.hisa_token_topk_workspace_size(p)
+    assert mn == p.top_m * p.block * 4 and pref == mn * p.n_q
+    assert lib.hisa_token_topk(ctypes.byref(p), a, a, a, a, None, None, a, mn - 4, None) == hs.HISA_ERR_WORKSPACE
+    fmin, fpref = hs.hisa_flat_topk_workspace_size(p)
+    assert fmin == 16 * 64 * 4
+    need_f = hs.hisa_forward_workspace_size(p)
+    assert lib.hisa_forward(ctypes.byref(p), a, a, a, a, a, a, None, None, None, None, a, need_f - 1,
+                            None) == hs.HISA_ERR_WORKSPACE
+
+
+def test_workspace_sizes_follow_the_shapes():
+    # decode: 32 sequences x 128K keys, m = 64, k = 2048, 16 heads
+    p = hs.params(32, 1, 131072, 128, 128, 64, 2048, 16, 16, 128)
+    mn, pref = hs.hisa_token_topk_workspace_size(p)
+    assert mn == 64 * 128 * 4 and pref == 32 * mn
+    # the attention list is split across CTAs when there are few queries
+    assert hs.hisa_sparse_attn_workspace_size(p) > 0
+    big = hs.params(1, 65536, 65536, 128, 128, 64, 2048, 16, 16, 128)
+    assert hs.hisa_sparse_attn_workspace_size(big) == 0
