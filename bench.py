@@ -45,8 +45,24 @@ def _args():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-flat", action="store_true", help="skip the flat-indexer comparator")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
+    ap.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE",
+                    help="override a workload field, e.g. --set n_q=32768 --set n_kv=32768")
     return ap.parse_args()
+
+
+def workload(a, seed_offset=0):
+    from synth.workloads import WORKLOADS
+
+    w = WORKLOADS[a.workload]
+    kw = {}
+    for item in a.set:
+        k, v = item.split("=", 1)
+        kw[k] = int(v)
+    if kw:
+        w = w.with_(name=w.name + "+" + ",".join(f"{k}={v}" for k, v in kw.items()), **kw)
+    return w.with_(seed=w.seed + seed_offset)
 
 
 def _peaks():
@@ -114,6 +130,23 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def max_over_ranks(value: float, device=None) -> float:
+    """The largest of one float over all ranks (the job's time is the slowest rank's)."""
+    import torch
+    import torch.distributed as dist
+
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(queries_per_rank: int, world: int, max_ms: float) -> float:
+    """Weak scaling: every rank runs its own copy, so the job processes world x the queries."""
+    return queries_per_rank * world / (max_ms * 1e-3)
+
+
 def closed_form_counts(w):
     """Per-query candidate counts and kept tokens from the closed forms of the path."""
     import numpy as np
@@ -164,11 +197,9 @@ def run_ours(a, rank, world, local_rank):
 
     import hierarchical_sparse_attention_block_b200 as hs
     import synth.device as sd
-    from synth.workloads import WORKLOADS
-
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = WORKLOADS[a.workload].with_(seed=WORKLOADS[a.workload].seed + rank)
+    w = workload(a, rank)
     p = hs.params_of(w)
     inp = sd.device_inputs(w, device=dev)
     torch.cuda.synchronize()
@@ -212,7 +243,7 @@ def run_ours(a, rank, world, local_rank):
 
     # the indexer alone and the flat comparator, for the speedup figure (outside the timed steps)
     comp = {}
-    if world == 1:
+    if world == 1 and not a.no_flat:
         flat_tok = torch.empty_like(tok)
         fmin, fpref = hs.hisa_flat_topk_workspace_size(p)
         ws_flat = torch.empty(fpref, dtype=torch.uint8, device=dev)
@@ -254,10 +285,7 @@ def run_ours(a, rank, world, local_rank):
         step_ms.append(ev[0].elapsed_time(ev[4]))
     ms = sum(step_ms) / len(step_ms)
     region_ms = g0.elapsed_time(g1)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dev)
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} in the timed steps")
 
@@ -276,7 +304,7 @@ def run_ours(a, rank, world, local_rank):
     launches = 3 + 2 * n_chunks + (1 if splits == 1 else 2)
 
     result = {
-        "metric": METRIC, "value": nq * world / (ms * 1e-3), "unit": UNIT, "n_gpus": world, "steps": a.steps,
+        "metric": METRIC, "value": job_value(nq, world, ms), "unit": UNIT, "n_gpus": world, "steps": a.steps,
         "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded SplitMix64; integer indexer q/k in [-4,4], unit-variance "
                                   "Irwin-Hall Q/K/V, planted needle blocks)",
@@ -343,13 +371,9 @@ def run_e2e(a, hs, w, p, inp, dev, st, world):
         one()
     e1.record(st)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / steps
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, dev)
     del host, d_in, ws
-    return {"value": w.batch * w.n_q * world / (ms * 1e-3), "unit": UNIT, "ms_per_step": ms,
+    return {"value": job_value(w.batch * w.n_q, world, ms), "unit": UNIT, "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
 
 
@@ -405,9 +429,7 @@ def main():
 
     if a.impl == "reference":
         if rank == 0:
-            from synth.workloads import WORKLOADS
-
-            w = WORKLOADS[a.workload]
+            w = workload(a)
             cpu = oracle_sample(w, a.cpu_seconds * max(1, a.steps) / 10.0)
             line = {"impl": "reference", "metric": METRIC, "value": cpu["value"], "unit": UNIT, "n_gpus": world,
                     "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * w.batch * w.n_q / cpu["value"],
@@ -427,9 +449,8 @@ def main():
     res = run_ours(a, rank, world, local_rank)
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         import synth.device as sd
-        from synth.workloads import WORKLOADS
 
-        w = WORKLOADS[a.workload]
+        w = workload(a)
         small = w.batch * w.n_q <= 8192
         dev_inp = None if small else sd.device_inputs(w, device=torch.device("cuda", local_rank))
         res["cpu_baseline"] = oracle_sample(w, a.cpu_seconds, dev_inp)

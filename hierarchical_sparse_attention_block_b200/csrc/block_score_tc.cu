@@ -245,7 +245,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
       const int64_t jb = j0 + cc * 32;
       if (row_ok && jb <= c) {
-        if (jb + 31 <= c) {
+        if (jb + 31 <= c && (n_blk & 3) == 0) {  // 16-byte aligned rows only
 #pragma unroll
           for (int t = 0; t < 32; t += 4)
             *reinterpret_cast<float4*>(out + jb + t) =
@@ -320,7 +320,6 @@ cudaError_t launch_tc(const Shape& s, const void* q_idx, const float* bk, float*
 }  // namespace
 
 bool block_score_tc_eligible(const Shape& s) {
-  if (true) return false;  // enabled once verified on the device
   return (s.d_idx == 64 || s.d_idx == 128) && s.n_q >= 64 && s.n_query <= 0x7FFFFFFFLL &&
          (int64_t)s.batch * s.n_blk <= 0x7FFFFFFFLL;
 }

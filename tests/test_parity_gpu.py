@@ -71,6 +71,18 @@ def test_stages_match_oracle(hs, oracle_lib, w):
     o = got["o"].float().cpu().numpy().reshape(n, w.n_heads, w.d_head)
     assert_close(o, ref["o"], "o")
     assert_close(got["lse"].cpu().numpy().reshape(n, w.n_heads), ref["lse"], "lse")
+    # block scores of the kept blocks: exact for full blocks (mean of integers over a
+    # power-of-two count), within fp32 rounding for a final partial block
+    bsc = got["block_scores"].cpu().numpy().reshape(n, w.top_m)
+    for r in range(0, n, max(1, n // 64)):
+        seq, i = divmod(r, w.n_q)
+        p = w.n_kv - w.n_q + i
+        sel, s_, sc = oracle_lib.block_topm(inp["q_idx"][seq, i], ref["block_keys"][seq], w.block, p, w.top_m,
+                                            scores=True)
+        full = (sel[:s_] + 1) * w.block <= w.n_kv
+        assert np.array_equal(bsc[r][:s_][full], sc[:s_][full].astype(np.float32)), r
+        assert np.allclose(bsc[r][:s_][~full], sc[:s_][~full], rtol=1e-5, atol=1e-4), r
+        assert np.all(np.isnan(bsc[r][s_:]))
 
 
 @pytest.mark.parametrize("w", SMALL[:3] + [WORKLOADS["prefill_8k"]], ids=lambda w: w.name)
