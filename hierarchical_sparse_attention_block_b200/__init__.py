@@ -23,7 +23,7 @@ EXPORTS = (
     "hisa_block_pool", "hisa_block_topm_workspace_size", "hisa_block_topm", "hisa_token_topk_workspace_size",
     "hisa_token_topk", "hisa_sparse_attn_workspace_size", "sparse_attn_fwd", "hisa_forward_workspace_size",
     "hisa_forward", "hisa_flat_topk_workspace_size", "hisa_flat_topk", "hisa_status_string",
-    "hisa_last_cuda_error", "hisa_version",
+    "hisa_last_cuda_error", "hisa_version", "hisa_token_topk_noalloc",
 )
 
 
@@ -50,7 +50,7 @@ class HisaError(RuntimeError):
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with "
-                          "`python -m hierarchical_sparse_attention_block_b200.build`")
+                          "`python hierarchical_sparse_attention_block_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     vp, i64, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.POINTER(ctypes.c_size_t)
     pp = ctypes.POINTER(HisaParams)
@@ -66,6 +66,7 @@ def _load():
         "hisa_forward": [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
         "hisa_flat_topk_workspace_size": [pp, sz, sz],
         "hisa_flat_topk": [pp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
+        "hisa_token_topk_noalloc": [pp, vp, vp, vp, vp, vp, vp, vp],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -200,6 +201,15 @@ def hisa_flat_topk(p, q_idx, k_idx, token_idx, token_scores=None, workspace=None
     _check("hisa_flat_topk", _lib.hisa_flat_topk(ctypes.byref(p), _ptr(q_idx), _ptr(k_idx), _ptr(token_idx),
                                                  _ptr(token_scores), _ptr(workspace), workspace.numel(),
                                                  _stream(stream)))
+
+
+def hisa_token_topk_noalloc(p, q_idx, k_idx, block_idx, token_idx, token_scores=None, dev_status=None,
+                            stream=None):
+    """hisa_token_topk for callers that cannot allocate: the library's fixed device scratch
+    array stands in for the workspace (see include/hisa.h)."""
+    _check("hisa_token_topk_noalloc",
+           _lib.hisa_token_topk_noalloc(ctypes.byref(p), _ptr(q_idx), _ptr(k_idx), _ptr(block_idx), _ptr(token_idx),
+                                        _ptr(token_scores), _ptr(dev_status), _stream(stream)))
 
 
 def hisa_version() -> str:

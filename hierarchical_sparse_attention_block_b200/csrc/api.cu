@@ -11,9 +11,9 @@
 
 namespace hisa {
 
-namespace {
-
 thread_local int32_t g_last_cuda_error = 0;
+
+namespace {
 
 hisa_status_t cuda_fail(cudaError_t e) {
   if (e == cudaSuccess) return HISA_OK;

@@ -50,6 +50,9 @@ size_t attn_partial_bytes(const Shape& s, int splits);
 cudaError_t launch_sparse_attn(const Shape& s, const void* q, const void* k, const void* v, const int32_t* token_idx,
                                void* o, float* lse, int32_t* status, int splits, void* partial, cudaStream_t st);
 
+// cudaError_t value behind the last HISA_ERR_CUDA on this host thread.
+extern thread_local int32_t g_last_cuda_error;
+
 // Dynamic shared memory opt-in, once per (kernel, device).
 cudaError_t ensure_smem(const void* func, int bytes);
 

@@ -155,6 +155,25 @@ hisa_status_t hisa_flat_topk(const hisa_params_t* params, const void* q_idx, con
                              int32_t* token_idx, float* token_scores, void* workspace, size_t workspace_bytes,
                              cudaStream_t stream);
 
+/* The token stage (steps 4-5) for callers that cannot allocate device memory.
+ * The pages have no counterpart of this call; it exists for users of the
+ * library, not for the method.  Same arguments, results and device checks as
+ * hisa_token_topk, minus the workspace: some callers only hand a library the
+ * buffers they already own (an inference engine that plans all device memory
+ * up front and gives plugins no allocator, a latency-critical loop that must
+ * not call the synchronizing cudaMalloc, a binding that cannot manage a
+ * scratch buffer's lifetime).  The scratch is a file-scope device array of
+ * 16 MiB that every GPU loading this part of the library holds until exit;
+ * queries run in chunks that fit it, and a request whose single query needs
+ * more than 16 MiB of candidate keys (top_m * block * 4 bytes) returns
+ * HISA_ERR_UNSUPPORTED.  Nothing is allocated by the call.  The first call on
+ * each device looks up the array's device address; make that first call
+ * before any stream capture.  All calls share the array: calls that overlap
+ * on the GPU (other streams or host threads) race, so serialize them. */
+hisa_status_t hisa_token_topk_noalloc(const hisa_params_t* params, const void* q_idx, const void* k_idx,
+                                      const int32_t* block_idx, int32_t* token_idx, float* token_scores,
+                                      int32_t* dev_status, cudaStream_t stream);
+
 /* Static text for a status code. */
 const char* hisa_status_string(hisa_status_t status);
 /* cudaError_t value of the last failed CUDA call on this host thread (0 if none). */
