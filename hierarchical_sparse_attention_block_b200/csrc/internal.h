@@ -41,6 +41,10 @@ cudaError_t launch_block_topm(const Shape& s, const float* scores, int32_t* bloc
 // indexer (block_idx == nullptr: slot r is block r).  keys: [nq][slots * B].
 cudaError_t launch_token_score(const Shape& s, const void* q_idx, const void* k_idx, const int32_t* block_idx,
                                int slots, uint32_t* keys, int32_t* status, int64_t q0, int64_t nq, cudaStream_t st);
+// Tensor-core version of launch_token_score for prefill (same key layout).
+bool token_score_tc_eligible(const Shape& s, int slots);
+cudaError_t launch_token_score_tc(const Shape& s, const void* q_idx, const void* k_idx, const int32_t* block_idx,
+                                  int slots, uint32_t* keys, int32_t* status, int64_t q0, int64_t nq, cudaStream_t st);
 cudaError_t launch_token_select(const Shape& s, const uint32_t* keys, const int32_t* block_idx, int slots,
                                 int32_t* token_idx, float* token_scores, int64_t q0, int64_t nq, cudaStream_t st);
 

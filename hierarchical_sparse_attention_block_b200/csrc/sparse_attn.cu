@@ -5,39 +5,80 @@
 // Work item = (head, query, split), heads outermost so that the CTAs running
 // at the same time gather from one head's K/V (n_kv * d * 4 B), which the L2
 // then serves to many queries.  A CTA has 4 warps; each warp owns every 4th
-// tile of 8 list entries and runs its own 4-stage cp.async pipeline (no CTA
-// barriers in the main loop).  Per tile: the K and V rows of 8 tokens
-// (2 x 8 x d bf16) land in the warp's shared-memory stage; 8 lanes score one
-// token (16-byte conflict-free reads, 3 shuffles), the warp updates its
-// running max / sum (base-2 online softmax), and every lane accumulates
-// d/32 output dimensions.  The four warps' partial states merge through
-// shared memory at the end.  Invalid entries are zero-filled and masked.
+// tile of 16 list entries and runs its own cp.async pipeline of kStages tiles
+// (rows padded by 16 bytes so the ldmatrix reads are bank-conflict free;
+// invalid entries are zero-filled and masked).  Per tile, on the tensor cores
+// (mma.sync m16n8k16, bf16 in, fp32 accumulate):
+//   * scores: [q; q; 0 ...] (16 x d) x K_tileᵀ (d x 8 tokens), twice; the
+//     scores of the 16 tokens land in lanes 0-7, laid out exactly as the
+//     output MMA wants its B operand, so no shuffles are needed;
+//   * base-2 softmax against a running max that is raised (and the state
+//     rescaled) only when a score exceeds it by more than 2^8 -- one vote per
+//     tile in the common case; per-lane partial row sums;
+//   * output: Oᵀ (d x 8) += V_tileᵀ (d x 16, ldmatrix.trans) x Pᵀ (16 x 8),
+//     column 0 of Pᵀ = bf16(p), column 1 = bf16(p - bf16(p)), so the two
+//     output columns add up to the weights carried to ~16 bits.
+// The four warps' (max, sum, output) states merge through shared memory.
 // When there are few queries (decode) the list is split across CTAs and a
-// second kernel merges the partial (max, sum, output) triples.
+// second kernel merges the partial states.  Out-of-range entries set bit 0 of
+// the status word.
 #include <math.h>
 
 #include "common.cuh"
 #include "internal.h"
 
+#ifndef HISA_ATTN_STAGES
+#define HISA_ATTN_STAGES 2
+#endif
+
 namespace hisa {
 namespace {
 
-constexpr int kNW = 4;  // warps per CTA
-constexpr int kTT = 8;  // list entries per warp tile
-constexpr int kNS = 4;  // pipeline stages per warp
+constexpr int kNW = 4;   // warps per CTA
+constexpr int kT = 16;   // list entries per warp tile
+constexpr int kNS = HISA_ATTN_STAGES;
 
 template <int D>
 struct AttnCfg {
-  static constexpr int ROW = D * 2;                   // bytes per K or V row
-  static constexpr int CH = D / 8;                    // 16-byte chunks per row
-  static constexpr int STAGE = kTT * 2 * ROW;         // K rows then V rows
-  static constexpr int IDS = kNS * kTT * 4;           // token ids per stage
-  static constexpr int WARP = kNS * STAGE + IDS;      // per-warp bytes
-  static constexpr int SMEM = kNW * WARP;
-  static constexpr int CPL = CH / 8;                  // chunks per lane in the score
-  static constexpr int PV = D / 32;                   // output dims per lane
-  static constexpr int TOK_PER_ITER = 32 / (2 * CH);  // tokens copied per warp instruction
+  static constexpr int ROW = D * 2;                    // bytes of one K or V row
+  static constexpr int PITCH = ROW + 16;               // padded shared-memory row pitch
+  static constexpr int CH = D / 8;                     // 16-byte chunks per row
+  static constexpr int ROWS_PER_ITER = 32 / (2 * CH);  // rows (K and V) moved per warp copy step
+  static constexpr int STAGE = 2 * kT * PITCH;         // 16 K rows, then 16 V rows
+  static constexpr int KSTEPS = D / 16;                // QK k-steps and PV m-tiles
+  static constexpr int WARP = kNS * STAGE;
+  static constexpr int MASK_OFF = kNW * WARP;          // token ids of every stage
+  static constexpr int SMEM = MASK_OFF + kNW * kNS * kT * 4;
 };
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+// 16-byte global -> shared copy through L2 only; pred == false zero-fills and reads nothing.
+__device__ __forceinline__ void cp_async16_u32(uint32_t dst, const void* src, bool pred) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(pred ? 16 : 0) : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// D (16x8 fp32) += A (16x16 bf16, row) x B (16x8 bf16, col)
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
 
 template <int D>
 __global__ void __launch_bounds__(kNW * 32)
@@ -48,7 +89,7 @@ __global__ void __launch_bounds__(kNW * 32)
                        float qscale, int64_t n_query) {
   using C = AttnCfg<D>;
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ int s_nuse[kNW];
+  __shared__ int s_last[kNW];
 
   const int64_t u = blockIdx.x;
   const int64_t per_head = n_query * splits;
@@ -60,6 +101,7 @@ __global__ void __launch_bounds__(kNW * 32)
   const int64_t p = n_kv - n_q + qg % n_q;
   const int g = h / (H / Hkv);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int gid = lane >> 2, tig = lane & 3;
   const int32_t* list = token_idx + qg * topk;
 
   // Entries past the last valid one are skipped.
@@ -68,74 +110,75 @@ __global__ void __launch_bounds__(kNW * 32)
     if (list[e] >= 0) last = e;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) last = max(last, __shfl_xor_sync(0xFFFFFFFFu, last, off));
-  if (lane == 0) s_nuse[warp] = last;
+  if (lane == 0) s_last[warp] = last;
   __syncthreads();
   int n_use = -1;
 #pragma unroll
-  for (int w = 0; w < kNW; ++w) n_use = max(n_use, s_nuse[w]);
+  for (int w = 0; w < kNW; ++w) n_use = max(n_use, s_last[w]);
   n_use += 1;
 
   int per = (n_use + splits - 1) / splits;
-  per = (per + kTT - 1) / kTT * kTT;
+  per = (per + kT - 1) / kT * kT;
   const int e0 = min(split * per, n_use), e1 = min(e0 + per, n_use);
-  const int n_tiles = (e1 - e0 + kTT - 1) / kTT;
+  const int n_tiles = (e1 - e0 + kT - 1) / kT;
+  const int my_tiles = n_tiles > warp ? (n_tiles - warp + kNW - 1) / kNW : 0;
 
-  // Query fragment for the score: lane `sub` of each 8-lane group holds chunks sub + 8u.
-  const int grp = lane >> 3, sub = lane & 7;
-  float qf[8 * C::CPL];
+  // q as the A operand of the score MMA, in rows 0 and 1 (rows 2..15 zero), so that the
+  // scores land in lanes 0-7, which are the lanes that feed P into the output MMA.
+  uint32_t qa[C::KSTEPS][2];
   {
     const uint16_t* qrow = q + (qg * H + h) * D;
 #pragma unroll
-    for (int uu = 0; uu < C::CPL; ++uu) {
-      const uint4 w = *reinterpret_cast<const uint4*>(qrow + (sub + 8 * uu) * 8);
-      qf[8 * uu + 0] = bf16_lo(w.x) * qscale; qf[8 * uu + 1] = bf16_hi(w.x) * qscale;
-      qf[8 * uu + 2] = bf16_lo(w.y) * qscale; qf[8 * uu + 3] = bf16_hi(w.y) * qscale;
-      qf[8 * uu + 4] = bf16_lo(w.z) * qscale; qf[8 * uu + 5] = bf16_hi(w.z) * qscale;
-      qf[8 * uu + 6] = bf16_lo(w.w) * qscale; qf[8 * uu + 7] = bf16_hi(w.w) * qscale;
+    for (int s = 0; s < C::KSTEPS; ++s) {
+      qa[s][0] = gid < 2 ? *reinterpret_cast<const uint32_t*>(qrow + 16 * s + 2 * tig) : 0u;
+      qa[s][1] = gid < 2 ? *reinterpret_cast<const uint32_t*>(qrow + 16 * s + 2 * tig + 8) : 0u;
     }
   }
 
+  // Copies: iteration i moves row i of the tile; lanes 0..CH-1 a K chunk, CH..2CH-1 a V chunk.
   uint8_t* wbuf = smem + warp * C::WARP;
-  int32_t* ids = reinterpret_cast<int32_t*>(wbuf + kNS * C::STAGE);
-  const int64_t kv_row0 = (int64_t)seq * n_kv;
+  const uint32_t wbase = smem_u32(wbuf);
+  const int part = (lane / C::CH) & 1;          // 0 = K, 1 = V
+  const int ch = lane % C::CH;
+  const uint16_t* src_base = (part ? v : k) + ((int64_t)seq * n_kv * Hkv + g) * D + ch * 8;
+  const int64_t tok_stride = (int64_t)Hkv * D;
+  const uint32_t dst_lane = (uint32_t)(part * kT * C::PITCH + ch * 16);
+  int32_t* ids_s = reinterpret_cast<int32_t*>(smem + C::MASK_OFF) + warp * kNS * kT;
 
-  // Issue the copies of this warp's j-th tile into stage j % kNS.
   auto issue = [&](int j) {
     const int t = warp + j * kNW;
     if (t < n_tiles) {
       const int stage = j % kNS;
-      uint8_t* sbuf = wbuf + stage * C::STAGE;
-      const int ebase = e0 + t * kTT;
-      int my_tok = -1;
-      if (lane < kTT) {
+      const int ebase = e0 + t * kT;
+      if (lane < kT) {
         const int e = ebase + lane;
-        if (e < e1) {
-          const int tok = list[e];
-          const bool ok = tok >= 0 && (int64_t)tok <= p;
-          if (!ok && tok != -1 && status) atomicOr(status, kStatusBadIndex);
-          my_tok = ok ? tok : -1;
-        }
-        ids[stage * kTT + lane] = my_tok;
+        int tok = e < e1 ? list[e] : -1;
+        const bool ok = tok >= 0 && (int64_t)tok <= p;
+        if (!ok && tok != -1 && status) atomicOr(status, kStatusBadIndex);
+        ids_s[stage * kT + lane] = ok ? tok : -1;
       }
+      __syncwarp();
+      const uint32_t sdst = wbase + stage * C::STAGE + dst_lane;
 #pragma unroll
-      for (int it = 0; it < kTT / C::TOK_PER_ITER; ++it) {
-        const int tl = it * C::TOK_PER_ITER + lane / (2 * C::CH);
-        const int part = (lane / C::CH) & 1;  // 0 = K, 1 = V
-        const int ch = lane % C::CH;
-        const int tok = __shfl_sync(0xFFFFFFFFu, my_tok, tl);
-        const uint16_t* src = (part ? v : k) + ((kv_row0 + (tok < 0 ? 0 : tok)) * Hkv + g) * D + ch * 8;
-        cp_async16(sbuf + part * kTT * C::ROW + tl * C::ROW + ch * 16, src, tok >= 0);
+      for (int i = 0; i < kT / C::ROWS_PER_ITER; ++i) {
+        const int r = i * C::ROWS_PER_ITER + lane / (2 * C::CH);
+        const int tok = ids_s[stage * kT + r];
+        cp_async16_u32(sdst + r * C::PITCH, src_base + (int64_t)(tok < 0 ? 0 : tok) * tok_stride, tok >= 0);
       }
     }
     cp_async_commit();
   };
 
-  float m_run = -INFINITY, l_run = 0.f;
-  float acc[C::PV];
+  float m_run = -INFINITY, l_part = 0.f;
+  float acc[C::KSTEPS][4];
 #pragma unroll
-  for (int e = 0; e < C::PV; ++e) acc[e] = 0.f;
+  for (int mt = 0; mt < C::KSTEPS; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
 
-  const int my_tiles = n_tiles > warp ? (n_tiles - warp + kNW - 1) / kNW : 0;
+  // ldmatrix row addresses within a stage: K^T fragments (non-transposed) and V^T (transposed).
+  const int mi = lane >> 3;
+  const uint32_t a_k = (uint32_t)(((lane & 7) + (mi >> 1) * 8) * C::PITCH + (mi & 1) * 16);
+  const uint32_t a_v = (uint32_t)((kT + (lane & 7) + (mi >> 1) * 8) * C::PITCH + (mi & 1) * 16);
+
 #pragma unroll
   for (int j = 0; j < kNS - 1; ++j) issue(j);
   for (int j = 0; j < my_tiles; ++j) {
@@ -143,78 +186,90 @@ __global__ void __launch_bounds__(kNW * 32)
     cp_async_wait<kNS - 1>();
     __syncwarp();
     const int stage = j % kNS;
-    const uint8_t* kb = wbuf + stage * C::STAGE;
-    const uint8_t* vb = kb + kTT * C::ROW;
-    // scores of tokens grp and 4 + grp
-    float sc[2];
+    const uint32_t sb = wbase + stage * C::STAGE;
+
+    // scores of tokens 2tig, 2tig+1 (first MMA) and 8+2tig, 9+2tig (second), in lanes 0-7
+    float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int tl = r * 4 + grp;
-      float dot = 0.f;
-#pragma unroll
-      for (int uu = 0; uu < C::CPL; ++uu) {
-        const uint4 w = *reinterpret_cast<const uint4*>(kb + tl * C::ROW + (sub + 8 * uu) * 16);
-        const float* qq = qf + 8 * uu;
-        dot = fmaf(qq[0], bf16_lo(w.x), dot); dot = fmaf(qq[1], bf16_hi(w.x), dot);
-        dot = fmaf(qq[2], bf16_lo(w.y), dot); dot = fmaf(qq[3], bf16_hi(w.y), dot);
-        dot = fmaf(qq[4], bf16_lo(w.z), dot); dot = fmaf(qq[5], bf16_hi(w.z), dot);
-        dot = fmaf(qq[6], bf16_lo(w.w), dot); dot = fmaf(qq[7], bf16_hi(w.w), dot);
-      }
-      dot += __shfl_xor_sync(0xFFFFFFFFu, dot, 4);
-      dot += __shfl_xor_sync(0xFFFFFFFFu, dot, 2);
-      dot += __shfl_xor_sync(0xFFFFFFFFu, dot, 1);
-      sc[r] = ids[stage * kTT + tl] >= 0 ? dot : -INFINITY;
+    for (int s = 0; s < C::KSTEPS; ++s) {
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4(sb + a_k + s * 32, b0, b1, b2, b3);
+      mma_bf16(s0, qa[s][0], 0u, qa[s][1], 0u, b0, b1);
+      mma_bf16(s1, qa[s][0], 0u, qa[s][1], 0u, b2, b3);
     }
-    float mt = fmaxf(sc[0], sc[1]);
-    mt = fmaxf(mt, __shfl_xor_sync(0xFFFFFFFFu, mt, 8));
-    mt = fmaxf(mt, __shfl_xor_sync(0xFFFFFFFFu, mt, 16));
-    const float m_new = fmaxf(m_run, mt);
-    if (m_new != -INFINITY) {
+    const int32_t* ids = ids_s + stage * kT;
+    float sc[4];
+    sc[0] = (gid < 2 && ids[2 * tig] >= 0) ? s0[0] * qscale : -INFINITY;
+    sc[1] = (gid < 2 && ids[2 * tig + 1] >= 0) ? s0[1] * qscale : -INFINITY;
+    sc[2] = (gid < 2 && ids[8 + 2 * tig] >= 0) ? s1[0] * qscale : -INFINITY;
+    sc[3] = (gid < 2 && ids[9 + 2 * tig] >= 0) ? s1[1] * qscale : -INFINITY;
+    const float smax = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+    // Rescale only when a score exceeds the running max by more than 2^8.
+    if (__any_sync(0xFFFFFFFFu, smax > m_run + 8.f)) {
+      float tmax = smax;
+      tmax = fmaxf(tmax, __shfl_xor_sync(0xFFFFFFFFu, tmax, 1));
+      tmax = fmaxf(tmax, __shfl_xor_sync(0xFFFFFFFFu, tmax, 2));
+      tmax = __shfl_sync(0xFFFFFFFFu, tmax, 0);
+      const float m_new = fmaxf(m_run, tmax);
       const float alpha = exp2f(m_run - m_new);
-      const float p0 = exp2f(sc[0] - m_new), p1 = exp2f(sc[1] - m_new);
-      float ps = p0 + p1;
-      ps += __shfl_xor_sync(0xFFFFFFFFu, ps, 8);
-      ps += __shfl_xor_sync(0xFFFFFFFFu, ps, 16);
-      l_run = l_run * alpha + ps;
+      l_part *= alpha;
 #pragma unroll
-      for (int e = 0; e < C::PV; ++e) acc[e] *= alpha;
-#pragma unroll
-      for (int src = 0; src < 4; ++src) {
-        const float pa = __shfl_sync(0xFFFFFFFFu, p0, src * 8);
-        const float pb = __shfl_sync(0xFFFFFFFFu, p1, src * 8);
-        const uint8_t* va = vb + src * C::ROW + lane * C::PV * 2;
-        const uint8_t* vbb = vb + (4 + src) * C::ROW + lane * C::PV * 2;
-        if constexpr (C::PV == 4) {
-          const uint2 a = *reinterpret_cast<const uint2*>(va);
-          const uint2 b = *reinterpret_cast<const uint2*>(vbb);
-          acc[0] = fmaf(pa, bf16_lo(a.x), acc[0]); acc[1] = fmaf(pa, bf16_hi(a.x), acc[1]);
-          acc[2] = fmaf(pa, bf16_lo(a.y), acc[2]); acc[3] = fmaf(pa, bf16_hi(a.y), acc[3]);
-          acc[0] = fmaf(pb, bf16_lo(b.x), acc[0]); acc[1] = fmaf(pb, bf16_hi(b.x), acc[1]);
-          acc[2] = fmaf(pb, bf16_lo(b.y), acc[2]); acc[3] = fmaf(pb, bf16_hi(b.y), acc[3]);
-        } else {
-          const uint32_t a = *reinterpret_cast<const uint32_t*>(va);
-          const uint32_t b = *reinterpret_cast<const uint32_t*>(vbb);
-          acc[0] = fmaf(pa, bf16_lo(a), acc[0]); acc[1] = fmaf(pa, bf16_hi(a), acc[1]);
-          acc[0] = fmaf(pb, bf16_lo(b), acc[0]); acc[1] = fmaf(pb, bf16_hi(b), acc[1]);
-        }
+      for (int mt = 0; mt < C::KSTEPS; ++mt) {
+        acc[mt][0] *= alpha;
+        acc[mt][1] *= alpha;
+        acc[mt][2] *= alpha;
+        acc[mt][3] *= alpha;
       }
       m_run = m_new;
+    }
+    if (m_run != -INFINITY) {
+      float pv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) pv[i] = exp2f(sc[i] - m_run);
+      if (gid == 0) l_part += (pv[0] + pv[1]) + (pv[2] + pv[3]);
+      // P^T column 0 (lanes 0-3) = bf16(p); column 1 (lanes 4-7) = bf16(p - bf16(p)).
+      const __nv_bfloat162 h01 = __floats2bfloat162_rn(pv[0], pv[1]);
+      const __nv_bfloat162 h89 = __floats2bfloat162_rn(pv[2], pv[3]);
+      uint32_t b0 = 0u, b1 = 0u;
+      if (gid == 0) {
+        b0 = *reinterpret_cast<const uint32_t*>(&h01);
+        b1 = *reinterpret_cast<const uint32_t*>(&h89);
+      } else if (gid == 1) {
+        const __nv_bfloat162 l01 = __floats2bfloat162_rn(pv[0] - __low2float(h01), pv[1] - __high2float(h01));
+        const __nv_bfloat162 l89 = __floats2bfloat162_rn(pv[2] - __low2float(h89), pv[3] - __high2float(h89));
+        b0 = *reinterpret_cast<const uint32_t*>(&l01);
+        b1 = *reinterpret_cast<const uint32_t*>(&l89);
+      }
+#pragma unroll
+      for (int mt = 0; mt < C::KSTEPS; ++mt) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4_t(sb + a_v + mt * 32, a0, a1, a2, a3);
+        mma_bf16(acc[mt], a0, a1, a2, a3, b0, b1);
+      }
     }
     __syncwarp();
   }
   cp_async_wait<0>();
+  // per-warp row sum: lanes 0-3 hold partial sums
+  l_part += __shfl_xor_sync(0xFFFFFFFFu, l_part, 1);
+  l_part += __shfl_xor_sync(0xFFFFFFFFu, l_part, 2);
   __syncthreads();
 
-  // Merge the warps' states.
-  float* mg = reinterpret_cast<float*>(smem);  // [kNW] max, [kNW] sum, [kNW][D] acc
+  // Merge the warps' states: [kNW] max, [kNW] sum, [kNW][D] output.
+  float* mg = reinterpret_cast<float*>(smem);
   if (lane == 0) {
     mg[warp] = m_run;
-    mg[kNW + warp] = l_run;
+    mg[kNW + warp] = l_part;
   }
+  if (tig == 0) {
 #pragma unroll
-  for (int e = 0; e < C::PV; ++e) mg[2 * kNW + warp * D + lane * C::PV + e] = acc[e];
+    for (int mtile = 0; mtile < C::KSTEPS; ++mtile) {
+      mg[2 * kNW + warp * D + 16 * mtile + gid] = acc[mtile][0] + acc[mtile][1];
+      mg[2 * kNW + warp * D + 16 * mtile + gid + 8] = acc[mtile][2] + acc[mtile][3];
+    }
+  }
   __syncthreads();
-  for (int d = threadIdx.x; d < D; d += kNW * 32) {
+  for (int dd = threadIdx.x; dd < D; dd += kNW * 32) {
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < kNW; ++w) M = fmaxf(M, mg[w]);
@@ -224,21 +279,21 @@ __global__ void __launch_bounds__(kNW * 32)
       for (int w = 0; w < kNW; ++w) {
         const float f = exp2f(mg[w] - M);
         L = fmaf(mg[kNW + w], f, L);
-        O = fmaf(mg[2 * kNW + w * D + d], f, O);
+        O = fmaf(mg[2 * kNW + w * D + dd], f, O);
       }
     }
     if (splits == 1) {
       const float out = L > 0.f ? O / L : 0.f;
       __nv_bfloat16 b = __float2bfloat16_rn(out);
-      o[(qg * H + h) * D + d] = *reinterpret_cast<uint16_t*>(&b);
-      if (d == 0 && lse) lse[qg * H + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
+      o[(qg * H + h) * D + dd] = *reinterpret_cast<uint16_t*>(&b);
+      if (dd == 0 && lse) lse[qg * H + h] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
     } else {
-      float* part = partial + ((qg * H + h) * splits + split) * (D + 2);
-      if (d == 0) {
-        part[0] = M;
-        part[1] = L;
+      float* pt = partial + ((qg * H + h) * splits + split) * (D + 2);
+      if (dd == 0) {
+        pt[0] = M;
+        pt[1] = L;
       }
-      part[2 + d] = O;
+      pt[2 + dd] = O;
     }
   }
 }

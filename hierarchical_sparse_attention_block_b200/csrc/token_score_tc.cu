@@ -1,0 +1,355 @@
+// Step 4 on the 5th-generation tensor cores (prefill): token scores of the
+// kept blocks.  "北大HISA稀疏注意力机制" section 1.2.2 item 1; QbitAI HISA
+// article, "塊內精挑字符".
+//
+// A kept block is a contiguous B x d_idx tile of k_idx, and 128 consecutive
+// queries keep overlapping sets of blocks.  So instead of gathering rows per
+// query, a CTA takes a tile of 128 queries of one sequence and a run of up to
+// kRun key blocks at or below the tile's causal limit, and for each block j:
+//   * TMA brings K_j (B rows, 128-byte swizzle: the K-major UMMA operand) into
+//     one of 2-3 shared-memory stages (the 128 query rows came once);
+//   * one thread issues d_idx/16 tcgen05.mma (kind::f16, M=128, N=B) writing
+//     all 128 x B scores to TMEM (fp32; exact on integer-valued inputs);
+//   * each warp reads its 32 query rows back (tcgen05.ld) -- only when one of
+//     its queries kept block j -- and writes that query's B order-preserving
+//     keys to its slot of the key buffer (0 for tokens after the query).
+// The slot of block j in each query's kept list comes from a per-CTA map
+// built by scanning the lists once (same acceptance rule as the CUDA-core
+// scorer: in range and above every earlier in-range entry).  The CTA holding
+// the first run also zero-fills unused slots and flags malformed entries.
+// With no list (the flat indexer) slot = block id.  Waits are bounded (1 s);
+// a timeout sets status bit 1.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace hisa {
+namespace {
+
+constexpr int kThreads = 128;
+constexpr int kTileQ = 128;
+constexpr int kRun = 64;      // key blocks per CTA
+constexpr int kStatusTimeout = 2;
+constexpr uint64_t kWaitNs = 1000000000ull;
+
+template <int D, int B>
+struct TsLayout {
+  static constexpr int HALVES = D / 64;
+  static constexpr int Q_BYTES = HALVES * kTileQ * 128;
+  static constexpr int K_BYTES = HALVES * B * 128;
+  static constexpr int STAGES = K_BYTES >= 65536 ? 2 : 3;  // K tiles in flight
+  static constexpr int Q_OFF = 0;
+  static constexpr int K_OFF = Q_OFF + Q_BYTES;
+  static constexpr int MAP_OFF = K_OFF + STAGES * K_BYTES;  // int16 [kTileQ][kRun]
+  static constexpr int BAR_OFF = MAP_OFF + kTileQ * kRun * 2;
+  static constexpr int SMEM = BAR_OFF + 8 * (2 + STAGES) + 16 + 1024;
+  static_assert(SMEM <= 227 * 1024, "shared memory budget");
+  static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(B >> 3) << 17) |
+                                    ((uint32_t)(kTileQ >> 4) << 24);
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = global_ns();
+  while (true) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    if (global_ns() - t0 > kWaitNs) return false;
+  }
+}
+
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1 << 16;            // leading byte offset (unused for this layout)
+  d |= (uint64_t)(1024 >> 4) << 32;  // 8-row groups 1024 B apart
+  d |= (uint64_t)1 << 46;            // sm_100 descriptor version
+  d |= (uint64_t)2 << 61;            // 128-byte swizzle
+  return d;
+}
+
+__device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+template <int D, int B>
+__global__ void __launch_bounds__(kThreads, 1)
+    token_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                          const int32_t* __restrict__ block_idx, int slots, uint32_t* __restrict__ keys,
+                          int32_t* __restrict__ status, int64_t n_q, int64_t n_kv, int q_tiles, int runs, int64_t q0,
+                          int64_t nq) {
+  using L = TsLayout<D, B>;
+  constexpr int kKStages = L::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+
+  // Tiles are enumerated over the queries of the chunk [q0, q0 + nq).
+  const int run = blockIdx.x % runs;
+  const int64_t tile_lin = blockIdx.x / runs;
+  const int64_t seq_first = q0 / n_q;
+  const int64_t tile0 = (q0 % n_q) / kTileQ;  // first tile of the first sequence touched
+  const int64_t tile_abs = tile0 + tile_lin;  // tile counted from the first sequence's start
+  const int64_t seq = seq_first + tile_abs / q_tiles;
+  const int64_t ti = tile_abs % q_tiles;
+  const int64_t tq0 = seq * n_q + ti * kTileQ;                 // first global query of the tile
+  const int64_t t_lo = max(tq0, q0);
+  const int64_t t_hi = min(min(tq0 + kTileQ, (seq + 1) * n_q), q0 + nq);  // exclusive
+  if (t_lo >= t_hi) return;
+  const int64_t c_max = (n_kv - n_q + (t_hi - 1 - seq * n_q)) / B;
+  const int64_t jb0 = (int64_t)run * kRun;
+  if (jb0 > c_max) return;
+  const int nb = (int)min((int64_t)kRun, c_max + 1 - jb0);
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint8_t* sQ = smem + L::Q_OFF;
+  uint8_t* sK = smem + L::K_OFF;
+  int16_t* smap = reinterpret_cast<int16_t*>(smem + L::MAP_OFF);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);  // [0] q, [1] mma, [2..] k stages
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::BAR_OFF + 8 * (2 + kKStages));
+
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"((uint32_t)(B < 32 ? 32 : B)));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  if (tid == 0) {
+    for (int i = 0; i < 2 + kKStages; ++i)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars[i])));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem = *tmem_slot;
+
+  // Producer: the query tile and the first K stages.
+  if (tid == 0) {
+    const uint32_t bq = smem_u32(&bars[0]);
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bq), "r"((uint32_t)L::Q_BYTES)
+                 : "memory");
+    for (int hh = 0; hh < L::HALVES; ++hh) tma_2d(smem_u32(sQ + hh * kTileQ * 128), &tmap_q, hh * 64, (int)tq0, bq);
+    for (int s = 0; s < kKStages && s < nb; ++s) {
+      const uint32_t bk = smem_u32(&bars[2 + s]);
+      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bk), "r"((uint32_t)L::K_BYTES)
+                   : "memory");
+      const int krow = (int)(seq * n_kv + (jb0 + s) * B);
+      for (int hh = 0; hh < L::HALVES; ++hh)
+        tma_2d(smem_u32(sK + s * L::K_BYTES + hh * B * 128), &tmap_k, hh * 64, krow, bk);
+    }
+  }
+
+  // Slot map of this thread's query row for blocks jb0 .. jb0+nb-1.
+  const int64_t qrow = tq0 + tid;  // global query id of this thread's row
+  const bool row_ok = qrow >= t_lo && qrow < t_hi;
+  const int64_t p = n_kv - n_q + (qrow - seq * n_q);
+  const int64_t c = p / B;
+  uint32_t* krow_keys = keys + (qrow - q0) * (int64_t)slots * B;
+  for (int jj = 0; jj < kRun; ++jj) smap[tid * kRun + jj] = -1;
+  if (row_ok) {
+    if (block_idx) {
+      const int32_t* lst = block_idx + qrow * slots;
+      int mx = -1;
+      for (int r = 0; r < slots; ++r) {
+        const int b = lst[r];
+        const bool in_range = b >= 0 && b <= c;
+        const bool ok = in_range && b > mx;
+        if (ok && b >= jb0 && b < jb0 + nb) smap[tid * kRun + (b - jb0)] = (int16_t)r;
+        if (run == 0 && !ok) {
+          if (b != -1 && status) atomicOr(status, kStatusBadIndex);
+          uint4* z = reinterpret_cast<uint4*>(krow_keys + (int64_t)r * B);
+          for (int i = 0; i < B / 4; ++i) z[i] = make_uint4(0, 0, 0, 0);
+        }
+        if (in_range) mx = max(mx, b);
+      }
+    } else {
+      for (int jj = 0; jj < nb; ++jj)
+        if (jb0 + jj <= c) smap[tid * kRun + jj] = (int16_t)(jb0 + jj);
+      if (run == 0) {  // blocks after the query's own block hold no candidate
+        for (int64_t r = c + 1; r < slots; ++r) {
+          uint4* z = reinterpret_cast<uint4*>(krow_keys + r * B);
+          for (int i = 0; i < B / 4; ++i) z[i] = make_uint4(0, 0, 0, 0);
+        }
+      }
+    }
+  }
+
+  bool ok = mbar_wait(smem_u32(&bars[0]), 0);
+  ok = __syncthreads_and(ok) != 0;
+  const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK);
+  for (int b = 0; b < nb && ok; ++b) {
+    const int stage = b % kKStages;
+    const uint32_t phase = (uint32_t)((b / kKStages) & 1);
+    if (tid == 0) {
+      if (mbar_wait(smem_u32(&bars[2 + stage]), phase)) {
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+#pragma unroll
+        for (int hh = 0; hh < L::HALVES; ++hh) {
+#pragma unroll
+          for (int s = 0; s < 4; ++s) {
+            const uint64_t ad = desc_sw128(q_base + hh * kTileQ * 128 + s * 32);
+            const uint64_t bd = desc_sw128(k_base + stage * L::K_BYTES + hh * B * 128 + s * 32);
+            const uint32_t acc = (hh | s) ? 1u : 0u;
+            asm volatile(
+                "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+                " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem),
+                "l"(ad), "l"(bd), "r"(L::IDESC), "r"(acc));
+          }
+        }
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                         smem_u32(&bars[1]))
+                     : "memory");
+      } else {
+        if (status) atomicOr(status, kStatusTimeout);
+      }
+    }
+    bool done = mbar_wait(smem_u32(&bars[1]), (uint32_t)(b & 1));
+    done = __syncthreads_and(done) != 0;
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    if (!done) {
+      ok = false;
+      if (tid == 0 && status) atomicOr(status, kStatusTimeout);
+      break;
+    }
+    // The MMA has consumed this K stage: refill it with block b + kKStages.
+    if (tid == 0 && b + kKStages < nb) {
+      const uint32_t bk = smem_u32(&bars[2 + stage]);
+      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bk), "r"((uint32_t)L::K_BYTES)
+                   : "memory");
+      const int krow = (int)(seq * n_kv + (jb0 + b + kKStages) * B);
+      for (int hh = 0; hh < L::HALVES; ++hh)
+        tma_2d(smem_u32(sK + stage * L::K_BYTES + hh * B * 128), &tmap_k, hh * 64, krow, bk);
+    }
+    // Epilogue: rows whose query kept block jb0 + b.
+    const int slot = row_ok ? smap[tid * kRun + b] : -1;
+    if (__any_sync(0xFFFFFFFFu, slot >= 0)) {
+      const int64_t j = jb0 + b;
+      const int64_t tok0 = j * B;
+      uint32_t* dst = krow_keys + (int64_t)(slot < 0 ? 0 : slot) * B;
+#pragma unroll 1
+      for (int cc = 0; cc < B / 32; ++cc) {
+        uint32_t v[32];
+        const uint32_t addr = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(cc * 32);
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+            "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+              "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
+              "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
+              "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]),
+              "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+            : "r"(addr));
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        if (slot >= 0) {
+#pragma unroll
+          for (int t = 0; t < 32; t += 4) {
+            const int64_t tk = tok0 + cc * 32 + t;
+            uint4 w;
+            w.x = tk <= p ? score_key(__uint_as_float(v[t])) : 0u;
+            w.y = tk + 1 <= p ? score_key(__uint_as_float(v[t + 1])) : 0u;
+            w.z = tk + 2 <= p ? score_key(__uint_as_float(v[t + 2])) : 0u;
+            w.w = tk + 3 <= p ? score_key(__uint_as_float(v[t + 3])) : 0u;
+            *reinterpret_cast<uint4*>(dst + cc * 32 + t) = w;
+          }
+        }
+      }
+    }
+    // TMEM is rewritten by the next block's MMA only after every warp has read it.
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+  }
+
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (warp == 0) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"((uint32_t)(B < 32 ? 32 : B)));
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool map_bf16_sw128(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int B>
+cudaError_t launch_ts(const Shape& s, const void* q_idx, const void* k_idx, const int32_t* block_idx, int slots,
+                      uint32_t* keys, int32_t* status, int64_t q0, int64_t nq, cudaStream_t st) {
+  using L = TsLayout<D, B>;
+  CUtensorMap mq, mk;
+  if (!map_bf16_sw128(&mq, q_idx, D, (uint64_t)s.n_query, kTileQ)) return cudaErrorNotSupported;
+  if (!map_bf16_sw128(&mk, k_idx, D, (uint64_t)s.batch * s.n_kv, B)) return cudaErrorNotSupported;
+  auto kern = token_score_tc_kernel<D, B>;
+  cudaError_t e = ensure_smem((const void*)kern, L::SMEM);
+  if (e != cudaSuccess) return e;
+  const int q_tiles = (int)((s.n_q + kTileQ - 1) / kTileQ);
+  const int runs = (int)((s.n_blk + kRun - 1) / kRun);
+  // tiles from the chunk's first tile to its last
+  const int64_t first = (q0 / s.n_q) * q_tiles + (q0 % s.n_q) / kTileQ;
+  const int64_t lastq = q0 + nq - 1;
+  const int64_t last = (lastq / s.n_q) * q_tiles + (lastq % s.n_q) / kTileQ;
+  const int64_t grid = (last - first + 1) * runs;
+  if (grid > 0x7FFFFFFFLL) return cudaErrorNotSupported;
+  kern<<<(unsigned)grid, kThreads, L::SMEM, st>>>(mq, mk, block_idx, slots, keys, status, s.n_q, s.n_kv, q_tiles,
+                                                  runs, q0, nq);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool token_score_tc_eligible(const Shape& s, int slots) {
+  return (s.d_idx == 64 || s.d_idx == 128) && (s.B == 32 || s.B == 64 || s.B == 128 || s.B == 256) &&
+         s.n_q >= kTileQ && slots < 32767 && s.n_query <= 0x7FFFFFFFLL &&
+         (int64_t)s.batch * s.n_kv <= 0x7FFFFFFFLL;
+}
+
+cudaError_t launch_token_score_tc(const Shape& s, const void* q_idx, const void* k_idx, const int32_t* block_idx,
+                                  int slots, uint32_t* keys, int32_t* status, int64_t q0, int64_t nq, cudaStream_t st) {
+  if (!token_score_tc_eligible(s, slots)) return cudaErrorNotSupported;
+#define HISA_TS_CASE(DD, BB) \
+  if (s.d_idx == DD && s.B == BB) return launch_ts<DD, BB>(s, q_idx, k_idx, block_idx, slots, keys, status, q0, nq, st);
+  HISA_TS_CASE(64, 32) HISA_TS_CASE(64, 64) HISA_TS_CASE(64, 128) HISA_TS_CASE(64, 256)
+  HISA_TS_CASE(128, 32) HISA_TS_CASE(128, 64) HISA_TS_CASE(128, 128) HISA_TS_CASE(128, 256)
+#undef HISA_TS_CASE
+  return cudaErrorNotSupported;
+}
+
+}  // namespace hisa

@@ -177,6 +177,11 @@ __global__ void __launch_bounds__(NT)
 cudaError_t launch_token_score(const Shape& s, const void* q_idx, const void* k_idx, const int32_t* block_idx,
                                int slots, uint32_t* keys, int32_t* status, int64_t q0, int64_t nq, cudaStream_t st) {
   if (nq <= 0) return cudaSuccess;
+  // Many queries per sequence: tensor-core tiles of 128 queries x one key block.
+  if (token_score_tc_eligible(s, slots)) {
+    const cudaError_t e = launch_token_score_tc(s, q_idx, k_idx, block_idx, slots, keys, status, q0, nq, st);
+    if (e != cudaErrorNotSupported) return e;
+  }
   int spc = 1024 / s.B;
   spc = spc < 1 ? 1 : (spc > kMaxSlotsPerCta ? kMaxSlotsPerCta : spc);
   if (spc > slots) spc = slots;
