@@ -6,8 +6,9 @@
 // at the same time gather from one head's K/V (n_kv * d * 4 B), which the L2
 // then serves to many queries.  A CTA has 4 warps; each warp owns every 4th
 // tile of 16 list entries and runs its own cp.async pipeline of kStages tiles
-// (rows padded by 16 bytes so the ldmatrix reads are bank-conflict free;
-// invalid entries are zero-filled and masked).  Per tile, on the tensor cores
+// (rows kept 2d-byte aligned, 16-byte chunks XOR-swizzled by row so the
+// ldmatrix reads are bank-conflict free; invalid entries are zero-filled and
+// masked).  Per tile, on the tensor cores
 // (mma.sync m16n8k16, bf16 in, fp32 accumulate):
 //   * scores: [q; q; 0 ...] (16 x d) x K_tileᵀ (d x 8 tokens), twice; the
 //     scores of the 16 tokens land in lanes 0-7, laid out exactly as the
@@ -41,14 +42,14 @@ constexpr int kNS = HISA_ATTN_STAGES;
 template <int D>
 struct AttnCfg {
   static constexpr int ROW = D * 2;                    // bytes of one K or V row
-  static constexpr int PITCH = ROW + 16;               // padded shared-memory row pitch
   static constexpr int CH = D / 8;                     // 16-byte chunks per row
   static constexpr int ROWS_PER_ITER = 32 / (2 * CH);  // rows (K and V) moved per warp copy step
-  static constexpr int STAGE = 2 * kT * PITCH;         // 16 K rows, then 16 V rows
+  static constexpr int STAGE = 2 * kT * ROW;           // 16 K rows, then 16 V rows
   static constexpr int KSTEPS = D / 16;                // QK k-steps and PV m-tiles
   static constexpr int WARP = kNS * STAGE;
-  static constexpr int MASK_OFF = kNW * WARP;          // token ids of every stage
-  static constexpr int SMEM = MASK_OFF + kNW * kNS * kT * 4;
+  static constexpr int IDS_OFF = kNW * WARP;           // token ids of every stage
+  static constexpr int MASK_OFF = IDS_OFF + kNW * kNS * kT * 4;
+  static constexpr int SMEM = MASK_OFF + kNW * kNS * 4;
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -136,34 +137,46 @@ __global__ void __launch_bounds__(kNW * 32)
   }
 
   // Copies: iteration i moves row i of the tile; lanes 0..CH-1 a K chunk, CH..2CH-1 a V chunk.
+  // Rows stay 2*d-byte aligned; 16-byte chunk c of row r is stored at chunk c ^ (r & 7), which
+  // makes the 8-row ldmatrix reads below bank-conflict free.
   uint8_t* wbuf = smem + warp * C::WARP;
   const uint32_t wbase = smem_u32(wbuf);
-  const int part = (lane / C::CH) & 1;          // 0 = K, 1 = V
+  const int part = (lane / C::CH) & 1;  // 0 = K, 1 = V
   const int ch = lane % C::CH;
   const uint16_t* src_base = (part ? v : k) + ((int64_t)seq * n_kv * Hkv + g) * D + ch * 8;
-  const int64_t tok_stride = (int64_t)Hkv * D;
-  const uint32_t dst_lane = (uint32_t)(part * kT * C::PITCH + ch * 16);
-  int32_t* ids_s = reinterpret_cast<int32_t*>(smem + C::MASK_OFF) + warp * kNS * kT;
+  const uint64_t tok_stride = (uint64_t)Hkv * D;
+  int32_t* ids_s = reinterpret_cast<int32_t*>(smem + C::IDS_OFF) + warp * kNS * kT;
+  uint32_t* mask_s = reinterpret_cast<uint32_t*>(smem + C::MASK_OFF) + warp * kNS;
 
   auto issue = [&](int j) {
     const int t = warp + j * kNW;
     if (t < n_tiles) {
       const int stage = j % kNS;
       const int ebase = e0 + t * kT;
+      bool ok = false;
       if (lane < kT) {
         const int e = ebase + lane;
-        int tok = e < e1 ? list[e] : -1;
-        const bool ok = tok >= 0 && (int64_t)tok <= p;
+        const int tok = e < e1 ? list[e] : -1;
+        ok = tok >= 0 && (int64_t)tok <= p;
         if (!ok && tok != -1 && status) atomicOr(status, kStatusBadIndex);
         ids_s[stage * kT + lane] = ok ? tok : -1;
       }
+      const uint32_t valid = __ballot_sync(0xFFFFFFFFu, ok);
+      if (lane == 0) mask_s[stage] = valid;
       __syncwarp();
-      const uint32_t sdst = wbase + stage * C::STAGE + dst_lane;
+      int tk[kT];
+#pragma unroll
+      for (int i = 0; i < kT; i += 4) {
+        const int4 t4 = *reinterpret_cast<const int4*>(ids_s + stage * kT + i);
+        tk[i] = t4.x; tk[i + 1] = t4.y; tk[i + 2] = t4.z; tk[i + 3] = t4.w;
+      }
+      const uint32_t sdst = wbase + stage * C::STAGE + part * kT * C::ROW;
 #pragma unroll
       for (int i = 0; i < kT / C::ROWS_PER_ITER; ++i) {
         const int r = i * C::ROWS_PER_ITER + lane / (2 * C::CH);
-        const int tok = ids_s[stage * kT + r];
-        cp_async16_u32(sdst + r * C::PITCH, src_base + (int64_t)(tok < 0 ? 0 : tok) * tok_stride, tok >= 0);
+        const int tok = C::ROWS_PER_ITER == 1 ? tk[i] : (lane / (2 * C::CH) ? tk[2 * i + 1] : tk[2 * i]);
+        cp_async16_u32(sdst + r * C::ROW + ((ch ^ (r & 7)) << 4),
+                       src_base + (uint64_t)(uint32_t)(tok < 0 ? 0 : tok) * tok_stride, tok >= 0);
       }
     }
     cp_async_commit();
@@ -174,10 +187,12 @@ __global__ void __launch_bounds__(kNW * 32)
 #pragma unroll
   for (int mt = 0; mt < C::KSTEPS; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
 
-  // ldmatrix row addresses within a stage: K^T fragments (non-transposed) and V^T (transposed).
+  // ldmatrix rows: lane supplies row (lane & 7) + 8 * (mi >> 1) of logical chunk 2s + (mi & 1),
+  // stored at chunk (2s + (mi & 1)) ^ (lane & 7) = 2s ^ y with y = (mi & 1) ^ (lane & 7).
   const int mi = lane >> 3;
-  const uint32_t a_k = (uint32_t)(((lane & 7) + (mi >> 1) * 8) * C::PITCH + (mi & 1) * 16);
-  const uint32_t a_v = (uint32_t)((kT + (lane & 7) + (mi >> 1) * 8) * C::PITCH + (mi & 1) * 16);
+  const uint32_t y16 = (uint32_t)(((mi & 1) ^ (lane & 7)) << 4);
+  const uint32_t a_k = (uint32_t)(((lane & 7) + (mi >> 1) * 8) * C::ROW);
+  const uint32_t a_v = (uint32_t)((kT + (lane & 7) + (mi >> 1) * 8) * C::ROW);
 
 #pragma unroll
   for (int j = 0; j < kNS - 1; ++j) issue(j);
@@ -193,16 +208,16 @@ __global__ void __launch_bounds__(kNW * 32)
 #pragma unroll
     for (int s = 0; s < C::KSTEPS; ++s) {
       uint32_t b0, b1, b2, b3;
-      ldsm_x4(sb + a_k + s * 32, b0, b1, b2, b3);
+      ldsm_x4(sb + a_k + (((uint32_t)s * 32u) ^ y16), b0, b1, b2, b3);
       mma_bf16(s0, qa[s][0], 0u, qa[s][1], 0u, b0, b1);
       mma_bf16(s1, qa[s][0], 0u, qa[s][1], 0u, b2, b3);
     }
-    const int32_t* ids = ids_s + stage * kT;
+    const uint32_t valid = gid < 2 ? mask_s[stage] >> (2 * tig) : 0u;
     float sc[4];
-    sc[0] = (gid < 2 && ids[2 * tig] >= 0) ? s0[0] * qscale : -INFINITY;
-    sc[1] = (gid < 2 && ids[2 * tig + 1] >= 0) ? s0[1] * qscale : -INFINITY;
-    sc[2] = (gid < 2 && ids[8 + 2 * tig] >= 0) ? s1[0] * qscale : -INFINITY;
-    sc[3] = (gid < 2 && ids[9 + 2 * tig] >= 0) ? s1[1] * qscale : -INFINITY;
+    sc[0] = (valid & 1u) ? s0[0] * qscale : -INFINITY;
+    sc[1] = (valid & 2u) ? s0[1] * qscale : -INFINITY;
+    sc[2] = (valid & 0x100u) ? s1[0] * qscale : -INFINITY;
+    sc[3] = (valid & 0x200u) ? s1[1] * qscale : -INFINITY;
     const float smax = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
     // Rescale only when a score exceeds the running max by more than 2^8.
     if (__any_sync(0xFFFFFFFFu, smax > m_run + 8.f)) {
@@ -243,7 +258,7 @@ __global__ void __launch_bounds__(kNW * 32)
 #pragma unroll
       for (int mt = 0; mt < C::KSTEPS; ++mt) {
         uint32_t a0, a1, a2, a3;
-        ldsm_x4_t(sb + a_v + mt * 32, a0, a1, a2, a3);
+        ldsm_x4_t(sb + a_v + (((uint32_t)mt * 32u) ^ y16), a0, a1, a2, a3);
         mma_bf16(acc[mt], a0, a1, a2, a3, b0, b1);
       }
     }
