@@ -103,6 +103,7 @@ __global__ void __launch_bounds__(NT) block_topm_kernel(const float* __restrict_
 }
 
 constexpr int kTopmThreads = 128;
+constexpr int kTopmThreadsWide = 1024;
 constexpr int64_t kTopmSmemKeys = 32768;
 
 }  // namespace
@@ -132,11 +133,14 @@ cudaError_t launch_block_topm(const Shape& s, const float* scores, int32_t* bloc
                               cudaStream_t st) {
   const int in_smem = s.n_blk <= kTopmSmemKeys ? 1 : 0;
   const int smem = in_smem ? (int)(s.n_blk * 4) : 0;
-  auto kern = block_topm_kernel<kTopmThreads>;
+  // Few queries (decode): wide CTAs over the long block lists.
+  const bool wide = s.n_query < 2 * 148;
+  auto kern = wide ? block_topm_kernel<kTopmThreadsWide> : block_topm_kernel<kTopmThreads>;
+  const int nt = wide ? kTopmThreadsWide : kTopmThreads;
   cudaError_t e = ensure_smem((const void*)kern, smem);
   if (e != cudaSuccess) return e;
-  kern<<<(unsigned)s.n_query, kTopmThreads, smem, st>>>(scores, block_idx, block_scores, s.n_q, s.n_kv, s.B, s.n_blk,
-                                                        s.m, in_smem);
+  kern<<<(unsigned)s.n_query, nt, smem, st>>>(scores, block_idx, block_scores, s.n_q, s.n_kv, s.B, s.n_blk, s.m,
+                                              in_smem);
   return cudaGetLastError();
 }
 

@@ -54,9 +54,19 @@ struct AttnCfg {
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
-// 16-byte global -> shared copy through L2 only; pred == false zero-fills and reads nothing.
-__device__ __forceinline__ void cp_async16_u32(uint32_t dst, const void* src, bool pred) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(dst), "l"(src), "r"(pred ? 16 : 0) : "memory");
+// 16-byte global -> shared copy through L2 only; skip == true zero-fills and reads nothing.
+__device__ __forceinline__ void cp_async16_u32(uint32_t dst, const void* src, bool skip) {
+  asm volatile(
+      "{\n .reg .pred q;\n setp.ne.b32 q, %2, 0;\n cp.async.cg.shared.global [%0], [%1], 16, q;\n}\n" ::"r"(dst),
+      "l"(src), "r"((int)skip)
+      : "memory");
+}
+
+// 2^x on the special-function unit (the weights are re-rounded to a bf16 pair right after).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -144,7 +154,7 @@ __global__ void __launch_bounds__(kNW * 32)
   const int part = (lane / C::CH) & 1;  // 0 = K, 1 = V
   const int ch = lane % C::CH;
   const uint16_t* src_base = (part ? v : k) + ((int64_t)seq * n_kv * Hkv + g) * D + ch * 8;
-  const uint64_t tok_stride = (uint64_t)Hkv * D;
+  const uint32_t tok_stride = (uint32_t)(Hkv * D);
   int32_t* ids_s = reinterpret_cast<int32_t*>(smem + C::IDS_OFF) + warp * kNS * kT;
   uint32_t* mask_s = reinterpret_cast<uint32_t*>(smem + C::MASK_OFF) + warp * kNS;
 
@@ -176,7 +186,7 @@ __global__ void __launch_bounds__(kNW * 32)
         const int r = i * C::ROWS_PER_ITER + lane / (2 * C::CH);
         const int tok = C::ROWS_PER_ITER == 1 ? tk[i] : (lane / (2 * C::CH) ? tk[2 * i + 1] : tk[2 * i]);
         cp_async16_u32(sdst + r * C::ROW + ((ch ^ (r & 7)) << 4),
-                       src_base + (uint64_t)(uint32_t)(tok < 0 ? 0 : tok) * tok_stride, tok >= 0);
+                       src_base + (uint64_t)(uint32_t)max(tok, 0) * tok_stride, tok < 0);
       }
     }
     cp_async_commit();
@@ -240,21 +250,17 @@ __global__ void __launch_bounds__(kNW * 32)
     if (m_run != -INFINITY) {
       float pv[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) pv[i] = exp2f(sc[i] - m_run);
-      if (gid == 0) l_part += (pv[0] + pv[1]) + (pv[2] + pv[3]);
-      // P^T column 0 (lanes 0-3) = bf16(p); column 1 (lanes 4-7) = bf16(p - bf16(p)).
+      for (int i = 0; i < 4; ++i) pv[i] = fast_exp2(sc[i] - m_run);  // 0 for masked entries
+      l_part += (pv[0] + pv[1]) + (pv[2] + pv[3]);                    // only lanes 0-3 are summed at the end
+      // P^T column 0 (lanes 0-3) = bf16(p); column 1 (lanes 4-7) = bf16(p - bf16(p)); other lanes 0.
       const __nv_bfloat162 h01 = __floats2bfloat162_rn(pv[0], pv[1]);
       const __nv_bfloat162 h89 = __floats2bfloat162_rn(pv[2], pv[3]);
-      uint32_t b0 = 0u, b1 = 0u;
-      if (gid == 0) {
-        b0 = *reinterpret_cast<const uint32_t*>(&h01);
-        b1 = *reinterpret_cast<const uint32_t*>(&h89);
-      } else if (gid == 1) {
-        const __nv_bfloat162 l01 = __floats2bfloat162_rn(pv[0] - __low2float(h01), pv[1] - __high2float(h01));
-        const __nv_bfloat162 l89 = __floats2bfloat162_rn(pv[2] - __low2float(h89), pv[3] - __high2float(h89));
-        b0 = *reinterpret_cast<const uint32_t*>(&l01);
-        b1 = *reinterpret_cast<const uint32_t*>(&l89);
-      }
+      const __nv_bfloat162 l01 = __floats2bfloat162_rn(pv[0] - __low2float(h01), pv[1] - __high2float(h01));
+      const __nv_bfloat162 l89 = __floats2bfloat162_rn(pv[2] - __low2float(h89), pv[3] - __high2float(h89));
+      const uint32_t uh01 = *reinterpret_cast<const uint32_t*>(&h01), uh89 = *reinterpret_cast<const uint32_t*>(&h89);
+      const uint32_t ul01 = *reinterpret_cast<const uint32_t*>(&l01), ul89 = *reinterpret_cast<const uint32_t*>(&l89);
+      const uint32_t b0 = gid == 0 ? uh01 : ul01;  // lanes >= 8 hold p = 0, so both are 0 there
+      const uint32_t b1 = gid == 0 ? uh89 : ul89;
 #pragma unroll
       for (int mt = 0; mt < C::KSTEPS; ++mt) {
         uint32_t a0, a1, a2, a3;

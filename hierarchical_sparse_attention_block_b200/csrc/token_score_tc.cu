@@ -119,7 +119,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (jb0 > c_max) return;
   const int nb = (int)min((int64_t)kRun, c_max + 1 - jb0);
 
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5;
   uint8_t* sQ = smem + L::Q_OFF;
   uint8_t* sK = smem + L::K_OFF;
   int16_t* smap = reinterpret_cast<int16_t*>(smem + L::MAP_OFF);

@@ -25,6 +25,7 @@ namespace {
 constexpr int kScoreThreads = 256;
 constexpr int kMaxSlotsPerCta = 64;
 constexpr int kSelectThreads = 256;
+constexpr int kSelectThreadsWide = 1024;
 constexpr int kSelectSmemKeys = 49152;  // 192 KiB of keys
 
 template <int D>
@@ -217,11 +218,13 @@ cudaError_t launch_token_select(const Shape& s, const uint32_t* keys, const int3
   if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
   int log2B = 0;
   while ((1 << log2B) < s.B) ++log2B;
-  auto kern = token_select_kernel<kSelectThreads>;
+  // Few queries (decode): one wide CTA per query keeps the selection from being latency-bound.
+  const bool wide = nq < 2 * 148;
+  auto kern = wide ? token_select_kernel<kSelectThreadsWide> : token_select_kernel<kSelectThreads>;
+  const int nt = wide ? kSelectThreadsWide : kSelectThreads;
   cudaError_t e = ensure_smem((const void*)kern, smem);
   if (e != cudaSuccess) return e;
-  kern<<<(unsigned)nq, kSelectThreads, smem, st>>>(keys, block_idx, slots, token_idx, token_scores, s.n_q, log2B, s.k,
-                                                   q0, in_smem);
+  kern<<<(unsigned)nq, nt, smem, st>>>(keys, block_idx, slots, token_idx, token_scores, s.n_q, log2B, s.k, q0, in_smem);
   return cudaGetLastError();
 }
 
