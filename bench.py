@@ -91,7 +91,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
         except Exception:
@@ -281,7 +281,15 @@ def run_ours(a, rank, world, local_rank):
     torch.cuda.synchronize()
     evs = [new_events() for _ in range(a.steps)]
     g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else 0) as clk:
+    clk = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
+    with clk:
+        # short timed regions (decode) are bracketed by extra untimed steps so the
+        # sampler sees the GPU under this load
+        t_pad = time.perf_counter()
+        while time.perf_counter() - t_pad < 0.3:
+            flush.zero_()
+            step(new_events())
+            torch.cuda.synchronize()
         g0.record(st)
         for s in range(a.steps):
             flush.zero_()
@@ -355,8 +363,9 @@ def run_ours(a, rank, world, local_rank):
 def run_e2e(a, hs, w, p, inp, dev, st, world):
     """The same metric through hisa_forward with host-resident inputs: every step copies its
     inputs from pinned host memory and reads the outputs back.  For prefill every input is a
-    step input; for decode the caches (k_idx, K, V) stay resident on the device, as in a
-    serving loop, and the step inputs are the new queries (q_idx, Q)."""
+    step input (hisa_forward); for decode the caches (k_idx, K, V) and their block keys stay
+    resident on the device, as in a serving loop, the step inputs are the new queries (q_idx,
+    Q), and hisa_forward_cached refreshes only the newest block."""
     import torch
 
     names = ["q_idx", "q"] if w.n_q == 1 else ["q_idx", "k_idx", "q", "k", "v"]
@@ -371,11 +380,20 @@ def run_e2e(a, hs, w, p, inp, dev, st, world):
     h2d = sum(v.numel() * v.element_size() for v in host.values())
     d2h = o.numel() * 2 + lse.numel() * 4
 
+    decode = w.n_q == 1
+    bk = torch.empty((w.batch, w.n_blk, w.d_idx), dtype=torch.float32, device=dev) if decode else None
+    if decode:  # the cache's block keys are pooled once and persist between decode steps
+        hs.hisa_block_pool(p, d_in["k_idx"], bk, stream=st)
+
     def one():
         for k in host:
             d_in[k].copy_(host[k], non_blocking=True)
-        hs.hisa_forward(p, d_in["q_idx"], d_in["k_idx"], d_in["q"], d_in["k"], d_in["v"], o, lse, None, None, None,
-                        ws, stream=st)
+        if decode:
+            hs.hisa_forward_cached(p, d_in["q_idx"], d_in["k_idx"], bk, w.n_blk - 1, d_in["q"], d_in["k"], d_in["v"],
+                                   o, lse, None, None, None, ws, stream=st)
+        else:
+            hs.hisa_forward(p, d_in["q_idx"], d_in["k_idx"], d_in["q"], d_in["k"], d_in["v"], o, lse, None, None,
+                            None, ws, stream=st)
         h_o.copy_(o, non_blocking=True)
         h_lse.copy_(lse, non_blocking=True)
 

@@ -23,7 +23,7 @@ EXPORTS = (
     "hisa_block_pool", "hisa_block_topm_workspace_size", "hisa_block_topm", "hisa_token_topk_workspace_size",
     "hisa_token_topk", "hisa_sparse_attn_workspace_size", "sparse_attn_fwd", "hisa_forward_workspace_size",
     "hisa_forward", "hisa_flat_topk_workspace_size", "hisa_flat_topk", "hisa_status_string",
-    "hisa_last_cuda_error", "hisa_version", "hisa_token_topk_noalloc",
+    "hisa_last_cuda_error", "hisa_version", "hisa_token_topk_noalloc", "hisa_forward_cached",
 )
 
 
@@ -67,6 +67,7 @@ def _load():
         "hisa_flat_topk_workspace_size": [pp, sz, sz],
         "hisa_flat_topk": [pp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
         "hisa_token_topk_noalloc": [pp, vp, vp, vp, vp, vp, vp, vp],
+        "hisa_forward_cached": [pp, vp, vp, vp, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -189,6 +190,17 @@ def hisa_forward(p, q_idx, k_idx, q, k, v, o, lse=None, block_idx_out=None, toke
     _check("hisa_forward", _lib.hisa_forward(ctypes.byref(p), _ptr(q_idx), _ptr(k_idx), _ptr(q), _ptr(k), _ptr(v),
                                              _ptr(o), _ptr(lse), _ptr(block_idx_out), _ptr(token_idx_out),
                                              _ptr(dev_status), _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def hisa_forward_cached(p, q_idx, k_idx, block_keys, refresh_begin, q, k, v, o, lse=None, block_idx_out=None,
+                        token_idx_out=None, dev_status=None, workspace=None, stream=None):
+    if workspace is None:
+        workspace = _workspace(hisa_forward_workspace_size(p), q_idx.device)
+    _check("hisa_forward_cached",
+           _lib.hisa_forward_cached(ctypes.byref(p), _ptr(q_idx), _ptr(k_idx), _ptr(block_keys), int(refresh_begin),
+                                    _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(block_idx_out),
+                                    _ptr(token_idx_out), _ptr(dev_status), _ptr(workspace), workspace.numel(),
+                                    _stream(stream)))
 
 
 def hisa_flat_topk_workspace_size(p):

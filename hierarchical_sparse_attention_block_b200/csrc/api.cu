@@ -280,6 +280,37 @@ hisa_status_t hisa_forward_workspace_size(const hisa_params_t* params, size_t* b
   return HISA_OK;
 }
 
+namespace {
+// Steps 1-6; block keys in bk, pooled for blocks [refresh_begin, n_blk).
+hisa_status_t forward_impl(const Shape& s, const FwdLayout& L, const void* q_idx, const void* k_idx, float* bk,
+                           int64_t refresh_begin, const void* q, const void* k, const void* v, void* o, float* lse,
+                           int32_t* block_idx_out, int32_t* token_idx_out, int32_t* dev_status, uint8_t* ws,
+                           size_t workspace_bytes, cudaStream_t stream) {
+  int32_t* blk = block_idx_out ? block_idx_out : reinterpret_cast<int32_t*>(ws + L.block_idx);
+  int32_t* tok = token_idx_out ? token_idx_out : reinterpret_cast<int32_t*>(ws + L.token_idx);
+  cudaError_t e = hisa::launch_block_pool(s, k_idx, refresh_begin, s.n_blk, bk, stream);
+  if (e != cudaSuccess) return hisa::cuda_fail(e);
+  hisa_status_t rc = hisa::run_block_stage(s, q_idx, bk, blk, nullptr, dev_status, ws + L.blk_stage, stream);
+  if (rc != HISA_OK) return rc;
+  rc = hisa::run_token_stage(s, q_idx, k_idx, blk, s.m, tok, nullptr, dev_status, ws + L.keys,
+                             workspace_bytes - L.keys, stream);
+  if (rc != HISA_OK) return rc;
+  const int splits = hisa::attn_pick_splits(s);
+  return hisa::cuda_fail(hisa::launch_sparse_attn(s, q, k, v, tok, o, lse, dev_status, splits, ws + L.attn, stream));
+}
+
+hisa_status_t check_forward_args(const void* q_idx, const void* k_idx, const void* q, const void* k, const void* v,
+                                 void* o, float* lse, int32_t* block_idx_out, int32_t* token_idx_out) {
+  const void* ptrs[] = {q_idx, k_idx, q, k, v, o};
+  for (const void* p : ptrs)
+    if (!p || !hisa::aligned16(p)) return HISA_ERR_INVALID_ARG;
+  if ((lse && !hisa::aligned16(lse)) || (block_idx_out && !hisa::aligned16(block_idx_out)) ||
+      (token_idx_out && !hisa::aligned16(token_idx_out)))
+    return HISA_ERR_INVALID_ARG;
+  return HISA_OK;
+}
+}  // namespace
+
 hisa_status_t hisa_forward(const hisa_params_t* params, const void* q_idx, const void* k_idx, const void* q,
                            const void* k, const void* v, void* o, float* lse, int32_t* block_idx_out,
                            int32_t* token_idx_out, int32_t* dev_status, void* workspace, size_t workspace_bytes,
@@ -287,28 +318,30 @@ hisa_status_t hisa_forward(const hisa_params_t* params, const void* q_idx, const
   Shape s;
   hisa_status_t rc = hisa::make_shape(params, true, true, &s);
   if (rc != HISA_OK) return rc;
-  const void* ptrs[] = {q_idx, k_idx, q, k, v, o};
-  for (const void* p : ptrs)
-    if (!p || !hisa::aligned16(p)) return HISA_ERR_INVALID_ARG;
-  if ((lse && !hisa::aligned16(lse)) || (block_idx_out && !hisa::aligned16(block_idx_out)) ||
-      (token_idx_out && !hisa::aligned16(token_idx_out)))
-    return HISA_ERR_INVALID_ARG;
+  rc = check_forward_args(q_idx, k_idx, q, k, v, o, lse, block_idx_out, token_idx_out);
+  if (rc != HISA_OK) return rc;
   const FwdLayout L = fwd_layout(s);
   if (!workspace || !hisa::aligned16(workspace) || workspace_bytes < L.total) return HISA_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  float* bk = reinterpret_cast<float*>(ws + L.bk);
-  int32_t* blk = block_idx_out ? block_idx_out : reinterpret_cast<int32_t*>(ws + L.block_idx);
-  int32_t* tok = token_idx_out ? token_idx_out : reinterpret_cast<int32_t*>(ws + L.token_idx);
+  return forward_impl(s, L, q_idx, k_idx, reinterpret_cast<float*>(ws + L.bk), 0, q, k, v, o, lse, block_idx_out,
+                      token_idx_out, dev_status, ws, workspace_bytes, stream);
+}
 
-  cudaError_t e = hisa::launch_block_pool(s, k_idx, 0, s.n_blk, bk, stream);
-  if (e != cudaSuccess) return hisa::cuda_fail(e);
-  rc = hisa::run_block_stage(s, q_idx, bk, blk, nullptr, dev_status, ws + L.blk_stage, stream);
+hisa_status_t hisa_forward_cached(const hisa_params_t* params, const void* q_idx, const void* k_idx,
+                                  float* block_keys, int64_t refresh_begin, const void* q, const void* k,
+                                  const void* v, void* o, float* lse, int32_t* block_idx_out, int32_t* token_idx_out,
+                                  int32_t* dev_status, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  Shape s;
+  hisa_status_t rc = hisa::make_shape(params, true, true, &s);
   if (rc != HISA_OK) return rc;
-  rc = hisa::run_token_stage(s, q_idx, k_idx, blk, s.m, tok, nullptr, dev_status, ws + L.keys,
-                             workspace_bytes - L.keys, stream);
+  rc = check_forward_args(q_idx, k_idx, q, k, v, o, lse, block_idx_out, token_idx_out);
   if (rc != HISA_OK) return rc;
-  const int splits = hisa::attn_pick_splits(s);
-  return hisa::cuda_fail(hisa::launch_sparse_attn(s, q, k, v, tok, o, lse, dev_status, splits, ws + L.attn, stream));
+  if (!block_keys || !hisa::aligned16(block_keys)) return HISA_ERR_INVALID_ARG;
+  if (refresh_begin < 0 || refresh_begin > s.n_blk) return HISA_ERR_INVALID_ARG;
+  const FwdLayout L = fwd_layout(s);
+  if (!workspace || !hisa::aligned16(workspace) || workspace_bytes < L.total) return HISA_ERR_WORKSPACE;
+  return forward_impl(s, L, q_idx, k_idx, block_keys, refresh_begin, q, k, v, o, lse, block_idx_out, token_idx_out,
+                      dev_status, static_cast<uint8_t*>(workspace), workspace_bytes, stream);
 }
 
 hisa_status_t hisa_flat_topk_workspace_size(const hisa_params_t* params, size_t* min_bytes, size_t* preferred_bytes) {

@@ -115,18 +115,22 @@ __global__ void __launch_bounds__(kNW * 32)
   const int gid = lane >> 2, tig = lane & 3;
   const int32_t* list = token_idx + qg * topk;
 
-  // Entries past the last valid one are skipped.
-  int last = -1;
-  for (int e = threadIdx.x; e < topk; e += kNW * 32)
-    if (list[e] >= 0) last = e;
+  // One work item per (query, head): entries past the last valid one are skipped.  A list
+  // split across CTAs (few queries) is cut at fixed positions; -1 entries are masked.
+  int n_use = topk;
+  if (splits == 1) {
+    int last = -1;
+    for (int e = threadIdx.x; e < topk; e += kNW * 32)
+      if (list[e] >= 0) last = e;
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) last = max(last, __shfl_xor_sync(0xFFFFFFFFu, last, off));
-  if (lane == 0) s_last[warp] = last;
-  __syncthreads();
-  int n_use = -1;
+    for (int off = 16; off > 0; off >>= 1) last = max(last, __shfl_xor_sync(0xFFFFFFFFu, last, off));
+    if (lane == 0) s_last[warp] = last;
+    __syncthreads();
+    n_use = -1;
 #pragma unroll
-  for (int w = 0; w < kNW; ++w) n_use = max(n_use, s_last[w]);
-  n_use += 1;
+    for (int w = 0; w < kNW; ++w) n_use = max(n_use, s_last[w]);
+    n_use += 1;
+  }
 
   int per = (n_use + splits - 1) / splits;
   per = (per + kT - 1) / kT * kT;
@@ -361,9 +365,13 @@ cudaError_t launch_d(const Shape& s, const void* q, const void* k, const void* v
 
 }  // namespace
 
+#ifndef HISA_ATTN_SPLIT_TARGET
+#define HISA_ATTN_SPLIT_TARGET (148 * 8)
+#endif
+
 int attn_pick_splits(const Shape& s) {
   const int64_t units = s.n_query * s.H;
-  const int64_t target = 148 * 8;
+  const int64_t target = HISA_ATTN_SPLIT_TARGET;
   if (units >= target) return 1;
   int64_t sp = (target + units - 1) / units;
   const int64_t max_sp = (s.k + 127) / 128;  // keep >= ~128 entries per split

@@ -145,6 +145,18 @@ hisa_status_t hisa_forward(const hisa_params_t* params, const void* q_idx, const
                            int32_t* token_idx_out, int32_t* dev_status, void* workspace, size_t workspace_bytes,
                            cudaStream_t stream);
 
+/* Steps 1-6 with caller-owned block keys that persist between calls (decode
+ * serving, [QB] "HISA的關鍵優勢在於": the KV cache is unchanged, so the pooled
+ * block keys of the cache can be kept).  block_keys [b][ceil(n_kv/B)][d_idx]
+ * fp32 is read for every block and first rewritten for blocks
+ * [refresh_begin, ceil(n_kv/B)): 0 pools everything (e.g. after a prefill),
+ * (n_kv - 1) / B refreshes only the block the newest token entered.  Results
+ * equal hisa_forward's.  Workspace: hisa_forward_workspace_size bytes. */
+hisa_status_t hisa_forward_cached(const hisa_params_t* params, const void* q_idx, const void* k_idx,
+                                  float* block_keys, int64_t refresh_begin, const void* q, const void* k,
+                                  const void* v, void* o, float* lse, int32_t* block_idx_out, int32_t* token_idx_out,
+                                  int32_t* dev_status, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* The flat token indexer the two-level one replaces ([IP] 1.1 item 1; [QB]
  * "兩步消除上下文索引瓶頸"): token_idx[s][i] = the min(k, p_i+1) best tokens
  * t <= p_i of the whole sequence.  Same output format as hisa_token_topk;

@@ -288,3 +288,38 @@ def test_decode_4x1m_m_sweep_sampled(hs, oracle_lib):
 def test_tolerance_constants():
     assert (ATOL, RTOL) == (2e-3, 1e-2)
     assert math.isclose(1 / math.sqrt(128), 0.08838834764831845)
+
+
+@pytest.mark.parametrize("n_kv,block", [(1000, 64), (1025, 64), (777, 16)])
+def test_forward_cached_decode_loop(hs, oracle_lib, n_kv, block):
+    """hisa_forward_cached: refreshing only the block the newest token entered gives the same
+    result as hisa_forward on the whole cache, and as the oracle."""
+    w = Workload("decode_loop", 3, 1, n_kv, 128, block, 6, 200, 4, 2, 64, needles=2)
+    inp = full_inputs(w)
+    dev = _dev(inp)
+    ref = run_forward(hs, w, dev)
+    # block keys of the cache before the newest token (n_kv - 1 tokens), pooled once
+    prev = w.with_(n_kv=n_kv - 1)
+    bk = torch.full((w.batch, w.n_blk, w.d_idx), 9.0, dtype=torch.float32, device="cuda")
+    k_prev = dev["k_idx"][:, : n_kv - 1].contiguous()
+    tmp = torch.empty((w.batch, prev.n_blk, w.d_idx), dtype=torch.float32, device="cuda")
+    hs.hisa_block_pool(hs.params_of(prev), k_prev, tmp)
+    bk[:, : prev.n_blk] = tmp  # a block the newest token opens still holds 9.0 here
+    p = hs.params_of(w)
+    o = torch.empty_like(ref["o"])
+    lse = torch.empty_like(ref["lse"])
+    blk = torch.empty_like(ref["block_idx"])
+    tok = torch.empty_like(ref["token_idx"])
+    hs.hisa_forward_cached(p, dev["q_idx"], dev["k_idx"], bk, (n_kv - 1) // block, dev["q"], dev["k"], dev["v"], o,
+                           lse, blk, tok)
+    torch.cuda.synchronize()
+    assert torch.equal(blk, ref["block_idx"]) and torch.equal(tok, ref["token_idx"])
+    assert torch.equal(o, ref["o"]) and torch.equal(lse, ref["lse"])
+    oref = oracle_lib.run(w, inp)
+    assert np.array_equal(tok.cpu().numpy().reshape(w.batch, w.top_k), oref["token_idx"])
+    assert_close(o.float().cpu().numpy().reshape(w.batch, w.n_heads, w.d_head), oref["o"], "o")
+    # refresh from block 0 recomputes every key
+    bk.fill_(5.0)
+    hs.hisa_forward_cached(p, dev["q_idx"], dev["k_idx"], bk, 0, dev["q"], dev["k"], dev["v"], o, lse, blk, tok)
+    torch.cuda.synchronize()
+    assert torch.equal(tok, ref["token_idx"]) and torch.equal(o, ref["o"])
