@@ -86,52 +86,65 @@ __device__ SelectResult radix_select(KeyFn keys, int n, int K, SelectShared<NT>&
 __device__ __forceinline__ SelectResult select_all_nonzero() { return SelectResult{0u, 0xFFFFFFFFu, 0}; }
 
 // Emit the taken positions in ascending order: emit(i, rank) for each taken i.
-// Returns the number emitted.  All NT threads must call.
+// Returns the number emitted.  All NT threads must call.  Each warp owns one
+// contiguous range of positions (read 32 at a time, so shared-memory reads stay
+// conflict-free); a first sweep counts what each warp takes, one CTA scan turns
+// the counts into offsets, and a second sweep emits.  Ties at the threshold are
+// taken in position order across warps.
 template <int NT, class KeyFn, class Emit>
 __device__ int emit_selected(KeyFn keys, int n, SelectResult r, SelectShared<NT>& sm, Emit emit) {
   constexpr int NW = NT / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const uint32_t below = (1u << lane) - 1u;
-  int base_sel = 0, base_eq = 0;
-  for (int c0 = 0; c0 < n; c0 += NT) {
-    const int i = c0 + threadIdx.x;
-    const uint32_t km = (i < n ? keys(i) : 0u) & r.mask;
-    const bool gt = i < n && km > r.prefix;
-    const bool eq = i < n && km == r.prefix;
-    bool sel;
-    if (r.take_eq < 0) {
-      sel = gt || eq;
-    } else if (r.take_eq == 0) {
-      sel = gt;
-    } else {
-      const uint32_t be = __ballot_sync(0xFFFFFFFFu, eq);
-      if (lane == 0) sm.warp_cnt[warp][0] = __popc(be);
-      __syncthreads();
-      int pre = base_eq, tot = 0;
-#pragma unroll
-      for (int w = 0; w < NW; ++w) {
-        const int v = (int)sm.warp_cnt[w][0];
-        pre += w < warp ? v : 0;
-        tot += v;
-      }
-      sel = gt || (eq && pre + __popc(be & below) < r.take_eq);
-      base_eq += tot;
-    }
-    const uint32_t bs = __ballot_sync(0xFFFFFFFFu, sel);
-    if (lane == 0) sm.warp_cnt[warp][1] = __popc(bs);
-    __syncthreads();
-    int pre = base_sel, tot = 0;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) {
-      const int v = (int)sm.warp_cnt[w][1];
-      pre += w < warp ? v : 0;
-      tot += v;
-    }
-    if (sel) emit(i, pre + __popc(bs & below));
-    base_sel += tot;
-    __syncthreads();
+  const int span = ((n + NW - 1) / NW + 31) & ~31;  // positions per warp, a multiple of 32
+  const int w0 = min(warp * span, n), w1 = min(w0 + span, n);
+  auto classify = [&](int i, bool& gt, bool& eq) {
+    const uint32_t km = (i < w1 ? keys(i) : 0u) & r.mask;
+    gt = i < w1 && km > r.prefix;
+    eq = i < w1 && km == r.prefix;
+  };
+  // sweep 1: how many keys above the threshold and at it does this warp hold?
+  int n_gt = 0, n_eq = 0;
+  for (int c0 = w0; c0 < w1; c0 += 32) {
+    bool gt, eq;
+    classify(c0 + lane, gt, eq);
+    n_gt += __popc(__ballot_sync(0xFFFFFFFFu, gt));
+    n_eq += __popc(__ballot_sync(0xFFFFFFFFu, eq));
   }
-  return base_sel;
+  if (lane == 0) {
+    sm.warp_cnt[warp][0] = (uint32_t)n_gt;
+    sm.warp_cnt[warp][1] = (uint32_t)n_eq;
+  }
+  __syncthreads();
+  // offsets of this warp: keys taken and ties seen before it
+  const int take_eq = r.take_eq < 0 ? 0x7FFFFFFF : r.take_eq;
+  int eq_before = 0, taken_before = 0, total = 0, eqb = 0;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) {
+    const int g = (int)sm.warp_cnt[w][0], e = (int)sm.warp_cnt[w][1];
+    const int t = g + max(0, min(e, take_eq - eqb));
+    if (w < warp) {
+      taken_before += t;
+      eq_before += e;
+    }
+    total += t;
+    eqb += e;
+  }
+  // sweep 2: emit in order
+  int rank = taken_before, eq_seen = eq_before;
+  for (int c0 = w0; c0 < w1; c0 += 32) {
+    const int i = c0 + lane;
+    bool gt, eq;
+    classify(i, gt, eq);
+    const uint32_t be = __ballot_sync(0xFFFFFFFFu, eq);
+    const bool sel = gt || (eq && eq_seen + __popc(be & below) < take_eq);
+    const uint32_t bs = __ballot_sync(0xFFFFFFFFu, sel);
+    if (sel) emit(i, rank + __popc(bs & below));
+    rank += __popc(bs);
+    eq_seen += __popc(be);
+  }
+  __syncthreads();
+  return total;
 }
 
 // Count of nonzero keys, CTA-wide (all threads get the result).

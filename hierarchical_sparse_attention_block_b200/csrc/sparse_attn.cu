@@ -217,15 +217,24 @@ __global__ void __launch_bounds__(kNW * 32)
     const int stage = j % kNS;
     const uint32_t sb = wbase + stage * C::STAGE;
 
-    // scores of tokens 2tig, 2tig+1 (first MMA) and 8+2tig, 9+2tig (second), in lanes 0-7
+    // scores of tokens 2tig, 2tig+1 (first MMA) and 8+2tig, 9+2tig (second), in lanes 0-7;
+    // even and odd k-steps accumulate separately to halve the dependent MMA chains
     float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+    float t0[4] = {0.f, 0.f, 0.f, 0.f}, t1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int s = 0; s < C::KSTEPS; ++s) {
-      uint32_t b0, b1, b2, b3;
+    for (int s = 0; s < C::KSTEPS; s += 2) {
+      uint32_t b0, b1, b2, b3, c0, c1, c2, c3;
       ldsm_x4(sb + a_k + (((uint32_t)s * 32u) ^ y16), b0, b1, b2, b3);
+      ldsm_x4(sb + a_k + (((uint32_t)(s + 1) * 32u) ^ y16), c0, c1, c2, c3);
       mma_bf16(s0, qa[s][0], 0u, qa[s][1], 0u, b0, b1);
       mma_bf16(s1, qa[s][0], 0u, qa[s][1], 0u, b2, b3);
+      mma_bf16(t0, qa[s + 1][0], 0u, qa[s + 1][1], 0u, c0, c1);
+      mma_bf16(t1, qa[s + 1][0], 0u, qa[s + 1][1], 0u, c2, c3);
     }
+    s0[0] += t0[0];
+    s0[1] += t0[1];
+    s1[0] += t1[0];
+    s1[1] += t1[1];
     const uint32_t valid = gid < 2 ? mask_s[stage] >> (2 * tig) : 0u;
     float sc[4];
     sc[0] = (valid & 1u) ? s0[0] * qscale : -INFINITY;
