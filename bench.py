@@ -46,6 +46,7 @@ def _args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-flat", action="store_true", help="skip the flat-indexer comparator")
+    ap.add_argument("--no-clock", action="store_true", help="no clock sampling (and no padding steps), for profiling")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
     ap.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE",
                     help="override a workload field, e.g. --set n_q=32768 --set n_kv=32768")
@@ -82,12 +83,15 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, enabled: bool = True):
         self.gpu = gpu_index
+        self.enabled = enabled
         self.proc = None
         self.lines = []
 
     def __enter__(self):
+        if not self.enabled:
+            return self
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
@@ -281,12 +285,12 @@ def run_ours(a, rank, world, local_rank):
     torch.cuda.synchronize()
     evs = [new_events() for _ in range(a.steps)]
     g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clk = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
+    clk = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else 0, enabled=not a.no_clock)
     with clk:
         # short timed regions (decode) are bracketed by extra untimed steps so the
         # sampler sees the GPU under this load
         t_pad = time.perf_counter()
-        while time.perf_counter() - t_pad < 0.3:
+        while not a.no_clock and time.perf_counter() - t_pad < 0.3:
             flush.zero_()
             step(new_events())
             torch.cuda.synchronize()
@@ -434,22 +438,32 @@ def oracle_sample(w, seconds: float, device_inputs=None):
     bkeys = np.stack([O.block_pool(inp["k_idx"][s], w.block) for s in range(w.batch)])
     pool_s = time.perf_counter() - t0
     nq = w.batch * w.n_q
-    n = 8
-    done, elapsed = 0, 0.0
+    done, elapsed, reps = 0, 0.0, 0
     rng = np.random.default_rng(0)
-    while elapsed < seconds and done < nq:
-        ids = np.sort(rng.choice(nq, size=min(n, nq), replace=False)).astype(np.int64)
-        t0 = time.perf_counter()
-        O.run(w, inp, query_ids=ids, block_keys=bkeys)
-        elapsed += time.perf_counter() - t0
-        done += len(ids)
-        n = min(n * 2, 4096)
+    if nq <= 8192:
+        # small workloads: whole passes over every query
+        while reps == 0 or elapsed < seconds:
+            t0 = time.perf_counter()
+            O.run(w, inp, block_keys=bkeys)
+            elapsed += time.perf_counter() - t0
+            done += nq
+            reps += 1
+        what = f"{reps} full pass(es) over all {nq} queries"
+    else:
+        n = 8
+        while elapsed < seconds:
+            ids = np.sort(rng.choice(nq, size=min(n, nq), replace=False)).astype(np.int64)
+            t0 = time.perf_counter()
+            O.run(w, inp, query_ids=ids, block_keys=bkeys)
+            elapsed += time.perf_counter() - t0
+            done += len(ids)
+            n = min(n * 2, 4096)
+        what = f"{done} query evaluations drawn uniformly over the {nq} positions"
     per_q = elapsed / done
     total_s = pool_s + per_q * nq
     return {"value": nq / total_s, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": f"{done} of {nq} queries drawn uniformly over positions, full path (pooling, top-m, top-k, "
-                      f"attention in fp64), plus pooling of every block; {elapsed + pool_s:.1f} s of CPU time, "
-                      f"scaled to the whole workload"}
+            "sample": f"{what}, full path (top-m, top-k, attention in fp64) plus pooling of every block; "
+                      f"{elapsed + pool_s:.1f} s of CPU time, scaled to the whole workload"}
 
 
 def oracle_sample_rows(w, seconds: float):
