@@ -47,6 +47,8 @@ def _args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-flat", action="store_true", help="skip the flat-indexer comparator")
     ap.add_argument("--no-clock", action="store_true", help="no clock sampling (and no padding steps), for profiling")
+    ap.add_argument("--graph", choices=["auto", "on", "off"], default="auto",
+                    help="replay each step from a CUDA graph (auto: for decode workloads)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU time of the oracle sample")
     ap.add_argument("--set", action="append", default=[], metavar="FIELD=VALUE",
                     help="override a workload field, e.g. --set n_q=32768 --set n_kv=32768")
@@ -180,15 +182,16 @@ def indexer_bytes(w, counts):
             + nq * w.d_idx * 2 + nq * (w.top_m + w.top_k) * 4)
 
 
-def _profile_traffic(kernel_file: str, summary_name: str):
-    """DRAM bytes per launch from the committed ncu summary, or None when the kernel changed since."""
+def _profile_traffic(kernel_file: str, summary_name: str, workload_name: str):
+    """DRAM bytes per launch from the committed ncu summary of this workload, or None when there
+    is none or the kernel changed since it was taken."""
     path = os.path.join(ROOT, "profiles", summary_name)
     src = os.path.join(ROOT, "hierarchical_sparse_attention_block_b200", "csrc", kernel_file)
     try:
         with open(path) as f:
             j = json.load(f)
         sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-        if j.get("source_sha256_16") != sha:
+        if j.get("source_sha256_16") != sha or j.get("workload") != workload_name:
             return None
         return j.get("dram_bytes_per_launch_full_workload")
     except Exception:
@@ -207,7 +210,8 @@ def run_ours(a, rank, world, local_rank):
     p = hs.params_of(w)
     inp = sd.device_inputs(w, device=dev)
     torch.cuda.synchronize()
-    st = torch.cuda.current_stream()
+    st = torch.cuda.Stream(device=dev)  # a side stream: CUDA graphs cannot be captured on the default one
+    torch.cuda.set_stream(st)
 
     nq = w.batch * w.n_q
     bk = torch.empty((w.batch, w.n_blk, w.d_idx), dtype=torch.float32, device=dev)
@@ -258,6 +262,34 @@ def run_ours(a, rank, world, local_rank):
     torch.cuda.synchronize()
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} after warm-up")
+
+    # Decode steps are microseconds long: replay them from a CUDA graph (one graph per
+    # stage, so the stage events stay outside the graphs).
+    use_graph = a.graph == "on" or (a.graph == "auto" and decode)
+    if use_graph:
+        calls = [
+            lambda: hs.hisa_block_pool(p, inp["k_idx"], bk, pool_begin, -1, stream=st),
+            lambda: hs.hisa_block_topm(p, inp["q_idx"], bk, blk, None, status, ws_topm, stream=st),
+            lambda: hs.hisa_token_topk(p, inp["q_idx"], inp["k_idx"], blk, tok, None, status, ws_tok, stream=st),
+            lambda: hs.sparse_attn_fwd(p, inp["q"], inp["k"], inp["v"], tok, o, lse, status, ws_attn, stream=st),
+        ]
+        graphs = []
+        for fn in calls:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=st):
+                fn()
+            graphs.append(g)
+        torch.cuda.synchronize()
+
+        def step(ev):  # noqa: F811
+            for j, g in enumerate(graphs):
+                ev[j].record(st)
+                g.replay()
+            ev[4].record(st)
+
+        for _ in range(a.warmup):
+            step(new_events())
+        torch.cuda.synchronize()
 
     # the indexer alone and the flat comparator, for the speedup figure (outside the timed steps)
     comp = {}
@@ -342,9 +374,10 @@ def run_ours(a, rank, world, local_rank):
                      "frac": achieved / hbm_gbs, "peak_kind": peak_kind,
                      "frac_of_nominal_8tbs": achieved / 8000.0,
                      "algorithmic_bytes_per_launch": a_bytes,
-                     "traffic": _profile_traffic("sparse_attn.cu", "sparse_attn_prefill_64k.json")},
+                     "traffic": _profile_traffic("sparse_attn.cu", f"sparse_attn_{w.name}.json", w.name)},
         "stages_ms": {n: statistics.mean(v) for n, v in stage_ms.items()},
         "pool_in_step": "newest block only (cache block keys persist)" if decode else "every block",
+        "cuda_graph": use_graph,
         "pool_setup_ms": pool_setup_ms,
         "indexer_ms": idx_ms, "indexer_queries_per_s": nq / (idx_ms * 1e-3),
         "tokens_per_s": counts["k_eff"] / (ms * 1e-3),

@@ -323,3 +323,44 @@ def test_forward_cached_decode_loop(hs, oracle_lib, n_kv, block):
     hs.hisa_forward_cached(p, dev["q_idx"], dev["k_idx"], bk, 0, dev["q"], dev["k"], dev["v"], o, lse, blk, tok)
     torch.cuda.synchronize()
     assert torch.equal(tok, ref["token_idx"]) and torch.equal(o, ref["o"])
+
+
+def test_decode_step_in_a_cuda_graph(hs, oracle_lib):
+    """A decode step (newest-block refresh + steps 2-6) captured once in a CUDA graph and
+    replayed gives the same outputs as the eager calls, for fresh query contents."""
+    w = Workload("graph_decode", 8, 1, 3000, 128, 64, 8, 256, 4, 4, 128)
+    inp = full_inputs(w)
+    dev = _dev(inp)
+    p = hs.params_of(w)
+    bk = torch.empty((w.batch, w.n_blk, w.d_idx), dtype=torch.float32, device="cuda")
+    hs.hisa_block_pool(p, dev["k_idx"], bk)
+    ws = torch.empty(hs.hisa_forward_workspace_size(p), dtype=torch.uint8, device="cuda")
+    o = torch.empty((w.batch, 1, w.n_heads, w.d_head), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((w.batch, 1, w.n_heads), dtype=torch.float32, device="cuda")
+    tok = torch.empty((w.batch, 1, w.top_k), dtype=torch.int32, device="cuda")
+    q_idx, q = dev["q_idx"].clone(), dev["q"].clone()
+
+    def step():
+        hs.hisa_forward_cached(p, q_idx, dev["k_idx"], bk, w.n_blk - 1, q, dev["k"], dev["v"], o, lse, None, tok,
+                               None, ws)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        step()  # warm-up: one-time kernel attributes are set outside the capture
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    for trial in range(2):
+        # new query contents each replay (a different sequence's queries rolled in)
+        q_idx.copy_(dev["q_idx"].roll(trial + 1, dims=0))
+        q.copy_(dev["q"].roll(trial + 1, dims=0))
+        g.replay()
+        torch.cuda.synchronize()
+        got_o, got_tok = o.clone(), tok.clone()
+        step()
+        torch.cuda.synchronize()
+        assert torch.equal(got_tok, tok) and torch.equal(got_o, o)
+    del g
