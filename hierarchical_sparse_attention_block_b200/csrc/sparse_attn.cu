@@ -28,6 +28,10 @@
 #include "common.cuh"
 #include "internal.h"
 
+// Tile shape of the prefill kernel: list entries per warp tile and pipeline stages.
+#ifndef HISA_ATTN_TILE
+#define HISA_ATTN_TILE 16
+#endif
 #ifndef HISA_ATTN_STAGES
 #define HISA_ATTN_STAGES 2
 #endif
@@ -35,16 +39,16 @@
 namespace hisa {
 namespace {
 
-constexpr int kNW = 4;   // warps per CTA
-constexpr int kT = 16;   // list entries per warp tile
-constexpr int kNS = HISA_ATTN_STAGES;
+constexpr int kNW = 4;  // warps per CTA
 
-template <int D>
+template <int D, int TT, int NS>
 struct AttnCfg {
+  static constexpr int kT = TT;                        // list entries per warp tile (8 or 16)
+  static constexpr int kNS = NS;                       // pipeline stages per warp
   static constexpr int ROW = D * 2;                    // bytes of one K or V row
   static constexpr int CH = D / 8;                     // 16-byte chunks per row
   static constexpr int ROWS_PER_ITER = 32 / (2 * CH);  // rows (K and V) moved per warp copy step
-  static constexpr int STAGE = 2 * kT * ROW;           // 16 K rows, then 16 V rows
+  static constexpr int STAGE = 2 * kT * ROW;           // kT K rows, then kT V rows
   static constexpr int KSTEPS = D / 16;                // QK k-steps and PV m-tiles
   static constexpr int WARP = kNS * STAGE;
   static constexpr int IDS_OFF = kNW * WARP;           // token ids of every stage
@@ -91,14 +95,23 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-template <int D>
-__global__ void __launch_bounds__(kNW * 32)
+// D (16x8 fp32) += A (16x8 bf16, row) x B (8x8 bf16, col)
+__device__ __forceinline__ void mma_bf16_k8(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t b0) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(b0));
+}
+
+template <int D, int TT, int NS, int MINB>
+__global__ void __launch_bounds__(kNW * 32, MINB)
     sparse_attn_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
                        const uint16_t* __restrict__ v, const int32_t* __restrict__ token_idx,
                        uint16_t* __restrict__ o, float* __restrict__ lse, int32_t* __restrict__ status,
                        float* __restrict__ partial, int64_t n_q, int64_t n_kv, int H, int Hkv, int topk, int splits,
                        float qscale, int64_t n_query) {
-  using C = AttnCfg<D>;
+  using C = AttnCfg<D, TT, NS>;
+  constexpr int kT = C::kT, kNS = C::kNS;
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ int s_last[kNW];
 
@@ -201,12 +214,16 @@ __global__ void __launch_bounds__(kNW * 32)
 #pragma unroll
   for (int mt = 0; mt < C::KSTEPS; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
 
-  // ldmatrix rows: lane supplies row (lane & 7) + 8 * (mi >> 1) of logical chunk 2s + (mi & 1),
-  // stored at chunk (2s + (mi & 1)) ^ (lane & 7) = 2s ^ y with y = (mi & 1) ^ (lane & 7).
+  // ldmatrix row addresses.  Rows keep their 2d-byte pitch; logical 16-byte chunk c of row r
+  // sits at chunk c ^ (r & 7).  16-token tiles: lane supplies row (lane & 7) + 8 * (mi >> 1) of
+  // logical chunk 2s + (mi & 1) -> stored at 2s ^ y with y = (mi & 1) ^ (lane & 7).  8-token
+  // tiles: lane supplies row (lane & 7) of chunk 2s + mi for an even s, stored at 2s ^ y with
+  // y = mi ^ (lane & 7) (no carry: 2s is a multiple of 4).
   const int mi = lane >> 3;
-  const uint32_t y16 = (uint32_t)(((mi & 1) ^ (lane & 7)) << 4);
-  const uint32_t a_k = (uint32_t)(((lane & 7) + (mi >> 1) * 8) * C::ROW);
-  const uint32_t a_v = (uint32_t)((kT + (lane & 7) + (mi >> 1) * 8) * C::ROW);
+  const uint32_t y16 = kT == 16 ? (uint32_t)(((mi & 1) ^ (lane & 7)) << 4) : (uint32_t)((mi ^ (lane & 7)) << 4);
+  const uint32_t a_k = kT == 16 ? (uint32_t)(((lane & 7) + (mi >> 1) * 8) * C::ROW) : (uint32_t)((lane & 7) * C::ROW);
+  const uint32_t a_v = kT == 16 ? (uint32_t)((kT + (lane & 7) + (mi >> 1) * 8) * C::ROW)
+                                : (uint32_t)((kT + (lane & 7)) * C::ROW);
 
 #pragma unroll
   for (int j = 0; j < kNS - 1; ++j) issue(j);
@@ -216,32 +233,46 @@ __global__ void __launch_bounds__(kNW * 32)
     __syncwarp();
     const int stage = j % kNS;
     const uint32_t sb = wbase + stage * C::STAGE;
+    constexpr int NSC = kT / 4;  // scores per lane (lanes 0-7)
 
-    // scores of tokens 2tig, 2tig+1 (first MMA) and 8+2tig, 9+2tig (second), in lanes 0-7;
-    // even and odd k-steps accumulate separately to halve the dependent MMA chains
-    float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
-    float t0[4] = {0.f, 0.f, 0.f, 0.f}, t1[4] = {0.f, 0.f, 0.f, 0.f};
+    // Scores in lanes 0-7: 16-token tiles hold tokens 2tig, 2tig+1, 8+2tig, 9+2tig; 8-token tiles
+    // 2tig, 2tig+1.  Even and odd k-steps accumulate separately (shorter MMA chains).
+    float sc[NSC];
+    {
+      float s0[4] = {0.f, 0.f, 0.f, 0.f}, t0[4] = {0.f, 0.f, 0.f, 0.f};
+      if constexpr (kT == 16) {
+        float s1[4] = {0.f, 0.f, 0.f, 0.f}, t1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int s = 0; s < C::KSTEPS; s += 2) {
-      uint32_t b0, b1, b2, b3, c0, c1, c2, c3;
-      ldsm_x4(sb + a_k + (((uint32_t)s * 32u) ^ y16), b0, b1, b2, b3);
-      ldsm_x4(sb + a_k + (((uint32_t)(s + 1) * 32u) ^ y16), c0, c1, c2, c3);
-      mma_bf16(s0, qa[s][0], 0u, qa[s][1], 0u, b0, b1);
-      mma_bf16(s1, qa[s][0], 0u, qa[s][1], 0u, b2, b3);
-      mma_bf16(t0, qa[s + 1][0], 0u, qa[s + 1][1], 0u, c0, c1);
-      mma_bf16(t1, qa[s + 1][0], 0u, qa[s + 1][1], 0u, c2, c3);
+        for (int s = 0; s < C::KSTEPS; s += 2) {
+          uint32_t b0, b1, b2, b3, c0, c1, c2, c3;
+          ldsm_x4(sb + a_k + (((uint32_t)s * 32u) ^ y16), b0, b1, b2, b3);
+          ldsm_x4(sb + a_k + (((uint32_t)(s + 1) * 32u) ^ y16), c0, c1, c2, c3);
+          mma_bf16(s0, qa[s][0], 0u, qa[s][1], 0u, b0, b1);
+          mma_bf16(s1, qa[s][0], 0u, qa[s][1], 0u, b2, b3);
+          mma_bf16(t0, qa[s + 1][0], 0u, qa[s + 1][1], 0u, c0, c1);
+          mma_bf16(t1, qa[s + 1][0], 0u, qa[s + 1][1], 0u, c2, c3);
+        }
+        const uint32_t valid = gid < 2 ? mask_s[stage] >> (2 * tig) : 0u;
+        sc[0] = (valid & 1u) ? (s0[0] + t0[0]) * qscale : -INFINITY;
+        sc[1] = (valid & 2u) ? (s0[1] + t0[1]) * qscale : -INFINITY;
+        sc[2 % NSC] = (valid & 0x100u) ? (s1[0] + t1[0]) * qscale : -INFINITY;
+        sc[3 % NSC] = (valid & 0x200u) ? (s1[1] + t1[1]) * qscale : -INFINITY;
+      } else {
+#pragma unroll
+        for (int s = 0; s < C::KSTEPS; s += 2) {
+          uint32_t b0, b1, c0, c1;
+          ldsm_x4(sb + a_k + (((uint32_t)s * 32u) ^ y16), b0, b1, c0, c1);
+          mma_bf16(s0, qa[s][0], 0u, qa[s][1], 0u, b0, b1);
+          mma_bf16(t0, qa[s + 1][0], 0u, qa[s + 1][1], 0u, c0, c1);
+        }
+        const uint32_t valid = gid < 2 ? mask_s[stage] >> (2 * tig) : 0u;
+        sc[0] = (valid & 1u) ? (s0[0] + t0[0]) * qscale : -INFINITY;
+        sc[1 % NSC] = (valid & 2u) ? (s0[1] + t0[1]) * qscale : -INFINITY;
+      }
     }
-    s0[0] += t0[0];
-    s0[1] += t0[1];
-    s1[0] += t1[0];
-    s1[1] += t1[1];
-    const uint32_t valid = gid < 2 ? mask_s[stage] >> (2 * tig) : 0u;
-    float sc[4];
-    sc[0] = (valid & 1u) ? s0[0] * qscale : -INFINITY;
-    sc[1] = (valid & 2u) ? s0[1] * qscale : -INFINITY;
-    sc[2] = (valid & 0x100u) ? s1[0] * qscale : -INFINITY;
-    sc[3] = (valid & 0x200u) ? s1[1] * qscale : -INFINITY;
-    const float smax = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+    float smax = sc[0];
+#pragma unroll
+    for (int i = 1; i < NSC; ++i) smax = fmaxf(smax, sc[i]);
     // Rescale only when a score exceeds the running max by more than 2^8.
     if (__any_sync(0xFFFFFFFFu, smax > m_run + 8.f)) {
       float tmax = smax;
@@ -261,24 +292,38 @@ __global__ void __launch_bounds__(kNW * 32)
       m_run = m_new;
     }
     if (m_run != -INFINITY) {
-      float pv[4];
+      float pv[NSC];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) pv[i] = fast_exp2(sc[i] - m_run);  // 0 for masked entries
-      l_part += (pv[0] + pv[1]) + (pv[2] + pv[3]);                    // only lanes 0-3 are summed at the end
+      for (int i = 0; i < NSC; ++i) pv[i] = fast_exp2(sc[i] - m_run);  // 0 for masked entries
+#pragma unroll
+      for (int i = 0; i < NSC; ++i) l_part += pv[i];  // only lanes 0-3 are summed at the end
       // P^T column 0 (lanes 0-3) = bf16(p); column 1 (lanes 4-7) = bf16(p - bf16(p)); other lanes 0.
-      const __nv_bfloat162 h01 = __floats2bfloat162_rn(pv[0], pv[1]);
-      const __nv_bfloat162 h89 = __floats2bfloat162_rn(pv[2], pv[3]);
-      const __nv_bfloat162 l01 = __floats2bfloat162_rn(pv[0] - __low2float(h01), pv[1] - __high2float(h01));
-      const __nv_bfloat162 l89 = __floats2bfloat162_rn(pv[2] - __low2float(h89), pv[3] - __high2float(h89));
-      const uint32_t uh01 = *reinterpret_cast<const uint32_t*>(&h01), uh89 = *reinterpret_cast<const uint32_t*>(&h89);
-      const uint32_t ul01 = *reinterpret_cast<const uint32_t*>(&l01), ul89 = *reinterpret_cast<const uint32_t*>(&l89);
+      const __nv_bfloat162 h01 = __floats2bfloat162_rn(pv[0], pv[1 % NSC]);
+      const __nv_bfloat162 l01 = __floats2bfloat162_rn(pv[0] - __low2float(h01), pv[1 % NSC] - __high2float(h01));
+      const uint32_t uh01 = *reinterpret_cast<const uint32_t*>(&h01);
+      const uint32_t ul01 = *reinterpret_cast<const uint32_t*>(&l01);
       const uint32_t b0 = gid == 0 ? uh01 : ul01;  // lanes >= 8 hold p = 0, so both are 0 there
-      const uint32_t b1 = gid == 0 ? uh89 : ul89;
+      if constexpr (kT == 16) {
+        const __nv_bfloat162 h89 = __floats2bfloat162_rn(pv[2 % NSC], pv[3 % NSC]);
+        const __nv_bfloat162 l89 =
+            __floats2bfloat162_rn(pv[2 % NSC] - __low2float(h89), pv[3 % NSC] - __high2float(h89));
+        const uint32_t uh89 = *reinterpret_cast<const uint32_t*>(&h89);
+        const uint32_t ul89 = *reinterpret_cast<const uint32_t*>(&l89);
+        const uint32_t b1 = gid == 0 ? uh89 : ul89;
 #pragma unroll
-      for (int mt = 0; mt < C::KSTEPS; ++mt) {
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4_t(sb + a_v + (((uint32_t)mt * 32u) ^ y16), a0, a1, a2, a3);
-        mma_bf16(acc[mt], a0, a1, a2, a3, b0, b1);
+        for (int mt = 0; mt < C::KSTEPS; ++mt) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_t(sb + a_v + (((uint32_t)mt * 32u) ^ y16), a0, a1, a2, a3);
+          mma_bf16(acc[mt], a0, a1, a2, a3, b0, b1);
+        }
+      } else {
+#pragma unroll
+        for (int mt = 0; mt < C::KSTEPS; mt += 2) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_t(sb + a_v + (((uint32_t)mt * 32u) ^ y16), a0, a1, a2, a3);
+          mma_bf16_k8(acc[mt], a0, a1, b0);
+          mma_bf16_k8(acc[mt + 1], a2, a3, b0);
+        }
       }
     }
     __syncwarp();
@@ -356,8 +401,10 @@ __global__ void __launch_bounds__(D) attn_merge_kernel(const float* __restrict__
 template <int D>
 cudaError_t launch_d(const Shape& s, const void* q, const void* k, const void* v, const int32_t* token_idx, void* o,
                      float* lse, int32_t* status, int splits, float* partial, cudaStream_t st) {
-  using C = AttnCfg<D>;
-  auto kern = sparse_attn_kernel<D>;
+  constexpr int TT = HISA_ATTN_TILE, NS = HISA_ATTN_STAGES;
+  constexpr int MINB = TT == 8 ? 4 : 1;
+  using C = AttnCfg<D, TT, NS>;
+  auto kern = sparse_attn_kernel<D, TT, NS, MINB>;
   cudaError_t e = ensure_smem((const void*)kern, C::SMEM);
   if (e != cudaSuccess) return e;
   const int64_t grid = s.n_query * s.H * splits;
