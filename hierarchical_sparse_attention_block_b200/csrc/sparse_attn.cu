@@ -163,33 +163,40 @@ __global__ void __launch_bounds__(kNW * 32, MINB)
     }
   }
 
-  // Copies: iteration i moves row i of the tile; lanes 0..CH-1 a K chunk, CH..2CH-1 a V chunk.
-  // Rows stay 2*d-byte aligned; 16-byte chunk c of row r is stored at chunk c ^ (r & 7), which
-  // makes the 8-row ldmatrix reads below bank-conflict free.
+  // Copies: step i moves rows i*RPI + hi (hi = lane / (2 CH)); lanes [hi*2CH, hi*2CH + CH) copy a
+  // K chunk, the next CH lanes a V chunk.  Rows keep their 2d-byte pitch; logical 16-byte chunk c
+  // of row r sits at chunk c ^ (r & 7), which keeps the 8-row ldmatrix reads conflict-free.
   uint8_t* wbuf = smem + warp * C::WARP;
   const uint32_t wbase = smem_u32(wbuf);
+  const int hi = lane / (2 * C::CH);    // 0 when a step moves one row (d = 128)
   const int part = (lane / C::CH) & 1;  // 0 = K, 1 = V
   const int ch = lane % C::CH;
   const uint16_t* src_base = (part ? v : k) + ((int64_t)seq * n_kv * Hkv + g) * D + ch * 8;
   const uint32_t tok_stride = (uint32_t)(Hkv * D);
   int32_t* ids_s = reinterpret_cast<int32_t*>(smem + C::IDS_OFF) + warp * kNS * kT;
   uint32_t* mask_s = reinterpret_cast<uint32_t*>(smem + C::MASK_OFF) + warp * kNS;
+  // destination of this lane's chunk of row (rc + hi) in stage 0, minus rc * ROW, per (rc & 7)
+  uint32_t dxo[8];
+  {
+    const uint32_t lane_base = wbase + (uint32_t)(part * kT * C::ROW + hi * C::ROW);
+    const int chx = ch ^ hi;  // (rc + hi) & 7 == (rc & 7) ^ hi for the even rc of two-row steps
+#pragma unroll
+    for (int x = 0; x < 8; ++x) dxo[x] = lane_base + (uint32_t)((chx ^ x) << 4);
+  }
 
   auto issue = [&](int j) {
     const int t = warp + j * kNW;
-    if (t < n_tiles) {
+    if (t < n_tiles) {  // warp-uniform
       const int stage = j % kNS;
-      const int ebase = e0 + t * kT;
-      bool ok = false;
-      if (lane < kT) {
-        const int e = ebase + lane;
-        const int tok = e < e1 ? list[e] : -1;
-        ok = tok >= 0 && (int64_t)tok <= p;
-        if (!ok && tok != -1 && status) atomicOr(status, kStatusBadIndex);
-        ids_s[stage * kT + lane] = ok ? tok : -1;
-      }
-      const uint32_t valid = __ballot_sync(0xFFFFFFFFu, ok);
-      if (lane == 0) mask_s[stage] = valid;
+      // entry ids: lanes l and l + kT (and so on) hold entry l & (kT - 1); invalid -> token 0 + a clear bit
+      const int e = e0 + t * kT + (lane & (kT - 1));
+      const int tok = e < e1 ? list[e] : -1;
+      const bool ok = tok >= 0 && (int64_t)tok <= p;
+      const bool bad = tok != -1 && !ok;
+      if (__any_sync(0xFFFFFFFFu, bad) && bad && status) atomicOr(status, kStatusBadIndex);
+      const uint32_t valid = __ballot_sync(0xFFFFFFFFu, ok) & ((1u << kT) - 1u);
+      ids_s[stage * kT + (lane & (kT - 1))] = ok ? tok : 0;
+      mask_s[stage] = valid;
       __syncwarp();
       int tk[kT];
 #pragma unroll
@@ -197,13 +204,14 @@ __global__ void __launch_bounds__(kNW * 32, MINB)
         const int4 t4 = *reinterpret_cast<const int4*>(ids_s + stage * kT + i);
         tk[i] = t4.x; tk[i + 1] = t4.y; tk[i + 2] = t4.z; tk[i + 3] = t4.w;
       }
-      const uint32_t sdst = wbase + stage * C::STAGE + part * kT * C::ROW;
+      const uint32_t vbits = valid >> hi;
+      const uint32_t sofs = (uint32_t)(stage * C::STAGE);
 #pragma unroll
       for (int i = 0; i < kT / C::ROWS_PER_ITER; ++i) {
-        const int r = i * C::ROWS_PER_ITER + lane / (2 * C::CH);
-        const int tok = C::ROWS_PER_ITER == 1 ? tk[i] : (lane / (2 * C::CH) ? tk[2 * i + 1] : tk[2 * i]);
-        cp_async16_u32(sdst + r * C::ROW + ((ch ^ (r & 7)) << 4),
-                       src_base + (uint64_t)(uint32_t)max(tok, 0) * tok_stride, tok < 0);
+        const int rc = i * C::ROWS_PER_ITER;
+        const int tok_r = C::ROWS_PER_ITER == 1 ? tk[rc] : (hi ? tk[rc + 1] : tk[rc]);
+        cp_async16_u32(dxo[rc & 7] + sofs + (uint32_t)(rc * C::ROW),
+                       src_base + (uint64_t)(uint32_t)tok_r * tok_stride, ((vbits >> rc) & 1u) == 0u);
       }
     }
     cp_async_commit();
@@ -224,6 +232,9 @@ __global__ void __launch_bounds__(kNW * 32, MINB)
   const uint32_t a_k = kT == 16 ? (uint32_t)(((lane & 7) + (mi >> 1) * 8) * C::ROW) : (uint32_t)((lane & 7) * C::ROW);
   const uint32_t a_v = kT == 16 ? (uint32_t)((kT + (lane & 7) + (mi >> 1) * 8) * C::ROW)
                                 : (uint32_t)((kT + (lane & 7)) * C::ROW);
+  uint32_t xs[C::KSTEPS];  // per k-step / m-tile chunk offsets, swizzle applied
+#pragma unroll
+  for (int s = 0; s < C::KSTEPS; ++s) xs[s] = ((uint32_t)s * 32u) ^ y16;
 
 #pragma unroll
   for (int j = 0; j < kNS - 1; ++j) issue(j);
@@ -233,6 +244,7 @@ __global__ void __launch_bounds__(kNW * 32, MINB)
     __syncwarp();
     const int stage = j % kNS;
     const uint32_t sb = wbase + stage * C::STAGE;
+    const uint32_t sbk = sb + a_k, sbv = sb + a_v;
     constexpr int NSC = kT / 4;  // scores per lane (lanes 0-7)
 
     // Scores in lanes 0-7: 16-token tiles hold tokens 2tig, 2tig+1, 8+2tig, 9+2tig; 8-token tiles
@@ -245,8 +257,8 @@ __global__ void __launch_bounds__(kNW * 32, MINB)
 #pragma unroll
         for (int s = 0; s < C::KSTEPS; s += 2) {
           uint32_t b0, b1, b2, b3, c0, c1, c2, c3;
-          ldsm_x4(sb + a_k + (((uint32_t)s * 32u) ^ y16), b0, b1, b2, b3);
-          ldsm_x4(sb + a_k + (((uint32_t)(s + 1) * 32u) ^ y16), c0, c1, c2, c3);
+          ldsm_x4(sbk + xs[s], b0, b1, b2, b3);
+          ldsm_x4(sbk + xs[s + 1], c0, c1, c2, c3);
           mma_bf16(s0, qa[s][0], 0u, qa[s][1], 0u, b0, b1);
           mma_bf16(s1, qa[s][0], 0u, qa[s][1], 0u, b2, b3);
           mma_bf16(t0, qa[s + 1][0], 0u, qa[s + 1][1], 0u, c0, c1);
@@ -261,7 +273,7 @@ __global__ void __launch_bounds__(kNW * 32, MINB)
 #pragma unroll
         for (int s = 0; s < C::KSTEPS; s += 2) {
           uint32_t b0, b1, c0, c1;
-          ldsm_x4(sb + a_k + (((uint32_t)s * 32u) ^ y16), b0, b1, c0, c1);
+          ldsm_x4(sbk + xs[s], b0, b1, c0, c1);
           mma_bf16(s0, qa[s][0], 0u, qa[s][1], 0u, b0, b1);
           mma_bf16(t0, qa[s + 1][0], 0u, qa[s + 1][1], 0u, c0, c1);
         }
@@ -313,14 +325,14 @@ __global__ void __launch_bounds__(kNW * 32, MINB)
 #pragma unroll
         for (int mt = 0; mt < C::KSTEPS; ++mt) {
           uint32_t a0, a1, a2, a3;
-          ldsm_x4_t(sb + a_v + (((uint32_t)mt * 32u) ^ y16), a0, a1, a2, a3);
+          ldsm_x4_t(sbv + xs[mt], a0, a1, a2, a3);
           mma_bf16(acc[mt], a0, a1, a2, a3, b0, b1);
         }
       } else {
 #pragma unroll
         for (int mt = 0; mt < C::KSTEPS; mt += 2) {
           uint32_t a0, a1, a2, a3;
-          ldsm_x4_t(sb + a_v + (((uint32_t)mt * 32u) ^ y16), a0, a1, a2, a3);
+          ldsm_x4_t(sbv + xs[mt], a0, a1, a2, a3);
           mma_bf16_k8(acc[mt], a0, a1, b0);
           mma_bf16_k8(acc[mt + 1], a2, a3, b0);
         }
@@ -398,10 +410,13 @@ __global__ void __launch_bounds__(D) attn_merge_kernel(const float* __restrict__
   if (threadIdx.x == 0 && lse) lse[row] = L > 0.f ? (M + log2f(L)) * 0.69314718055994531f : -INFINITY;
 }
 
-template <int D>
-cudaError_t launch_d(const Shape& s, const void* q, const void* k, const void* v, const int32_t* token_idx, void* o,
-                     float* lse, int32_t* status, int splits, float* partial, cudaStream_t st) {
-  constexpr int TT = HISA_ATTN_TILE, NS = HISA_ATTN_STAGES;
+#ifndef HISA_ATTN_SPLIT_STAGES
+#define HISA_ATTN_SPLIT_STAGES 2
+#endif
+
+template <int D, int TT, int NS>
+cudaError_t launch_tiled(const Shape& s, const void* q, const void* k, const void* v, const int32_t* token_idx,
+                         void* o, float* lse, int32_t* status, int splits, float* partial, cudaStream_t st) {
   constexpr int MINB = TT == 8 ? 4 : 1;
   using C = AttnCfg<D, TT, NS>;
   auto kern = sparse_attn_kernel<D, TT, NS, MINB>;
@@ -417,6 +432,15 @@ cudaError_t launch_d(const Shape& s, const void* q, const void* k, const void* v
   if (e != cudaSuccess || splits == 1) return e;
   attn_merge_kernel<D><<<(unsigned)(s.n_query * s.H), D, 0, st>>>(partial, static_cast<uint16_t*>(o), lse, splits);
   return cudaGetLastError();
+}
+
+// One work item per (query, head) (prefill) or lists split across CTAs (decode).
+template <int D>
+cudaError_t launch_d(const Shape& s, const void* q, const void* k, const void* v, const int32_t* token_idx, void* o,
+                     float* lse, int32_t* status, int splits, float* partial, cudaStream_t st) {
+  if (splits > 1)
+    return launch_tiled<D, 16, HISA_ATTN_SPLIT_STAGES>(s, q, k, v, token_idx, o, lse, status, splits, partial, st);
+  return launch_tiled<D, HISA_ATTN_TILE, HISA_ATTN_STAGES>(s, q, k, v, token_idx, o, lse, status, splits, partial, st);
 }
 
 }  // namespace
