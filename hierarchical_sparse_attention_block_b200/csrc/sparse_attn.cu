@@ -25,6 +25,8 @@
 // the status word.
 #include <math.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -93,6 +95,15 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Calls f(std::integral_constant<int, I>) for I = B .. E-1 (compile-time loop).
+template <int B, int E, class F>
+__device__ __forceinline__ void static_for(F&& f) {
+  if constexpr (B < E) {
+    f(std::integral_constant<int, B>{});
+    static_for<B + 1, E>(f);
+  }
 }
 
 // D (16x8 fp32) += A (16x8 bf16, row) x B (8x8 bf16, col)
@@ -184,10 +195,10 @@ __global__ void __launch_bounds__(kNW * 32, MINB)
     for (int x = 0; x < 8; ++x) dxo[x] = lane_base + (uint32_t)((chx ^ x) << 4);
   }
 
-  auto issue = [&](int j) {
+  auto issue = [&](int j, auto stage_c) {
+    constexpr int stage = decltype(stage_c)::value;
     const int t = warp + j * kNW;
     if (t < n_tiles) {  // warp-uniform
-      const int stage = j % kNS;
       // entry ids: lanes l and l + kT (and so on) hold entry l & (kT - 1); invalid -> token 0 + a clear bit
       const int e = e0 + t * kT + (lane & (kT - 1));
       const int tok = e < e1 ? list[e] : -1;
@@ -236,13 +247,9 @@ __global__ void __launch_bounds__(kNW * 32, MINB)
 #pragma unroll
   for (int s = 0; s < C::KSTEPS; ++s) xs[s] = ((uint32_t)s * 32u) ^ y16;
 
-#pragma unroll
-  for (int j = 0; j < kNS - 1; ++j) issue(j);
-  for (int j = 0; j < my_tiles; ++j) {
-    issue(j + kNS - 1);
-    cp_async_wait<kNS - 1>();
-    __syncwarp();
-    const int stage = j % kNS;
+  // One tile: wait for its copies, then scores, softmax and output on the tensor cores.
+  auto compute = [&](auto stage_c) {
+    constexpr int stage = decltype(stage_c)::value;
     const uint32_t sb = wbase + stage * C::STAGE;
     const uint32_t sbk = sb + a_k, sbv = sb + a_v;
     constexpr int NSC = kT / 4;  // scores per lane (lanes 0-7)
@@ -339,6 +346,21 @@ __global__ void __launch_bounds__(kNW * 32, MINB)
       }
     }
     __syncwarp();
+  };
+
+  // Stages cycle with the tile index, so the loop is unrolled by the stage count and every
+  // stage offset is a compile-time constant.
+  static_for<0, kNS - 1>([&](auto u) { issue(decltype(u)::value, u); });
+  for (int j = 0; j < my_tiles; j += kNS) {
+    static_for<0, kNS>([&](auto u) {
+      constexpr int U = decltype(u)::value;
+      if (j + U < my_tiles) {  // warp-uniform
+        issue(j + U + kNS - 1, std::integral_constant<int, (U + kNS - 1) % kNS>{});
+        cp_async_wait<kNS - 1>();
+        __syncwarp();
+        compute(u);
+      }
+    });
   }
   cp_async_wait<0>();
   // per-warp row sum: lanes 0-3 hold partial sums
