@@ -68,6 +68,23 @@ __device__ __forceinline__ void cp_async16_u32(uint32_t dst, const void* src, bo
       : "memory");
 }
 
+// bf16 pair of the high halves of two fp32 values (truncation), and of their exact remainders
+// (rounded to nearest).  x == hi + lo up to the rounding of lo.
+__device__ __forceinline__ uint32_t hi_pair(float x0, float x1) {
+  return __byte_perm(__float_as_uint(x0), __float_as_uint(x1), 0x7632);
+}
+__device__ __forceinline__ uint32_t lo_pair(float x0, float x1) {
+  const float r0 = x0 - __uint_as_float(__float_as_uint(x0) & 0xFFFF0000u);
+  const float r1 = x1 - __uint_as_float(__float_as_uint(x1) & 0xFFFF0000u);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(r0, r1);
+  return *reinterpret_cast<const uint32_t*>(&l);
+}
+
+// Unpredicated 16-byte global -> shared copy through L2 only.
+__device__ __forceinline__ void cp_async16_all(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src) : "memory");
+}
+
 // 2^x on the special-function unit (the weights are re-rounded to a bf16 pair right after).
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
@@ -216,19 +233,30 @@ __global__ void __launch_bounds__(kNW * 32, MINB)
         tk[i] = t4.x; tk[i + 1] = t4.y; tk[i + 2] = t4.z; tk[i + 3] = t4.w;
       }
       const uint32_t vbits = valid >> hi;
-      const uint32_t sofs = (uint32_t)(stage * C::STAGE);
+      constexpr uint32_t sofs = (uint32_t)(stage * C::STAGE);
+      if (valid == (1u << kT) - 1u) {  // warp-uniform: every entry valid (the common case)
 #pragma unroll
-      for (int i = 0; i < kT / C::ROWS_PER_ITER; ++i) {
-        const int rc = i * C::ROWS_PER_ITER;
-        const int tok_r = C::ROWS_PER_ITER == 1 ? tk[rc] : (hi ? tk[rc + 1] : tk[rc]);
-        cp_async16_u32(dxo[rc & 7] + sofs + (uint32_t)(rc * C::ROW),
-                       src_base + (uint64_t)(uint32_t)tok_r * tok_stride, ((vbits >> rc) & 1u) == 0u);
+        for (int i = 0; i < kT / C::ROWS_PER_ITER; ++i) {
+          const int rc = i * C::ROWS_PER_ITER;
+          const int tok_r = C::ROWS_PER_ITER == 1 ? tk[rc] : (hi ? tk[rc + 1] : tk[rc]);
+          cp_async16_all(dxo[rc & 7] + sofs + (uint32_t)(rc * C::ROW),
+                         src_base + (uint64_t)(uint32_t)tok_r * tok_stride);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < kT / C::ROWS_PER_ITER; ++i) {
+          const int rc = i * C::ROWS_PER_ITER;
+          const int tok_r = C::ROWS_PER_ITER == 1 ? tk[rc] : (hi ? tk[rc + 1] : tk[rc]);
+          cp_async16_u32(dxo[rc & 7] + sofs + (uint32_t)(rc * C::ROW),
+                         src_base + (uint64_t)(uint32_t)tok_r * tok_stride, ((vbits >> rc) & 1u) == 0u);
+        }
       }
     }
     cp_async_commit();
   };
 
   float m_run = -INFINITY, l_part = 0.f;
+  float m_lim = -INFINITY, neg_mq = 0.f;  // rescale threshold and -m_run * qscale
   float acc[C::KSTEPS][4];
 #pragma unroll
   for (int mt = 0; mt < C::KSTEPS; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
@@ -272,10 +300,10 @@ __global__ void __launch_bounds__(kNW * 32, MINB)
           mma_bf16(t1, qa[s + 1][0], 0u, qa[s + 1][1], 0u, c2, c3);
         }
         const uint32_t valid = gid < 2 ? mask_s[stage] >> (2 * tig) : 0u;
-        sc[0] = (valid & 1u) ? (s0[0] + t0[0]) * qscale : -INFINITY;
-        sc[1] = (valid & 2u) ? (s0[1] + t0[1]) * qscale : -INFINITY;
-        sc[2 % NSC] = (valid & 0x100u) ? (s1[0] + t1[0]) * qscale : -INFINITY;
-        sc[3 % NSC] = (valid & 0x200u) ? (s1[1] + t1[1]) * qscale : -INFINITY;
+        sc[0] = (valid & 1u) ? s0[0] + t0[0] : -INFINITY;
+        sc[1] = (valid & 2u) ? s0[1] + t0[1] : -INFINITY;
+        sc[2 % NSC] = (valid & 0x100u) ? s1[0] + t1[0] : -INFINITY;
+        sc[3 % NSC] = (valid & 0x200u) ? s1[1] + t1[1] : -INFINITY;
       } else {
 #pragma unroll
         for (int s = 0; s < C::KSTEPS; s += 2) {
@@ -285,21 +313,22 @@ __global__ void __launch_bounds__(kNW * 32, MINB)
           mma_bf16(t0, qa[s + 1][0], 0u, qa[s + 1][1], 0u, c0, c1);
         }
         const uint32_t valid = gid < 2 ? mask_s[stage] >> (2 * tig) : 0u;
-        sc[0] = (valid & 1u) ? (s0[0] + t0[0]) * qscale : -INFINITY;
-        sc[1 % NSC] = (valid & 2u) ? (s0[1] + t0[1]) * qscale : -INFINITY;
+        sc[0] = (valid & 1u) ? s0[0] + t0[0] : -INFINITY;
+        sc[1 % NSC] = (valid & 2u) ? s0[1] + t0[1] : -INFINITY;
       }
     }
     float smax = sc[0];
 #pragma unroll
     for (int i = 1; i < NSC; ++i) smax = fmaxf(smax, sc[i]);
-    // Rescale only when a score exceeds the running max by more than 2^8.
-    if (__any_sync(0xFFFFFFFFu, smax > m_run + 8.f)) {
+    // Scores stay unscaled (q.k); m_run is their running max.  The state is rescaled only when
+    // a score passes m_run + 8 / qscale, i.e. when a weight would exceed 2^8.
+    if (__any_sync(0xFFFFFFFFu, smax > m_lim)) {
       float tmax = smax;
       tmax = fmaxf(tmax, __shfl_xor_sync(0xFFFFFFFFu, tmax, 1));
       tmax = fmaxf(tmax, __shfl_xor_sync(0xFFFFFFFFu, tmax, 2));
       tmax = __shfl_sync(0xFFFFFFFFu, tmax, 0);
       const float m_new = fmaxf(m_run, tmax);
-      const float alpha = exp2f(m_run - m_new);
+      const float alpha = exp2f((m_run - m_new) * qscale);
       l_part *= alpha;
 #pragma unroll
       for (int mt = 0; mt < C::KSTEPS; ++mt) {
@@ -309,26 +338,20 @@ __global__ void __launch_bounds__(kNW * 32, MINB)
         acc[mt][3] *= alpha;
       }
       m_run = m_new;
+      m_lim = m_new + 8.f / qscale;
+      neg_mq = -m_new * qscale;
     }
     if (m_run != -INFINITY) {
       float pv[NSC];
 #pragma unroll
-      for (int i = 0; i < NSC; ++i) pv[i] = fast_exp2(sc[i] - m_run);  // 0 for masked entries
+      for (int i = 0; i < NSC; ++i) pv[i] = fast_exp2(fmaf(sc[i], qscale, neg_mq));  // 0 for masked entries
 #pragma unroll
       for (int i = 0; i < NSC; ++i) l_part += pv[i];  // only lanes 0-3 are summed at the end
-      // P^T column 0 (lanes 0-3) = bf16(p); column 1 (lanes 4-7) = bf16(p - bf16(p)); other lanes 0.
-      const __nv_bfloat162 h01 = __floats2bfloat162_rn(pv[0], pv[1 % NSC]);
-      const __nv_bfloat162 l01 = __floats2bfloat162_rn(pv[0] - __low2float(h01), pv[1 % NSC] - __high2float(h01));
-      const uint32_t uh01 = *reinterpret_cast<const uint32_t*>(&h01);
-      const uint32_t ul01 = *reinterpret_cast<const uint32_t*>(&l01);
-      const uint32_t b0 = gid == 0 ? uh01 : ul01;  // lanes >= 8 hold p = 0, so both are 0 there
+      // P^T column 0 (lanes 0-3) = p truncated to bf16 (its high half); column 1 (lanes 4-7) =
+      // the exact remainder rounded to bf16: together ~16 significant bits.  Other lanes hold 0.
+      const uint32_t b0 = gid == 0 ? hi_pair(pv[0], pv[1 % NSC]) : lo_pair(pv[0], pv[1 % NSC]);
       if constexpr (kT == 16) {
-        const __nv_bfloat162 h89 = __floats2bfloat162_rn(pv[2 % NSC], pv[3 % NSC]);
-        const __nv_bfloat162 l89 =
-            __floats2bfloat162_rn(pv[2 % NSC] - __low2float(h89), pv[3 % NSC] - __high2float(h89));
-        const uint32_t uh89 = *reinterpret_cast<const uint32_t*>(&h89);
-        const uint32_t ul89 = *reinterpret_cast<const uint32_t*>(&l89);
-        const uint32_t b1 = gid == 0 ? uh89 : ul89;
+        const uint32_t b1 = gid == 0 ? hi_pair(pv[2 % NSC], pv[3 % NSC]) : lo_pair(pv[2 % NSC], pv[3 % NSC]);
 #pragma unroll
         for (int mt = 0; mt < C::KSTEPS; ++mt) {
           uint32_t a0, a1, a2, a3;
@@ -371,7 +394,7 @@ __global__ void __launch_bounds__(kNW * 32, MINB)
   // Merge the warps' states: [kNW] max, [kNW] sum, [kNW][D] output.
   float* mg = reinterpret_cast<float*>(smem);
   if (lane == 0) {
-    mg[warp] = m_run;
+    mg[warp] = m_run * qscale;  // == -neg_mq: the offset the weights were taken against
     mg[kNW + warp] = l_part;
   }
   if (tig == 0) {
