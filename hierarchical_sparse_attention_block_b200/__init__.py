@@ -23,7 +23,7 @@ EXPORTS = (
     "hisa_block_pool", "hisa_block_topm_workspace_size", "hisa_block_topm", "hisa_token_topk_workspace_size",
     "hisa_token_topk", "hisa_sparse_attn_workspace_size", "sparse_attn_fwd", "hisa_forward_workspace_size",
     "hisa_forward", "hisa_flat_topk_workspace_size", "hisa_flat_topk", "hisa_status_string",
-    "hisa_last_cuda_error", "hisa_version", "hisa_token_topk_noalloc", "hisa_forward_cached",
+    "hisa_last_cuda_error", "hisa_version", "hisa_token_topk_noalloc", "hisa_forward_cached", "hisa_gather_probe",
 )
 
 
@@ -68,6 +68,7 @@ def _load():
         "hisa_flat_topk": [pp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
         "hisa_token_topk_noalloc": [pp, vp, vp, vp, vp, vp, vp, vp],
         "hisa_forward_cached": [pp, vp, vp, vp, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
+        "hisa_gather_probe": [vp, i64, ctypes.c_int32, i64, ctypes.c_uint32, vp, vp],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -222,6 +223,14 @@ def hisa_token_topk_noalloc(p, q_idx, k_idx, block_idx, token_idx, token_scores=
     _check("hisa_token_topk_noalloc",
            _lib.hisa_token_topk_noalloc(ctypes.byref(p), _ptr(q_idx), _ptr(k_idx), _ptr(block_idx), _ptr(token_idx),
                                         _ptr(token_scores), _ptr(dev_status), _stream(stream)))
+
+
+def hisa_gather_probe(rows, row_bytes, n_gathers, sink, seed=1, stream=None):
+    """Measurement helper: n_gathers copies of hashed rows of `rows` into shared memory, the
+    attention kernel's gather pattern without its arithmetic (see include/hisa.h)."""
+    n_rows = rows.numel() * rows.element_size() // row_bytes
+    _check("hisa_gather_probe", _lib.hisa_gather_probe(_ptr(rows), n_rows, row_bytes, n_gathers, seed, _ptr(sink),
+                                                       _stream(stream)))
 
 
 def hisa_version() -> str:

@@ -19,13 +19,9 @@
 //     and stores the causally visible scores.
 // Every wait is bounded (1 s of %globaltimer); a timeout sets status bit 1
 // and the CTA skips to releasing its TMEM.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
-#include <mutex>
-
 #include "common.cuh"
 #include "internal.h"
+#include "tc_common.cuh"
 
 namespace hisa {
 namespace {
@@ -33,8 +29,6 @@ namespace {
 constexpr int kTcThreads = 128;
 constexpr int kTileM = 128;  // queries per tile
 constexpr int kTileN = 128;  // blocks per tile
-constexpr int kStatusTimeout = 2;
-constexpr uint64_t kWaitNs = 1000000000ull;
 
 template <int D>
 struct TcLayout {
@@ -50,37 +44,7 @@ struct TcLayout {
   static constexpr int SMEM = BAR_OFF + 64 + 1024;     // + slack for 1024-byte alignment
 };
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-__device__ __forceinline__ uint64_t global_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase) {
-  const uint64_t t0 = global_ns();
-  while (true) {
-    uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(bar), "r"(phase)
-        : "memory");
-    if (ok) return true;
-    if (global_ns() - t0 > kWaitNs) return false;
-  }
-}
-
-// K-major operand, 128-byte swizzle: rows of 128 B, 8-row groups 1024 B apart.
-__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
-  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
-  d |= (uint64_t)1 << 16;           // leading byte offset (unused for this layout): 16 B
-  d |= (uint64_t)(1024 >> 4) << 32; // stride byte offset: 1024 B between 8-row groups
-  d |= (uint64_t)1 << 46;           // descriptor version (sm_100)
-  d |= (uint64_t)2 << 61;           // swizzle: 128 B
-  return d;
-}
+using namespace tc;
 
 // kind::f16 instruction descriptor: bf16 x bf16 -> fp32, both K-major, M = 128, N = 128.
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kTileN >> 3) << 17) |
@@ -205,8 +169,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int h = 0; h < L::HALVES; ++h) {
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
-          const uint64_t ad = umma_desc_sw128(a0 + h * kTileM * 128 + s * 32);
-          const uint64_t bd = umma_desc_sw128(b0 + pl * L::B_PLANE + h * kTileN * 128 + s * 32);
+          const uint64_t ad = desc_kmajor_sw128(a0 + h * kTileM * 128 + s * 32);
+          const uint64_t bd = desc_kmajor_sw128(b0 + pl * L::B_PLANE + h * kTileN * 128 + s * 32);
           const uint32_t acc = first ? 0u : 1u;
           asm volatile(
               "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
@@ -267,31 +231,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == 0) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)kTileN));
   }
-}
-
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
-bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, int esize, const void* base, uint64_t cols, uint64_t rows,
-                 uint32_t box_c, uint32_t box_r, CUtensorMapSwizzle sw) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * (uint64_t)esize};
-  cuuint32_t box[2] = {box_c, box_r};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int D>

@@ -53,6 +53,19 @@ int attn_pick_splits(const Shape& s);
 size_t attn_partial_bytes(const Shape& s, int splits);
 cudaError_t launch_sparse_attn(const Shape& s, const void* q, const void* k, const void* v, const int32_t* token_idx,
                                void* o, float* lse, int32_t* status, int splits, void* partial, cudaStream_t st);
+// Merge of the per-split (max, sum, output) states into O and the LSE.
+cudaError_t launch_attn_merge(const Shape& s, const float* partial, void* o, float* lse, int splits, cudaStream_t st);
+// Step 6 on the tensor cores (tcgen05, TMA gather), head dimension 128; cudaErrorNotSupported
+// when the shape is outside its range.
+bool sparse_attn_tc_eligible(const Shape& s);
+cudaError_t launch_sparse_attn_tc(const Shape& s, const void* q, const void* k, const void* v,
+                                  const int32_t* token_idx, void* o, float* lse, int32_t* status, int splits,
+                                  float* partial, cudaStream_t st);
+
+// Measurement helper: gathers of hashed rows into shared memory (see hisa_gather_probe).
+bool gather_probe_row_bytes_ok(int row_bytes);
+cudaError_t launch_gather_probe(const void* rows, int64_t n_rows, int row_bytes, int64_t n_gathers, uint32_t seed,
+                                uint32_t* sink, cudaStream_t st);
 
 // cudaError_t value behind the last HISA_ERR_CUDA on this host thread.
 extern thread_local int32_t g_last_cuda_error;

@@ -475,8 +475,7 @@ cudaError_t launch_tiled(const Shape& s, const void* q, const void* k, const voi
       static_cast<uint16_t*>(o), lse, status, partial, s.n_q, s.n_kv, s.H, s.Hkv, s.k, splits, qscale, s.n_query);
   e = cudaGetLastError();
   if (e != cudaSuccess || splits == 1) return e;
-  attn_merge_kernel<D><<<(unsigned)(s.n_query * s.H), D, 0, st>>>(partial, static_cast<uint16_t*>(o), lse, splits);
-  return cudaGetLastError();
+  return launch_attn_merge(s, partial, o, lse, splits, st);
 }
 
 // One work item per (query, head) (prefill) or lists split across CTAs (decode).
@@ -495,6 +494,18 @@ cudaError_t launch_d(const Shape& s, const void* q, const void* k, const void* v
 #endif
 
 int attn_pick_splits(const Shape& s) {
+  if (sparse_attn_tc_eligible(s)) {
+    // Persistent CTAs, one per SM, each taking the heads of one KV group at a time: about two
+    // items per CTA, every split at least two tiles of 128 entries.
+    const int G = s.H / s.Hkv;
+    const int64_t units = s.n_query * s.Hkv * ((G + 15) / 16);
+    const int64_t target = 2 * 148;
+    if (units >= target) return 1;
+    int64_t sp = (target + units - 1) / units;
+    const int64_t max_sp = (s.k + 255) / 256;
+    if (sp > max_sp) sp = max_sp;
+    return sp < 1 ? 1 : (int)sp;
+  }
   const int64_t units = s.n_query * s.H;
   const int64_t target = HISA_ATTN_SPLIT_TARGET;
   if (units >= target) return 1;
@@ -509,9 +520,28 @@ size_t attn_partial_bytes(const Shape& s, int splits) {
   return (size_t)s.n_query * s.H * splits * (s.d + 2) * sizeof(float);
 }
 
+cudaError_t launch_attn_merge(const Shape& s, const float* partial, void* o, float* lse, int splits, cudaStream_t st) {
+  switch (s.d) {
+    case 64:
+      attn_merge_kernel<64><<<(unsigned)(s.n_query * s.H), 64, 0, st>>>(partial, static_cast<uint16_t*>(o), lse, splits);
+      break;
+    case 128:
+      attn_merge_kernel<128><<<(unsigned)(s.n_query * s.H), 128, 0, st>>>(partial, static_cast<uint16_t*>(o), lse,
+                                                                          splits);
+      break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
 cudaError_t launch_sparse_attn(const Shape& s, const void* q, const void* k, const void* v, const int32_t* token_idx,
                                void* o, float* lse, int32_t* status, int splits, void* partial, cudaStream_t st) {
   float* part = static_cast<float*>(partial);
+  // Heads sharing K/V (GQA/MQA): the tensor-core kernel takes a KV group's heads together.
+  if (sparse_attn_tc_eligible(s)) {
+    const cudaError_t e = launch_sparse_attn_tc(s, q, k, v, token_idx, o, lse, status, splits, part, st);
+    if (e != cudaErrorNotSupported) return e;
+  }
   switch (s.d) {
     case 64: return launch_d<64>(s, q, k, v, token_idx, o, lse, status, splits, part, st);
     case 128: return launch_d<128>(s, q, k, v, token_idx, o, lse, status, splits, part, st);

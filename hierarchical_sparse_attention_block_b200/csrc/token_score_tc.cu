@@ -19,13 +19,9 @@
 // the first run also zero-fills unused slots and flags malformed entries.
 // With no list (the flat indexer) slot = block id.  Waits are bounded (1 s);
 // a timeout sets status bit 1.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
-#include <mutex>
-
 #include "common.cuh"
 #include "internal.h"
+#include "tc_common.cuh"
 
 namespace hisa {
 namespace {
@@ -33,8 +29,6 @@ namespace {
 constexpr int kThreads = 128;
 constexpr int kTileQ = 128;
 constexpr int kRun = 64;      // key blocks per CTA
-constexpr int kStatusTimeout = 2;
-constexpr uint64_t kWaitNs = 1000000000ull;
 
 template <int D, int B>
 struct TsLayout {
@@ -52,44 +46,7 @@ struct TsLayout {
                                     ((uint32_t)(kTileQ >> 4) << 24);
 };
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-__device__ __forceinline__ uint64_t global_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-  const uint64_t t0 = global_ns();
-  while (true) {
-    uint32_t ok;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    if (ok) return true;
-    if (global_ns() - t0 > kWaitNs) return false;
-  }
-}
-
-__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
-  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
-  d |= (uint64_t)1 << 16;            // leading byte offset (unused for this layout)
-  d |= (uint64_t)(1024 >> 4) << 32;  // 8-row groups 1024 B apart
-  d |= (uint64_t)1 << 46;            // sm_100 descriptor version
-  d |= (uint64_t)2 << 61;            // 128-byte swizzle
-  return d;
-}
-
-__device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-          dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-      : "memory");
-}
+using namespace tc;
 
 template <int D, int B>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -146,14 +103,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t bq = smem_u32(&bars[0]);
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bq), "r"((uint32_t)L::Q_BYTES)
                  : "memory");
-    for (int hh = 0; hh < L::HALVES; ++hh) tma_2d(smem_u32(sQ + hh * kTileQ * 128), &tmap_q, hh * 64, (int)tq0, bq);
+    for (int hh = 0; hh < L::HALVES; ++hh) tma_load_2d(smem_u32(sQ + hh * kTileQ * 128), &tmap_q, hh * 64, (int)tq0, bq);
     for (int s = 0; s < kKStages && s < nb; ++s) {
       const uint32_t bk = smem_u32(&bars[2 + s]);
       asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bk), "r"((uint32_t)L::K_BYTES)
                    : "memory");
       const int krow = (int)(seq * n_kv + (jb0 + s) * B);
       for (int hh = 0; hh < L::HALVES; ++hh)
-        tma_2d(smem_u32(sK + s * L::K_BYTES + hh * B * 128), &tmap_k, hh * 64, krow, bk);
+        tma_load_2d(smem_u32(sK + s * L::K_BYTES + hh * B * 128), &tmap_k, hh * 64, krow, bk);
     }
   }
 
@@ -205,8 +162,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int hh = 0; hh < L::HALVES; ++hh) {
 #pragma unroll
           for (int s = 0; s < 4; ++s) {
-            const uint64_t ad = desc_sw128(q_base + hh * kTileQ * 128 + s * 32);
-            const uint64_t bd = desc_sw128(k_base + stage * L::K_BYTES + hh * B * 128 + s * 32);
+            const uint64_t ad = desc_kmajor_sw128(q_base + hh * kTileQ * 128 + s * 32);
+            const uint64_t bd = desc_kmajor_sw128(k_base + stage * L::K_BYTES + hh * B * 128 + s * 32);
             const uint32_t acc = (hh | s) ? 1u : 0u;
             asm volatile(
                 "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
@@ -236,7 +193,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                    : "memory");
       const int krow = (int)(seq * n_kv + (jb0 + b + kKStages) * B);
       for (int hh = 0; hh < L::HALVES; ++hh)
-        tma_2d(smem_u32(sK + stage * L::K_BYTES + hh * B * 128), &tmap_k, hh * 64, krow, bk);
+        tma_load_2d(smem_u32(sK + stage * L::K_BYTES + hh * B * 128), &tmap_k, hh * 64, krow, bk);
     }
     // Epilogue: rows whose query kept block jb0 + b.
     const int slot = row_ok ? smap[tid * kRun + b] : -1;
@@ -283,31 +240,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"((uint32_t)(B < 32 ? 32 : B)));
   }
-}
-
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
-bool map_bf16_sw128(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {cols, rows};
-  cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {64, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int D, int B>

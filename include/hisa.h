@@ -186,6 +186,19 @@ hisa_status_t hisa_token_topk_noalloc(const hisa_params_t* params, const void* q
                                       const int32_t* block_idx, int32_t* token_idx, float* token_scores,
                                       int32_t* dev_status, cudaStream_t stream);
 
+/* Measurement helper, not a step of the method (the pages have no
+ * counterpart): n_gathers copies of row h(e) (row_bytes each; h a hash of the
+ * gather number e and seed, uniform over [0, n_rows)) into shared memory with
+ * 16-byte cp.async, the copy pattern of sparse_attn_fwd's gathers without any
+ * of its arithmetic or index reads, so that timing it gives that kernel a
+ * measured ceiling for rows the L2 serves.  rows: device, [n_rows][row_bytes],
+ * 16-byte aligned, n_rows < 2^31; row_bytes a multiple of 16, at most 256,
+ * with 32 / (row_bytes / 16) integral; sink: one device word the kernel adds a
+ * copied word to, so the copies cannot be optimised away.  Returns
+ * HISA_ERR_INVALID_ARG for bad arguments; asynchronous on stream. */
+hisa_status_t hisa_gather_probe(const void* rows, int64_t n_rows, int32_t row_bytes, int64_t n_gathers,
+                                uint32_t seed, uint32_t* sink, cudaStream_t stream);
+
 /* Static text for a status code. */
 const char* hisa_status_string(hisa_status_t status);
 /* cudaError_t value of the last failed CUDA call on this host thread (0 if none). */
