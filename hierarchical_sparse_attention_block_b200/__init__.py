@@ -24,6 +24,8 @@ EXPORTS = (
     "hisa_token_topk", "hisa_sparse_attn_workspace_size", "sparse_attn_fwd", "hisa_forward_workspace_size",
     "hisa_forward", "hisa_flat_topk_workspace_size", "hisa_flat_topk", "hisa_status_string",
     "hisa_last_cuda_error", "hisa_version", "hisa_token_topk_noalloc", "hisa_forward_cached", "hisa_gather_probe",
+    "hisa_block_candidates_workspace_size", "hisa_block_candidates", "hisa_topk_merge", "hisa_remap_ids",
+    "hisa_lse_merge",
 )
 
 
@@ -69,6 +71,11 @@ def _load():
         "hisa_token_topk_noalloc": [pp, vp, vp, vp, vp, vp, vp, vp],
         "hisa_forward_cached": [pp, vp, vp, vp, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
         "hisa_gather_probe": [vp, i64, ctypes.c_int32, i64, ctypes.c_uint32, vp, vp],
+        "hisa_block_candidates_workspace_size": [pp, sz],
+        "hisa_block_candidates": [pp, i64, i64, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
+        "hisa_topk_merge": [vp, vp, ctypes.c_int32, i64, ctypes.c_int32, ctypes.c_int32, vp, vp, vp],
+        "hisa_remap_ids": [vp, i64, ctypes.c_int32, i64, i64, i64, vp, vp],
+        "hisa_lse_merge": [vp, vp, ctypes.c_int32, i64, ctypes.c_int32, vp, vp, vp],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -223,6 +230,44 @@ def hisa_token_topk_noalloc(p, q_idx, k_idx, block_idx, token_idx, token_scores=
     _check("hisa_token_topk_noalloc",
            _lib.hisa_token_topk_noalloc(ctypes.byref(p), _ptr(q_idx), _ptr(k_idx), _ptr(block_idx), _ptr(token_idx),
                                         _ptr(token_scores), _ptr(dev_status), _stream(stream)))
+
+
+def hisa_block_candidates_workspace_size(p) -> int:
+    return _size(_lib.hisa_block_candidates_workspace_size, p)
+
+
+def hisa_block_candidates(p_local, n_kv_global, first_block, q_idx, block_keys, cand_scores, cand_ids,
+                          workspace=None, stream=None):
+    """This rank's step-3 candidates (see include/hisa.h): [batch][top_m] scores and global block ids."""
+    if workspace is None:
+        workspace = _workspace(hisa_block_candidates_workspace_size(p_local), q_idx.device)
+    _check("hisa_block_candidates",
+           _lib.hisa_block_candidates(ctypes.byref(p_local), n_kv_global, first_block, _ptr(q_idx), _ptr(block_keys),
+                                      _ptr(cand_scores), _ptr(cand_ids), _ptr(workspace), workspace.numel(),
+                                      _stream(stream)))
+
+
+def hisa_topk_merge(scores, ids, k, out_ids, out_scores=None, stream=None):
+    """Best k of the candidates in scores / ids [n_parts][rows][n_per] (ascending ids within a row)."""
+    n_parts, rows, n_per = scores.shape
+    _check("hisa_topk_merge", _lib.hisa_topk_merge(_ptr(scores), _ptr(ids), n_parts, rows, n_per, k, _ptr(out_ids),
+                                                   _ptr(out_scores), _stream(stream)))
+
+
+def hisa_remap_ids(ids, lo, hi, delta, out=None, stream=None):
+    """Entries of each row of ids [rows][cols] inside [lo, hi), shifted by delta, compacted, -1 padded."""
+    out = ids if out is None else out
+    rows, cols = ids.reshape(-1, ids.shape[-1]).shape
+    _check("hisa_remap_ids", _lib.hisa_remap_ids(_ptr(ids), rows, cols, lo, hi, delta, _ptr(out), _stream(stream)))
+    return out
+
+
+def hisa_lse_merge(o_parts, lse_parts, o, lse=None, stream=None):
+    """o_parts [n_parts][rows..][d] bf16 and lse_parts [n_parts][rows..] merged into o (and lse)."""
+    n_parts, d = o_parts.shape[0], o_parts.shape[-1]
+    rows = lse_parts[0].numel()
+    _check("hisa_lse_merge", _lib.hisa_lse_merge(_ptr(o_parts), _ptr(lse_parts), n_parts, rows, d, _ptr(o), _ptr(lse),
+                                                 _stream(stream)))
 
 
 def hisa_gather_probe(rows, row_bytes, n_gathers, sink, seed=1, stream=None):

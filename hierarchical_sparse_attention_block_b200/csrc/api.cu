@@ -117,20 +117,20 @@ hisa_status_t run_block_stage(const Shape& s, const void* q_idx, const float* bl
 cudaError_t ensure_smem(const void* func, int bytes) {
   if (bytes <= 48 * 1024) return cudaSuccess;
   static std::mutex mu;
-  static const void* done_f[64][16];
-  static int done_b[64][16];
+  static const void* done_f[64][64];
+  static int done_b[64][64];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lock(mu);
   if (dev >= 0 && dev < 64) {
-    for (int i = 0; i < 16; ++i)
+    for (int i = 0; i < 64; ++i)
       if (done_f[dev][i] == func && done_b[dev][i] >= bytes) return cudaSuccess;
   }
   e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e != cudaSuccess) return e;
   if (dev >= 0 && dev < 64) {
-    for (int i = 0; i < 16; ++i) {
+    for (int i = 0; i < 64; ++i) {
       if (done_f[dev][i] == nullptr || done_f[dev][i] == func) {
         done_f[dev][i] = func;
         done_b[dev][i] = bytes;
@@ -367,6 +367,59 @@ hisa_status_t hisa_flat_topk(const hisa_params_t* params, const void* q_idx, con
   if (s.n_blk > 50000 || s.n_blk * (int64_t)s.B > ((int64_t)1 << 30)) return HISA_ERR_UNSUPPORTED;
   return hisa::run_token_stage(s, q_idx, k_idx, nullptr, (int)s.n_blk, token_idx, token_scores, nullptr, workspace,
                                workspace_bytes, stream);
+}
+
+hisa_status_t hisa_block_candidates_workspace_size(const hisa_params_t* local, size_t* bytes) {
+  Shape s;
+  hisa_status_t rc = hisa::make_shape(local, true, false, &s);
+  if (rc != HISA_OK) return rc;
+  if (!bytes) return HISA_ERR_INVALID_ARG;
+  *bytes = (size_t)s.n_query * s.n_blk * sizeof(float);
+  return HISA_OK;
+}
+
+hisa_status_t hisa_block_candidates(const hisa_params_t* local, int64_t n_kv_global, int64_t first_block,
+                                    const void* q_idx, const float* block_keys, float* cand_scores, int32_t* cand_ids,
+                                    void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  Shape s;
+  hisa_status_t rc = hisa::make_shape(local, true, false, &s);
+  if (rc != HISA_OK) return rc;
+  if (s.n_q != 1) return HISA_ERR_UNSUPPORTED;  // decode: the query is the newest token of the whole context
+  if (first_block < 0 || n_kv_global < 1 || first_block * s.B + s.n_kv > n_kv_global) return HISA_ERR_INVALID_ARG;
+  if (!q_idx || !block_keys || !cand_scores || !cand_ids) return HISA_ERR_INVALID_ARG;
+  if (!hisa::aligned16(q_idx) || !hisa::aligned16(block_keys)) return HISA_ERR_INVALID_ARG;
+  if (!workspace || !hisa::aligned16(workspace) || workspace_bytes < (size_t)s.n_query * s.n_blk * sizeof(float))
+    return HISA_ERR_WORKSPACE;
+  float* scores = static_cast<float*>(workspace);
+  cudaError_t e = hisa::launch_block_score(s, q_idx, block_keys, scores, stream);
+  if (e != cudaSuccess) return hisa::cuda_fail(e);
+  const int64_t c = (n_kv_global - 1) / s.B;
+  return hisa::cuda_fail(
+      hisa::launch_block_candidates(s, scores, first_block, c, s.m - 2, cand_scores, cand_ids, stream));
+}
+
+hisa_status_t hisa_topk_merge(const float* scores, const int32_t* ids, int32_t n_parts, int64_t rows, int32_t n_per,
+                              int32_t k, int32_t* out_ids, float* out_scores, cudaStream_t stream) {
+  if (!scores || !ids || !out_ids || n_parts < 1 || rows < 0 || rows > 0x7FFFFFFFLL || n_per < 1 || k < 1)
+    return HISA_ERR_INVALID_ARG;
+  if ((int64_t)n_parts * n_per > (1 << 24)) return HISA_ERR_UNSUPPORTED;
+  if (rows == 0) return HISA_OK;
+  return hisa::cuda_fail(hisa::launch_topk_merge(scores, ids, n_parts, rows, n_per, k, out_ids, out_scores, stream));
+}
+
+hisa_status_t hisa_remap_ids(const int32_t* in, int64_t rows, int32_t cols, int64_t lo, int64_t hi, int64_t delta,
+                             int32_t* out, cudaStream_t stream) {
+  if (!in || !out || rows < 0 || cols < 1 || lo > hi) return HISA_ERR_INVALID_ARG;
+  if (hi + delta > 0x7FFFFFFFLL || lo + delta < 0) return HISA_ERR_INVALID_ARG;
+  if (rows == 0) return HISA_OK;
+  return hisa::cuda_fail(hisa::launch_remap_ids(in, rows, cols, lo, hi, delta, out, stream));
+}
+
+hisa_status_t hisa_lse_merge(const void* o_parts, const float* lse_parts, int32_t n_parts, int64_t rows, int32_t d,
+                             void* o, float* lse, cudaStream_t stream) {
+  if (!o_parts || !lse_parts || !o || n_parts < 1 || rows < 0 || d < 1) return HISA_ERR_INVALID_ARG;
+  if (rows == 0) return HISA_OK;
+  return hisa::cuda_fail(hisa::launch_lse_merge(o_parts, lse_parts, n_parts, rows, d, o, lse, stream));
 }
 
 hisa_status_t hisa_gather_probe(const void* rows, int64_t n_rows, int32_t row_bytes, int64_t n_gathers, uint32_t seed,

@@ -62,6 +62,16 @@ cudaError_t launch_sparse_attn_tc(const Shape& s, const void* q, const void* k, 
                                   const int32_t* token_idx, void* o, float* lse, int32_t* status, int splits,
                                   float* partial, cudaStream_t st);
 
+// Context-parallel decode (see the hisa_block_candidates family in hisa.h).
+cudaError_t launch_block_candidates(const Shape& s, const float* scores, int64_t first, int64_t c, int r,
+                                    float* cand_scores, int32_t* cand_ids, cudaStream_t st);
+cudaError_t launch_topk_merge(const float* scores, const int32_t* ids, int n_parts, int64_t rows, int n_per, int k,
+                              int32_t* out_ids, float* out_scores, cudaStream_t st);
+cudaError_t launch_remap_ids(const int32_t* in, int64_t rows, int cols, int64_t lo, int64_t hi, int64_t delta,
+                             int32_t* out, cudaStream_t st);
+cudaError_t launch_lse_merge(const void* o_parts, const float* lse_parts, int G, int64_t rows, int d, void* o,
+                             float* lse, cudaStream_t st);
+
 // Measurement helper: gathers of hashed rows into shared memory (see hisa_gather_probe).
 bool gather_probe_row_bytes_ok(int row_bytes);
 cudaError_t launch_gather_probe(const void* rows, int64_t n_rows, int row_bytes, int64_t n_gathers, uint32_t seed,

@@ -186,6 +186,54 @@ hisa_status_t hisa_token_topk_noalloc(const hisa_params_t* params, const void* q
                                       const int32_t* block_idx, int32_t* token_idx, float* token_scores,
                                       int32_t* dev_status, cudaStream_t stream);
 
+/* ---- Decode with the context split across ranks (context parallelism) ----
+ * Rank r owns tokens [t0, t0 + n_loc) of every sequence, t0 = first_block * B
+ * (whole blocks; the last rank may end on a partial block), and runs the path
+ * on its slice with `local` parameters (n_kv = n_loc, n_q = 1).  The pages
+ * describe one device; splitting rests on two facts about the method: the
+ * selections of steps 3 and 5 ([IP] 1.2.1 item 3, 1.2.2 item 2; [QB]
+ * "塊級粗過濾", "塊內精挑字符") are the best entries under a total order
+ * (score descending, index ascending), so the global best r are among the
+ * union of every rank's best r; and attention over disjoint token sets merges
+ * by log-sum-exp ([QB] "HISA的關鍵優勢在於": the attention itself is unchanged).
+ * A step: hisa_block_candidates -> all-gather -> hisa_topk_merge (k = m) ->
+ * hisa_remap_ids (global -> local blocks) -> hisa_token_topk (local) ->
+ * hisa_remap_ids (local -> global tokens) -> all-gather -> hisa_topk_merge
+ * (k) -> hisa_remap_ids (global -> local tokens) -> sparse_attn_fwd (local)
+ * -> all-gather -> hisa_lse_merge.  All device pointers, asynchronous. */
+
+/* Scratch for hisa_block_candidates: n_q * batch * ceil(n_kv / B) floats of `local`. */
+hisa_status_t hisa_block_candidates_workspace_size(const hisa_params_t* local, size_t* bytes);
+/* This rank's block candidates for step 3: its best top_m - 2 blocks among the
+ * global blocks 1 .. c - 1 (c = (n_kv_global - 1) / B, the query's own block)
+ * by the block score of step 2, plus the forced blocks 0 and c if it owns
+ * them (score +inf).  Written as cand_scores / cand_ids [batch][top_m]
+ * (global block ids), ascending by id, padded with (NaN, -1).  local.n_q must
+ * be 1 (HISA_ERR_UNSUPPORTED otherwise); block_keys are this rank's pooled
+ * keys [batch][ceil(n_loc / B)][d_idx]. */
+hisa_status_t hisa_block_candidates(const hisa_params_t* local, int64_t n_kv_global, int64_t first_block,
+                                    const void* q_idx, const float* block_keys, float* cand_scores,
+                                    int32_t* cand_ids, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+/* The best k (score descending, id ascending) of each row's candidates, given
+ * as n_parts parts of [rows][n_per] each (the rank-major all-gather layout
+ * [n_parts][rows][n_per]; entries with id -1 are empty).  Ties are resolved by
+ * position, so the candidates must arrive in ascending id order within a row.
+ * out_ids [rows][k]: ascending ids, -1 padded; out_scores (nullable) aligned,
+ * NaN padded.  n_parts * n_per <= 2^24. */
+hisa_status_t hisa_topk_merge(const float* scores, const int32_t* ids, int32_t n_parts, int64_t rows, int32_t n_per,
+                              int32_t k, int32_t* out_ids, float* out_scores, cudaStream_t stream);
+/* Index renumbering between global and shard-local ids (no counterpart on the
+ * pages; argument marshalling between the steps above): for each row of
+ * in [rows][cols], the entries with lo <= id < hi, in order, shifted by delta,
+ * then -1.  in and out may be the same array. */
+hisa_status_t hisa_remap_ids(const int32_t* in, int64_t rows, int32_t cols, int64_t lo, int64_t hi, int64_t delta,
+                             int32_t* out, cudaStream_t stream);
+/* Attention over disjoint token sets merged: o_parts [n_parts][rows][d] bf16
+ * and lse_parts [n_parts][rows] (natural log, -inf for an empty set) ->
+ * o [rows][d] bf16, lse [rows] (nullable). */
+hisa_status_t hisa_lse_merge(const void* o_parts, const float* lse_parts, int32_t n_parts, int64_t rows, int32_t d,
+                             void* o, float* lse, cudaStream_t stream);
+
 /* Measurement helper, not a step of the method (the pages have no
  * counterpart): n_gathers copies of row h(e) (row_bytes each; h a hash of the
  * gather number e and seed, uniform over [0, n_rows)) into shared memory with
