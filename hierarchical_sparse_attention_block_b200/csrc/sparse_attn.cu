@@ -41,7 +41,10 @@
 namespace hisa {
 namespace {
 
-constexpr int kNW = 4;  // warps per CTA
+#ifndef HISA_ATTN_WARPS
+#define HISA_ATTN_WARPS 4
+#endif
+constexpr int kNW = HISA_ATTN_WARPS;  // warps per CTA
 
 template <int D, int TT, int NS>
 struct AttnCfg {
