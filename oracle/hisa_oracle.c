@@ -20,7 +20,11 @@
  *
  * Readings of points the pages leave open (each one is listed with its reason
  * in the design notes):
- *   - the indexer score is a single-head dot product q.k;
+ *   - the indexer score is a single-head dot product q.k, or, when the
+ *     indexer has H >= 1 query heads, sum_j w_j * max(0, q_j . k) with the
+ *     query's head weights w_j (the original indexer's own score function,
+ *     which [IP] 1.3 item 4 asks to keep; the form is the multi-head indexer
+ *     of DeepSeek-V3.2);
  *   - "first and last block" = block 0 and the query's own block
  *     c = floor(p / B), the newest block the query can see;
  *   - the two forced blocks count toward m;
@@ -74,6 +78,30 @@ static double dot_bf16_f64(const uint16_t *a, const double *b, int32_t n) {
   return s;
 }
 
+/* The indexer's score of one key -- [IP] 1.2.1 item 2 and 1.2.2 item 1 (the
+ * original indexer's score function), 1.3 item 4 (the same score function as
+ * the original model).  n_idx_heads = 0: the dot product q . key.
+ * n_idx_heads = H >= 1: sum over the query's H heads q_j ([H][d_idx]) of
+ * w_j * max(0, q_j . key).  One version per key type: block keys are fp64
+ * means, token keys bf16. */
+static double relu(double x) { return x > 0.0 ? x : 0.0; }
+
+static double score_block_key(const uint16_t *q, const double *w, int32_t n_idx_heads, const double *key,
+                              int32_t d_idx) {
+  if (n_idx_heads == 0) return dot_bf16_f64(q, key, d_idx);
+  double s = 0.0;
+  for (int32_t j = 0; j < n_idx_heads; ++j) s += w[j] * relu(dot_bf16_f64(q + (int64_t)j * d_idx, key, d_idx));
+  return s;
+}
+
+static double score_token_key(const uint16_t *q, const double *w, int32_t n_idx_heads, const uint16_t *key,
+                              int32_t d_idx) {
+  if (n_idx_heads == 0) return dot_bf16_bf16(q, key, d_idx);
+  double s = 0.0;
+  for (int32_t j = 0; j < n_idx_heads; ++j) s += w[j] * relu(dot_bf16_bf16(q + (int64_t)j * d_idx, key, d_idx));
+  return s;
+}
+
 /* Step 1 -- [IP] 1.2.1 item 1, [QB] "塊級粗過濾" first bullet: cut the keys into
  * fixed blocks of B tokens and mean-pool each block into one block key.  The
  * last block may be partial; its mean is over the tokens it holds.
@@ -94,13 +122,15 @@ void hisa_oracle_block_pool(const uint16_t *k_idx, int64_t n_kv, int32_t d_idx, 
 
 /* Steps 2-3 -- [IP] 1.2.1 items 2-3, [QB] "塊級粗過濾" bullets 2-3 and the
  * forced-block remark of "塊內精挑字符": score the query against the block keys
- * it can see with the indexer's dot product and keep m blocks, always
+ * it can see with the indexer's score and keep m blocks, always
  * including the first block and the query's own block.
  * Returns s = min(m, c+1), the number of selected blocks.  sel[0..m) receives
  * the selected block ids in ascending order, -1 padded.  sel_scores (may be
- * NULL) receives q . block_key for each selected block (NAN for padding). */
-int32_t hisa_oracle_block_topm(const uint16_t *q_row, const double *block_keys, int32_t d_idx, int32_t block,
-                               int64_t p, int32_t top_m, int32_t *sel, double *sel_scores) {
+ * NULL) receives the score of each selected block (NAN for padding).  q_row:
+ * [max(1, n_idx_heads)][d_idx]; w: [n_idx_heads] (unused when 0). */
+int32_t hisa_oracle_block_topm(const uint16_t *q_row, const double *w, int32_t n_idx_heads, const double *block_keys,
+                               int32_t d_idx, int32_t block, int64_t p, int32_t top_m, int32_t *sel,
+                               double *sel_scores) {
   int64_t c = p / block; /* the query's own block */
   int64_t n_vis = c + 1;
   int64_t s = top_m < n_vis ? top_m : n_vis;
@@ -113,7 +143,7 @@ int32_t hisa_oracle_block_topm(const uint16_t *q_row, const double *block_keys, 
     int64_t n_mid = c - 1;
     scored_t *cand = (scored_t *)malloc(sizeof(scored_t) * (size_t)n_mid);
     for (int64_t j = 1; j <= c - 1; ++j) {
-      cand[j - 1].score = dot_bf16_f64(q_row, block_keys + j * d_idx, d_idx);
+      cand[j - 1].score = score_block_key(q_row, w, n_idx_heads, block_keys + j * d_idx, d_idx);
       cand[j - 1].index = j;
     }
     qsort(cand, (size_t)n_mid, sizeof(scored_t), by_score_desc_index_asc);
@@ -126,7 +156,8 @@ int32_t hisa_oracle_block_topm(const uint16_t *q_row, const double *block_keys, 
   for (int64_t r = n; r < top_m; ++r) sel[r] = -1;
   if (sel_scores) {
     for (int64_t r = 0; r < top_m; ++r)
-      sel_scores[r] = sel[r] >= 0 ? dot_bf16_f64(q_row, block_keys + (int64_t)sel[r] * d_idx, d_idx) : NAN;
+      sel_scores[r] =
+          sel[r] >= 0 ? score_block_key(q_row, w, n_idx_heads, block_keys + (int64_t)sel[r] * d_idx, d_idx) : NAN;
   }
   return (int32_t)s;
 }
@@ -150,9 +181,9 @@ static int32_t keep_top_k(scored_t *cand, int64_t n, int32_t top_k, int32_t *tok
  * indexer's format (ascending token ids, -1 padded), so attention is unchanged.
  * k_idx: [n_kv][d_idx] of the query's sequence.  Returns k_eff; *n_cand gets
  * the number of candidates scanned. */
-int32_t hisa_oracle_token_topk(const uint16_t *q_row, const uint16_t *k_idx, int32_t d_idx, int32_t block,
-                               int64_t n_kv, int64_t p, const int32_t *sel, int32_t top_m, int32_t top_k,
-                               int32_t *tok, double *tok_scores, int64_t *n_cand) {
+int32_t hisa_oracle_token_topk(const uint16_t *q_row, const double *w, int32_t n_idx_heads, const uint16_t *k_idx,
+                               int32_t d_idx, int32_t block, int64_t n_kv, int64_t p, const int32_t *sel,
+                               int32_t top_m, int32_t top_k, int32_t *tok, double *tok_scores, int64_t *n_cand) {
   int64_t cap = (int64_t)top_m * block, n = 0;
   scored_t *cand = (scored_t *)malloc(sizeof(scored_t) * (size_t)(cap > 0 ? cap : 1));
   for (int32_t r = 0; r < top_m; ++r) {
@@ -162,7 +193,7 @@ int32_t hisa_oracle_token_topk(const uint16_t *q_row, const uint16_t *k_idx, int
     if (t1 > n_kv) t1 = n_kv;
     if (t1 > p + 1) t1 = p + 1;
     for (int64_t t = t0; t < t1; ++t) {
-      cand[n].score = dot_bf16_bf16(q_row, k_idx + t * d_idx, d_idx);
+      cand[n].score = score_token_key(q_row, w, n_idx_heads, k_idx + t * d_idx, d_idx);
       cand[n].index = t;
       ++n;
     }
@@ -175,11 +206,11 @@ int32_t hisa_oracle_token_topk(const uint16_t *q_row, const uint16_t *k_idx, int
 
 /* The flat token indexer the two-level one replaces ([IP] 1.1 item 1, [QB]
  * "兩步消除上下文索引瓶頸"): score every token t <= p and keep the top k. */
-int32_t hisa_oracle_flat_topk(const uint16_t *q_row, const uint16_t *k_idx, int32_t d_idx, int64_t p,
-                              int32_t top_k, int32_t *tok, double *tok_scores) {
+int32_t hisa_oracle_flat_topk(const uint16_t *q_row, const double *w, int32_t n_idx_heads, const uint16_t *k_idx,
+                              int32_t d_idx, int64_t p, int32_t top_k, int32_t *tok, double *tok_scores) {
   scored_t *cand = (scored_t *)malloc(sizeof(scored_t) * (size_t)(p + 1));
   for (int64_t t = 0; t <= p; ++t) {
-    cand[t].score = dot_bf16_bf16(q_row, k_idx + t * d_idx, d_idx);
+    cand[t].score = score_token_key(q_row, w, n_idx_heads, k_idx + t * d_idx, d_idx);
     cand[t].index = t;
   }
   int32_t k_eff = keep_top_k(cand, p + 1, top_k, tok, tok_scores);
@@ -230,11 +261,13 @@ void hisa_oracle_sparse_attn(const uint16_t *q_row, const uint16_t *k, const uin
 /* The whole path for a list of queries (ids seq * n_q + i; position
  * p = n_kv - n_q + i), in parallel over queries.  block_keys comes from
  * hisa_oracle_block_pool of every sequence ([batch][n_blk][d_idx]).  Outputs
- * are one row per listed query.  With flat != 0 the token list comes from the
+ * are one row per listed query.  q_idx: [batch][n_q][max(1, n_idx_heads)][d_idx];
+ * idx_w: [batch][n_q][n_idx_heads] (NULL when n_idx_heads is 0).  With flat != 0 the token list comes from the
  * flat indexer and block_idx is left untouched.  q, k, v may be NULL (indexer
  * only).  n_cand (may be NULL) gets the candidates each query scanned. */
 int32_t hisa_oracle_run(int32_t batch, int64_t n_q, int64_t n_kv, int32_t d_idx, int32_t block, int32_t top_m,
                         int32_t top_k, int32_t n_heads, int32_t n_kv_heads, int32_t d_head, double scale,
+                        int32_t n_idx_heads, const double *idx_w,
                         const uint16_t *q_idx, const uint16_t *k_idx, const double *block_keys, const uint16_t *q,
                         const uint16_t *k, const uint16_t *v, const int64_t *query_ids, int64_t n_queries,
                         int32_t *block_idx, int32_t *token_idx, double *o, double *lse, int64_t *n_cand,
@@ -252,17 +285,20 @@ int32_t hisa_oracle_run(int32_t batch, int64_t n_q, int64_t n_kv, int32_t d_idx,
       continue;
     }
     int64_t p = n_kv - n_q + i;
-    const uint16_t *qi = q_idx + id * d_idx;
+    const int32_t qh = n_idx_heads > 0 ? n_idx_heads : 1;
+    const uint16_t *qi = q_idx + id * qh * d_idx;
+    const double *wi = n_idx_heads > 0 ? idx_w + id * n_idx_heads : NULL;
     const uint16_t *ks = k_idx + seq * n_kv * d_idx;
     int32_t *tok = token_idx + r * top_k;
     int64_t nc = 0;
     if (flat) {
-      hisa_oracle_flat_topk(qi, ks, d_idx, p, top_k, tok, NULL);
+      hisa_oracle_flat_topk(qi, wi, n_idx_heads, ks, d_idx, p, top_k, tok, NULL);
       nc = p + 1;
     } else {
       int32_t *sel = block_idx + r * top_m;
-      hisa_oracle_block_topm(qi, block_keys + seq * n_blk * d_idx, d_idx, block, p, top_m, sel, NULL);
-      hisa_oracle_token_topk(qi, ks, d_idx, block, n_kv, p, sel, top_m, top_k, tok, NULL, &nc);
+      hisa_oracle_block_topm(qi, wi, n_idx_heads, block_keys + seq * n_blk * d_idx, d_idx, block, p, top_m, sel,
+                             NULL);
+      hisa_oracle_token_topk(qi, wi, n_idx_heads, ks, d_idx, block, n_kv, p, sel, top_m, top_k, tok, NULL, &nc);
     }
     if (n_cand) n_cand[r] = nc;
     if (q && k && v && o && lse) {

@@ -16,6 +16,8 @@ Value maps
   * integer indexer values: ``((u >> 32) * 9 >> 32) - 4`` in {-4..4}, stored as
     exact bf16.  With these, every block sum and dot product of the indexer is
     an integer below 2**24, so fp32 results are exact.
+  * head weights of a multi-head indexer: ``((u >> 32) * 5 >> 32)`` mapped to
+    {-2, -1, 1, 2, 3} (fp32), so every weighted score stays an exact integer.
   * unit-variance stand-ins for N(0,1): Irwin-Hall with n = 4 over the four
     16-bit fields of ``u``: ``(sum - 131070) * C`` with ``C = sqrt(3/(2**32-1))``
     rounded once to fp32, one fp32 multiply (round to nearest even), then bf16
@@ -30,7 +32,7 @@ _M1 = np.uint64(0xBF58476D1CE4E5B9)
 _M2 = np.uint64(0x94D049BB133111EB)
 
 # Tensor ids of the streams.
-T_QIDX, T_KIDX, T_Q, T_K, T_V, T_NEEDLE = 1, 2, 3, 4, 5, 6
+T_QIDX, T_KIDX, T_Q, T_K, T_V, T_NEEDLE, T_WIDX = 1, 2, 3, 4, 5, 6, 7
 
 # fp32 constant sqrt(3 / (65536**2 - 1)); the value the device generator uses
 # is the same bit pattern (checked in tests).
@@ -74,6 +76,15 @@ def _f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
 
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
     return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+_WEIGHTS = np.array([-2.0, -1.0, 1.0, 2.0, 3.0], dtype=np.float32)
+
+
+def weight_values(seed: int, tensor: int, start: int, count: int) -> np.ndarray:
+    """Indexer head weights in {-2, -1, 1, 2, 3} as fp32."""
+    u = raw_u64(seed, tensor, start, count)
+    return _WEIGHTS[((u >> np.uint64(32)) * np.uint64(5)) >> np.uint64(32)]
 
 
 def int_values(seed: int, tensor: int, start: int, count: int) -> np.ndarray:

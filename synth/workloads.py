@@ -14,7 +14,7 @@ from dataclasses import dataclass, replace
 
 import numpy as np
 
-from . import (T_K, T_KIDX, T_Q, T_QIDX, T_V, apply_needles, int_bf16, int_values,
+from . import (T_K, T_KIDX, T_Q, T_QIDX, T_V, T_WIDX, apply_needles, int_bf16, int_values, weight_values,
                needle_blocks, needle_signs, normal_bf16)
 
 
@@ -33,6 +33,7 @@ class Workload:
     d_head: int
     needles: int = 0
     seed: int = 0
+    n_idx_heads: int = 0  # 0: one indexer head scored by a plain dot product; H >= 1: H heads, weighted ReLU
 
     @property
     def n_blk(self) -> int:
@@ -54,13 +55,23 @@ WORKLOADS = {
 
 
 def q_idx_rows(w: Workload, seq: int, i0: int, count: int) -> np.ndarray:
-    """bf16 bits of q_idx[seq][i0:i0+count] -> uint16 [count][d_idx]."""
-    start = (seq * w.n_q + i0) * w.d_idx
-    return int_bf16(w.seed, T_QIDX, start, count * w.d_idx).reshape(count, w.d_idx)
+    """bf16 bits of q_idx[seq][i0:i0+count] -> uint16 [count][d_idx] ([count][H_idx][d_idx] with a
+    multi-head indexer)."""
+    nh = max(1, w.n_idx_heads)
+    start = (seq * w.n_q + i0) * nh * w.d_idx
+    rows = int_bf16(w.seed, T_QIDX, start, count * nh * w.d_idx)
+    return rows.reshape(count, w.d_idx) if w.n_idx_heads == 0 else rows.reshape(count, nh, w.d_idx)
+
+
+def w_idx_rows(w: Workload, seq: int, i0: int, count: int) -> np.ndarray:
+    """Indexer head weights [count][H_idx] (fp32) of queries i0 .. i0+count-1."""
+    return weight_values(w.seed, T_WIDX, (seq * w.n_q + i0) * w.n_idx_heads,
+                         count * w.n_idx_heads).reshape(count, w.n_idx_heads)
 
 
 def probe_signs(w: Workload, seq: int) -> np.ndarray:
-    return needle_signs(q_idx_rows(w, seq, w.n_q - 1, 1)[0])
+    q = q_idx_rows(w, seq, w.n_q - 1, 1)[0]
+    return needle_signs(q if q.ndim == 1 else q[0])  # a multi-head indexer: its first head
 
 
 def needle_table(w: Workload, seq: int) -> np.ndarray:
@@ -131,4 +142,7 @@ def full_inputs(w: Workload) -> dict:
     allt = np.arange(w.n_kv)
     k = np.stack([k_rows(w, s, allt) for s in range(w.batch)])
     v = np.stack([v_rows(w, s, allt) for s in range(w.batch)])
-    return {"q_idx": q_idx, "k_idx": k_idx, "q": q, "k": k, "v": v}
+    out = {"q_idx": q_idx, "k_idx": k_idx, "q": q, "k": k, "v": v}
+    if w.n_idx_heads:
+        out["w_idx"] = np.stack([w_idx_rows(w, s, 0, w.n_q) for s in range(w.batch)])
+    return out

@@ -315,6 +315,81 @@ def check_attention_special_cases(O):
         assert np.array_equal(og[hh], _bf16_to_f64(vv[5, 0]))
 
 
+# ---------------------------------------------------------------- the multi-head indexer score
+
+def _mh_case(rng, n_kv, d, heads):
+    q = _ints(rng, (heads, d))
+    k = _ints(rng, (n_kv, d))
+    w = rng.choice(np.array([-2.0, -1.0, 1.0, 2.0, 3.0]), size=heads)
+    return q, k, w
+
+
+def _mh_score_int(q, w, key_int):
+    """sum_j w_j * max(0, q_j . key) in exact integer arithmetic (int64)."""
+    dots = q.astype(np.int64) @ key_int.astype(np.int64)
+    return sum(int(w[j]) * max(0, int(dots[j])) for j in range(len(w)))
+
+
+def check_multihead_token_scores_bruteforce(O):
+    """Token scores and top-k of the multi-head indexer equal a brute-force integer evaluation of
+    sum_j w_j * ReLU(q_j . k) ranked by numpy lexsort."""
+    rng = np.random.default_rng(31)
+    for heads, n_kv, block, top_m, top_k in [(1, 90, 8, 4, 17), (3, 200, 16, 5, 40), (8, 130, 32, 3, 64)]:
+        d = 16
+        q, k, w = _mh_case(rng, n_kv, d, heads)
+        p = n_kv - 1
+        sel = np.arange(0, -(-n_kv // block), dtype=np.int32)  # every block: all tokens are candidates
+        sel_m = np.full(len(sel), -1, dtype=np.int32)
+        sel_m[: len(sel)] = sel
+        tok, k_eff, _, sc = O.token_topk(_bf(q), _bf(k), block, p, sel_m, top_k, scores=True, w=w)
+        exact = np.array([_mh_score_int(q, w, k[t]) for t in range(n_kv)])
+        want = np.sort(_order(exact, np.arange(n_kv))[:top_k])
+        assert k_eff == min(top_k, n_kv)
+        assert np.array_equal(tok[:k_eff], want), (heads, tok[:k_eff], want)
+        assert np.array_equal(sc[:k_eff], exact[tok[:k_eff]].astype(np.float64))
+
+
+def check_multihead_block_scores_exact(O):
+    """Block scores of the multi-head indexer equal sum_j w_j * ReLU(q_j . mean) in exact rational
+    arithmetic, and the kept blocks are the forced pair plus the best m-2 by those scores."""
+    rng = np.random.default_rng(37)
+    for heads, n_kv, block, top_m in [(2, 300, 16, 6), (5, 257, 8, 9)]:
+        d = 8
+        q, k, w = _mh_case(rng, n_kv, d, heads)
+        bk = O.block_pool(_bf(k), block)
+        p = n_kv - 1
+        c = p // block
+        sel, s_, sc = O.block_topm(_bf(q), bk, block, p, top_m, scores=True, w=w)
+        exact = []
+        for j in range(c + 1):
+            t0, t1 = j * block, min(n_kv, (j + 1) * block)
+            mean = [Fraction(int(k[t0:t1, e].sum()), t1 - t0) for e in range(d)]
+            sj = sum(Fraction(int(w[h])) * max(Fraction(0), sum(int(q[h, e]) * mean[e] for e in range(d)))
+                     for h in range(heads))
+            exact.append(sj)
+        mid = _order(np.array([float(x) for x in exact[1:c]]), np.arange(1, c))[: s_ - 2]
+        assert np.array_equal(sel[:s_], np.sort(np.concatenate([[0, c], mid]))), (sel, mid)
+        for r in range(s_):
+            assert sc[r] == float(exact[sel[r]])
+
+
+def check_multihead_reduces_to_dot_product(O):
+    """One head with weight 1 and non-negative inputs (so every dot product is >= 0 and the ReLU
+    is the identity) selects exactly what the plain dot-product indexer selects."""
+    rng = np.random.default_rng(41)
+    n_kv, d, block, top_m, top_k = 400, 16, 16, 6, 50
+    q = _ints(rng, (d,), 0, 4)
+    k = _ints(rng, (n_kv, d), 0, 4)
+    bk = O.block_pool(_bf(k), block)
+    p = n_kv - 1
+    sel_plain, _ = O.block_topm(_bf(q), bk, block, p, top_m)
+    sel_mh, _ = O.block_topm(_bf(q[None]), bk, block, p, top_m, w=np.array([1.0]))
+    assert np.array_equal(sel_plain, sel_mh)
+    tok_plain, _, _ = O.token_topk(_bf(q), _bf(k), block, p, sel_plain, top_k)
+    tok_mh, _, _ = O.token_topk(_bf(q[None]), _bf(k), block, p, sel_plain, top_k, w=np.array([1.0]))
+    assert np.array_equal(tok_plain, tok_mh)
+
+
 ALL_CHECKS = [
     check_pool_exact,
     check_block_scores_exact,
@@ -326,4 +401,7 @@ ALL_CHECKS = [
     check_constructed_ranking,
     check_dense_equivalence,
     check_attention_special_cases,
+    check_multihead_token_scores_bruteforce,
+    check_multihead_block_scores_exact,
+    check_multihead_reduces_to_dot_product,
 ]

@@ -52,6 +52,15 @@ MUTANTS = [
     ("wrong query-head to kv-head map",
      "int32_t g = h / group;",
      "int32_t g = h % n_kv_heads;"),
+    ("multi-head block score without the ReLU",
+     "s += w[j] * relu(dot_bf16_f64(q + (int64_t)j * d_idx, key, d_idx));",
+     "s += w[j] * dot_bf16_f64(q + (int64_t)j * d_idx, key, d_idx);"),
+    ("multi-head token score ignores the head weights",
+     "s += w[j] * relu(dot_bf16_bf16(q + (int64_t)j * d_idx, key, d_idx));",
+     "s += relu(dot_bf16_bf16(q + (int64_t)j * d_idx, key, d_idx));"),
+    ("multi-head token score reads head 0 for every head",
+     "s += w[j] * relu(dot_bf16_bf16(q + (int64_t)j * d_idx, key, d_idx));",
+     "s += w[j] * relu(dot_bf16_bf16(q, key, d_idx));"),
 ]
 
 
