@@ -231,6 +231,7 @@ def run_ours(a, rank, world, local_rank):
     w = workload(a, rank)
     p = hs.params_of(w)
     inp = sd.device_inputs(w, device=dev)
+    wi = inp.get("w_idx")  # the indexer's head weights (multi-head indexer only)
     torch.cuda.synchronize()
     st = torch.cuda.Stream(device=dev)  # a side stream: CUDA graphs cannot be captured on the default one
     torch.cuda.set_stream(st)
@@ -268,9 +269,9 @@ def run_ours(a, rank, world, local_rank):
         ev[0].record(st)
         hs.hisa_block_pool(p, inp["k_idx"], bk, pool_begin, -1, stream=st)
         ev[1].record(st)
-        hs.hisa_block_topm(p, inp["q_idx"], bk, blk, None, status, ws_topm, stream=st)
+        hs.hisa_block_topm(p, inp["q_idx"], bk, blk, None, status, ws_topm, stream=st, idx_weights=wi)
         ev[2].record(st)
-        hs.hisa_token_topk(p, inp["q_idx"], inp["k_idx"], blk, tok, None, status, ws_tok, stream=st)
+        hs.hisa_token_topk(p, inp["q_idx"], inp["k_idx"], blk, tok, None, status, ws_tok, stream=st, idx_weights=wi)
         ev[3].record(st)
         hs.sparse_attn_fwd(p, inp["q"], inp["k"], inp["v"], tok, o, lse, status, ws_attn, stream=st)
         ev[4].record(st)
@@ -291,8 +292,9 @@ def run_ours(a, rank, world, local_rank):
     if use_graph:
         calls = [
             lambda: hs.hisa_block_pool(p, inp["k_idx"], bk, pool_begin, -1, stream=st),
-            lambda: hs.hisa_block_topm(p, inp["q_idx"], bk, blk, None, status, ws_topm, stream=st),
-            lambda: hs.hisa_token_topk(p, inp["q_idx"], inp["k_idx"], blk, tok, None, status, ws_tok, stream=st),
+            lambda: hs.hisa_block_topm(p, inp["q_idx"], bk, blk, None, status, ws_topm, stream=st, idx_weights=wi),
+            lambda: hs.hisa_token_topk(p, inp["q_idx"], inp["k_idx"], blk, tok, None, status, ws_tok, stream=st,
+                                       idx_weights=wi),
             lambda: hs.sparse_attn_fwd(p, inp["q"], inp["k"], inp["v"], tok, o, lse, status, ws_attn, stream=st),
         ]
         graphs = []
@@ -320,14 +322,14 @@ def run_ours(a, rank, world, local_rank):
         fmin, fpref = hs.hisa_flat_topk_workspace_size(p)
         ws_flat = torch.empty(fpref, dtype=torch.uint8, device=dev)
         for _ in range(2):
-            hs.hisa_flat_topk(p, inp["q_idx"], inp["k_idx"], flat_tok, None, ws_flat, stream=st)
+            hs.hisa_flat_topk(p, inp["q_idx"], inp["k_idx"], flat_tok, None, ws_flat, stream=st, idx_weights=wi)
         reps = max(2, min(a.steps, 5))
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         tt = []
         for _ in range(reps):
             flush.zero_()
             e0.record(st)
-            hs.hisa_flat_topk(p, inp["q_idx"], inp["k_idx"], flat_tok, None, ws_flat, stream=st)
+            hs.hisa_flat_topk(p, inp["q_idx"], inp["k_idx"], flat_tok, None, ws_flat, stream=st, idx_weights=wi)
             e1.record(st)
             e1.synchronize()
             tt.append(e0.elapsed_time(e1))
@@ -438,9 +440,13 @@ def run_e2e(a, hs, w, p, inp, dev, st, world):
     import torch
 
     names = ["q_idx", "q"] if w.n_q == 1 else ["q_idx", "k_idx", "q", "k", "v"]
+    all_names = ["q_idx", "k_idx", "q", "k", "v"]
+    if "w_idx" in inp:  # the indexer's head weights come with each step's queries
+        names.append("w_idx")
+        all_names.append("w_idx")
     host = {k: inp[k].cpu().pin_memory() for k in names}
     d_in = {k: (torch.empty_like(v, device=dev) if k in host else v) for k, v in
-            ((k, host.get(k, inp[k])) for k in ["q_idx", "k_idx", "q", "k", "v"])}
+            ((k, host.get(k, inp[k])) for k in all_names)}
     o = torch.empty((w.batch, w.n_q, w.n_heads, w.d_head), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((w.batch, w.n_q, w.n_heads), dtype=torch.float32, device=dev)
     h_o = torch.empty(o.shape, dtype=o.dtype).pin_memory()
@@ -459,10 +465,10 @@ def run_e2e(a, hs, w, p, inp, dev, st, world):
             d_in[k].copy_(host[k], non_blocking=True)
         if decode:
             hs.hisa_forward_cached(p, d_in["q_idx"], d_in["k_idx"], bk, w.n_blk - 1, d_in["q"], d_in["k"], d_in["v"],
-                                   o, lse, None, None, None, ws, stream=st)
+                                   o, lse, None, None, None, ws, stream=st, idx_weights=d_in.get("w_idx"))
         else:
             hs.hisa_forward(p, d_in["q_idx"], d_in["k_idx"], d_in["q"], d_in["k"], d_in["v"], o, lse, None, None,
-                            None, ws, stream=st)
+                            None, ws, stream=st, idx_weights=d_in.get("w_idx"))
         h_o.copy_(o, non_blocking=True)
         h_lse.copy_(lse, non_blocking=True)
 
@@ -495,7 +501,9 @@ def oracle_sample(w, seconds: float, device_inputs=None):
     O = oracle.Oracle()
     threads = O.threads()
     if device_inputs is not None:
-        inp = {k: v.view(__import__("torch").int16).cpu().numpy().view(np.uint16)
+        import torch
+
+        inp = {k: (v.cpu().numpy() if v.dtype == torch.float32 else v.view(torch.int16).cpu().numpy().view(np.uint16))
                for k, v in device_inputs.items() if not k.startswith("_")}
     else:
         inp = full_inputs(w)
@@ -540,7 +548,7 @@ def oracle_sample_rows(w, seconds: float):
     import numpy as np
 
     import oracle
-    from synth.workloads import k_idx_rows, k_rows, q_idx_rows, q_rows, v_rows
+    from synth.workloads import k_idx_rows, k_rows, q_idx_rows, q_rows, v_rows, w_idx_rows
 
     O = oracle.Oracle()
     timed, done_q, seqs = 0.0, 0, 0
@@ -553,9 +561,10 @@ def oracle_sample_rows(w, seconds: float):
         for i in range(w.n_q):
             p = w.n_kv - w.n_q + i
             qi = q_idx_rows(w, seq, i, 1)[0]
+            wi = w_idx_rows(w, seq, i, 1)[0] if w.n_idx_heads else None
             t0 = time.perf_counter()
-            sel, _ = O.block_topm(qi, bk, w.block, p, w.top_m)
-            tok, _, _ = O.token_topk(qi, k_idx, w.block, p, sel, w.top_k)
+            sel, _ = O.block_topm(qi, bk, w.block, p, w.top_m, w=wi)
+            tok, _, _ = O.token_topk(qi, k_idx, w.block, p, sel, w.top_k, w=wi)
             timed += time.perf_counter() - t0
             valid = tok[tok >= 0]
             kk, vv = k_rows(w, seq, valid), v_rows(w, seq, valid)

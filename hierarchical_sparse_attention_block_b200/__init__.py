@@ -36,7 +36,7 @@ class HisaParams(ctypes.Structure):
         ("batch", ctypes.c_int32), ("d_idx", ctypes.c_int32), ("n_q", ctypes.c_int64), ("n_kv", ctypes.c_int64),
         ("block", ctypes.c_int32), ("top_m", ctypes.c_int32), ("top_k", ctypes.c_int32),
         ("n_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32), ("d_head", ctypes.c_int32),
-        ("scale", ctypes.c_float), ("flags", ctypes.c_int32),
+        ("scale", ctypes.c_float), ("flags", ctypes.c_int32), ("n_idx_heads", ctypes.c_int32),
     ]
 
 
@@ -59,20 +59,20 @@ def _load():
     sig = {
         "hisa_block_pool": [pp, vp, i64, i64, vp, vp],
         "hisa_block_topm_workspace_size": [pp, sz],
-        "hisa_block_topm": [pp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
+        "hisa_block_topm": [pp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
         "hisa_token_topk_workspace_size": [pp, sz, sz],
-        "hisa_token_topk": [pp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
+        "hisa_token_topk": [pp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
         "hisa_sparse_attn_workspace_size": [pp, sz],
         "sparse_attn_fwd": [pp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
         "hisa_forward_workspace_size": [pp, sz],
-        "hisa_forward": [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
+        "hisa_forward": [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
         "hisa_flat_topk_workspace_size": [pp, sz, sz],
-        "hisa_flat_topk": [pp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
-        "hisa_token_topk_noalloc": [pp, vp, vp, vp, vp, vp, vp, vp],
-        "hisa_forward_cached": [pp, vp, vp, vp, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
+        "hisa_flat_topk": [pp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
+        "hisa_token_topk_noalloc": [pp, vp, vp, vp, vp, vp, vp, vp, vp],
+        "hisa_forward_cached": [pp, vp, vp, vp, vp, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
         "hisa_gather_probe": [vp, i64, ctypes.c_int32, i64, ctypes.c_uint32, vp, vp],
         "hisa_block_candidates_workspace_size": [pp, sz],
-        "hisa_block_candidates": [pp, i64, i64, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
+        "hisa_block_candidates": [pp, i64, i64, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
         "hisa_topk_merge": [vp, vp, ctypes.c_int32, i64, ctypes.c_int32, ctypes.c_int32, vp, vp, vp],
         "hisa_remap_ids": [vp, i64, ctypes.c_int32, i64, i64, i64, vp, vp],
         "hisa_lse_merge": [vp, vp, ctypes.c_int32, i64, ctypes.c_int32, vp, vp, vp],
@@ -96,15 +96,16 @@ def lib():
 
 
 def params(batch, n_q, n_kv, d_idx, block, top_m, top_k, n_heads=1, n_kv_heads=None, d_head=64,
-           scale=0.0) -> HisaParams:
+           scale=0.0, n_idx_heads=0) -> HisaParams:
     return HisaParams(batch=batch, d_idx=d_idx, n_q=n_q, n_kv=n_kv, block=block, top_m=top_m, top_k=top_k,
                       n_heads=n_heads, n_kv_heads=n_kv_heads if n_kv_heads else n_heads, d_head=d_head,
-                      scale=scale, flags=0)
+                      scale=scale, flags=0, n_idx_heads=n_idx_heads)
 
 
 def params_of(w) -> HisaParams:
     """hisa_params_t of a workload description (synth.workloads.Workload or alike)."""
-    return params(w.batch, w.n_q, w.n_kv, w.d_idx, w.block, w.top_m, w.top_k, w.n_heads, w.n_kv_heads, w.d_head)
+    return params(w.batch, w.n_q, w.n_kv, w.d_idx, w.block, w.top_m, w.top_k, w.n_heads, w.n_kv_heads, w.d_head,
+                  n_idx_heads=getattr(w, "n_idx_heads", 0))
 
 
 def _ptr(t):
@@ -152,10 +153,11 @@ def hisa_block_topm_workspace_size(p) -> int:
 
 
 def hisa_block_topm(p, q_idx, block_keys, block_idx, block_scores=None, dev_status=None, workspace=None,
-                    stream=None):
+                    stream=None, idx_weights=None):
     if workspace is None:
         workspace = _workspace(hisa_block_topm_workspace_size(p), q_idx.device)
-    _check("hisa_block_topm", _lib.hisa_block_topm(ctypes.byref(p), _ptr(q_idx), _ptr(block_keys), _ptr(block_idx),
+    _check("hisa_block_topm", _lib.hisa_block_topm(ctypes.byref(p), _ptr(q_idx), _ptr(idx_weights), _ptr(block_keys),
+                                                   _ptr(block_idx),
                                                    _ptr(block_scores), _ptr(dev_status), _ptr(workspace),
                                                    workspace.numel(), _stream(stream)))
 
@@ -166,10 +168,11 @@ def hisa_token_topk_workspace_size(p):
 
 
 def hisa_token_topk(p, q_idx, k_idx, block_idx, token_idx, token_scores=None, dev_status=None, workspace=None,
-                    stream=None):
+                    stream=None, idx_weights=None):
     if workspace is None:
         workspace = _workspace(hisa_token_topk_workspace_size(p)[1], q_idx.device)
-    _check("hisa_token_topk", _lib.hisa_token_topk(ctypes.byref(p), _ptr(q_idx), _ptr(k_idx), _ptr(block_idx),
+    _check("hisa_token_topk", _lib.hisa_token_topk(ctypes.byref(p), _ptr(q_idx), _ptr(idx_weights), _ptr(k_idx),
+                                                   _ptr(block_idx),
                                                    _ptr(token_idx), _ptr(token_scores), _ptr(dev_status),
                                                    _ptr(workspace), workspace.numel(), _stream(stream)))
 
@@ -192,20 +195,22 @@ def hisa_forward_workspace_size(p) -> int:
 
 
 def hisa_forward(p, q_idx, k_idx, q, k, v, o, lse=None, block_idx_out=None, token_idx_out=None, dev_status=None,
-                 workspace=None, stream=None):
+                 workspace=None, stream=None, idx_weights=None):
     if workspace is None:
         workspace = _workspace(hisa_forward_workspace_size(p), q_idx.device)
-    _check("hisa_forward", _lib.hisa_forward(ctypes.byref(p), _ptr(q_idx), _ptr(k_idx), _ptr(q), _ptr(k), _ptr(v),
+    _check("hisa_forward", _lib.hisa_forward(ctypes.byref(p), _ptr(q_idx), _ptr(idx_weights), _ptr(k_idx), _ptr(q),
+                                             _ptr(k), _ptr(v),
                                              _ptr(o), _ptr(lse), _ptr(block_idx_out), _ptr(token_idx_out),
                                              _ptr(dev_status), _ptr(workspace), workspace.numel(), _stream(stream)))
 
 
 def hisa_forward_cached(p, q_idx, k_idx, block_keys, refresh_begin, q, k, v, o, lse=None, block_idx_out=None,
-                        token_idx_out=None, dev_status=None, workspace=None, stream=None):
+                        token_idx_out=None, dev_status=None, workspace=None, stream=None, idx_weights=None):
     if workspace is None:
         workspace = _workspace(hisa_forward_workspace_size(p), q_idx.device)
     _check("hisa_forward_cached",
-           _lib.hisa_forward_cached(ctypes.byref(p), _ptr(q_idx), _ptr(k_idx), _ptr(block_keys), int(refresh_begin),
+           _lib.hisa_forward_cached(ctypes.byref(p), _ptr(q_idx), _ptr(idx_weights), _ptr(k_idx), _ptr(block_keys),
+                                    int(refresh_begin),
                                     _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(block_idx_out),
                                     _ptr(token_idx_out), _ptr(dev_status), _ptr(workspace), workspace.numel(),
                                     _stream(stream)))
@@ -215,20 +220,22 @@ def hisa_flat_topk_workspace_size(p):
     return _size(_lib.hisa_flat_topk_workspace_size, p, two=True)
 
 
-def hisa_flat_topk(p, q_idx, k_idx, token_idx, token_scores=None, workspace=None, stream=None):
+def hisa_flat_topk(p, q_idx, k_idx, token_idx, token_scores=None, workspace=None, stream=None, idx_weights=None):
     if workspace is None:
         workspace = _workspace(hisa_flat_topk_workspace_size(p)[1], q_idx.device)
-    _check("hisa_flat_topk", _lib.hisa_flat_topk(ctypes.byref(p), _ptr(q_idx), _ptr(k_idx), _ptr(token_idx),
+    _check("hisa_flat_topk", _lib.hisa_flat_topk(ctypes.byref(p), _ptr(q_idx), _ptr(idx_weights), _ptr(k_idx),
+                                                 _ptr(token_idx),
                                                  _ptr(token_scores), _ptr(workspace), workspace.numel(),
                                                  _stream(stream)))
 
 
 def hisa_token_topk_noalloc(p, q_idx, k_idx, block_idx, token_idx, token_scores=None, dev_status=None,
-                            stream=None):
+                            stream=None, idx_weights=None):
     """hisa_token_topk for callers that cannot allocate: the library's fixed device scratch
     array stands in for the workspace (see include/hisa.h)."""
     _check("hisa_token_topk_noalloc",
-           _lib.hisa_token_topk_noalloc(ctypes.byref(p), _ptr(q_idx), _ptr(k_idx), _ptr(block_idx), _ptr(token_idx),
+           _lib.hisa_token_topk_noalloc(ctypes.byref(p), _ptr(q_idx), _ptr(idx_weights), _ptr(k_idx), _ptr(block_idx),
+                                        _ptr(token_idx),
                                         _ptr(token_scores), _ptr(dev_status), _stream(stream)))
 
 
@@ -237,12 +244,13 @@ def hisa_block_candidates_workspace_size(p) -> int:
 
 
 def hisa_block_candidates(p_local, n_kv_global, first_block, q_idx, block_keys, cand_scores, cand_ids,
-                          workspace=None, stream=None):
+                          workspace=None, stream=None, idx_weights=None):
     """This rank's step-3 candidates (see include/hisa.h): [batch][top_m] scores and global block ids."""
     if workspace is None:
         workspace = _workspace(hisa_block_candidates_workspace_size(p_local), q_idx.device)
     _check("hisa_block_candidates",
-           _lib.hisa_block_candidates(ctypes.byref(p_local), n_kv_global, first_block, _ptr(q_idx), _ptr(block_keys),
+           _lib.hisa_block_candidates(ctypes.byref(p_local), n_kv_global, first_block, _ptr(q_idx), _ptr(idx_weights),
+                                      _ptr(block_keys),
                                       _ptr(cand_scores), _ptr(cand_ids), _ptr(workspace), workspace.numel(),
                                       _stream(stream)))
 
@@ -284,8 +292,9 @@ def hisa_version() -> str:
 
 # ---------------------------------------------------------------- convenience front end
 
-def forward(p, q_idx, k_idx, q, k, v, return_indices=False, stream=None):
-    """Allocate the outputs with torch and run hisa_forward; returns (o, lse[, block_idx, token_idx])."""
+def forward(p, q_idx, k_idx, q, k, v, return_indices=False, stream=None, idx_weights=None):
+    """Allocate the outputs with torch and run hisa_forward; returns (o, lse[, block_idx, token_idx]).
+    idx_weights: the indexer's head weights [b][n_q][n_idx_heads] when p.n_idx_heads > 0."""
     import torch
 
     dev = q_idx.device
@@ -295,7 +304,7 @@ def forward(p, q_idx, k_idx, q, k, v, return_indices=False, stream=None):
     if return_indices:
         blk = torch.empty((p.batch, p.n_q, p.top_m), dtype=torch.int32, device=dev)
         tok = torch.empty((p.batch, p.n_q, p.top_k), dtype=torch.int32, device=dev)
-    hisa_forward(p, q_idx, k_idx, q, k, v, o, lse, blk, tok, stream=stream)
+    hisa_forward(p, q_idx, k_idx, q, k, v, o, lse, blk, tok, stream=stream, idx_weights=idx_weights)
     return (o, lse, blk, tok) if return_indices else (o, lse)
 
 

@@ -72,14 +72,14 @@ class Phases:
     def __init__(self, stream=None):
         self.stream = stream
 
-    def blocks(self, pl, shard: Shard, q_idx, block_keys):
+    def blocks(self, pl, shard: Shard, q_idx, block_keys, idx_weights=None):
         import torch
 
         b, m = pl.batch, pl.top_m
         scores = torch.empty((b, m), dtype=torch.float32, device=q_idx.device)
         ids = torch.empty((b, m), dtype=torch.int32, device=q_idx.device)
         hisa_block_candidates(pl, shard.n_kv_global, shard.first_block, q_idx, block_keys, scores, ids,
-                              stream=self.stream)
+                              stream=self.stream, idx_weights=idx_weights)
         return scores, ids
 
     def merge(self, scores_all, ids_all, k):
@@ -91,7 +91,7 @@ class Phases:
         hisa_topk_merge(scores_all, ids_all, k, out_ids, out_scores, stream=self.stream)
         return out_ids, out_scores
 
-    def tokens(self, pl, shard: Shard, q_idx, k_idx, block_idx, status=None):
+    def tokens(self, pl, shard: Shard, q_idx, k_idx, block_idx, status=None, idx_weights=None):
         import torch
 
         b = pl.batch
@@ -101,7 +101,7 @@ class Phases:
                        out=local_blk, stream=self.stream)
         tok = torch.empty((b, 1, pl.top_k), dtype=torch.int32, device=dev)
         scores = torch.empty((b, 1, pl.top_k), dtype=torch.float32, device=dev)
-        hisa_token_topk(pl, q_idx, k_idx, local_blk, tok, scores, status, stream=self.stream)
+        hisa_token_topk(pl, q_idx, k_idx, local_blk, tok, scores, status, stream=self.stream, idx_weights=idx_weights)
         hisa_remap_ids(tok, 0, shard.n_loc, shard.t0, stream=self.stream)  # local -> global ids, in place
         return scores.view(b, pl.top_k), tok.view(b, pl.top_k)
 
@@ -126,20 +126,22 @@ class Phases:
         return o, lse
 
 
-def decode_step(p, shard: Shard, q_idx, k_idx, block_keys, q, k, v, exchange, phases=None, status=None):
+def decode_step(p, shard: Shard, q_idx, k_idx, block_keys, q, k, v, exchange, phases=None, status=None,
+                idx_weights=None):
     """One decode step of the whole context, run by every rank on its slice.
 
     p: the global problem (n_kv = the whole context, n_q = 1).  q_idx, q: the
     new token's indexer query and attention queries (the same on every rank);
     k_idx, k, v, block_keys: this rank's slice of the caches and its pooled
     block keys.  Returns (block_idx [b][m], token_idx [b][k], o, lse) of the
-    whole context, the same on every rank.
+    whole context, the same on every rank.  idx_weights: the indexer's head weights with a
+    multi-head indexer (p.n_idx_heads > 0), the same on every rank.
     """
     ph = phases if phases is not None else Phases()
     pl = local_params(p, shard)
-    cs, ci = ph.blocks(pl, shard, q_idx, block_keys)
+    cs, ci = ph.blocks(pl, shard, q_idx, block_keys, idx_weights)
     blk, _ = ph.merge(exchange(cs), exchange(ci), p.top_m)
-    ts, ti = ph.tokens(pl, shard, q_idx, k_idx, blk, status)
+    ts, ti = ph.tokens(pl, shard, q_idx, k_idx, blk, status, idx_weights)
     tok, _ = ph.merge(exchange(ts), exchange(ti), p.top_k)
     o_part, lse_part = ph.attention(pl, shard, q, k, v, tok, status)
     o, lse = ph.lse_merge(exchange(o_part), exchange(lse_part))

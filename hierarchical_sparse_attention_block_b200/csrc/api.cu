@@ -27,6 +27,8 @@ bool pow2(int64_t x) { return x > 0 && (x & (x - 1)) == 0; }
 constexpr size_t kAlign = 256;
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
+}  // namespace
+
 // Validation shared by every call.  need_attn: the attention fields matter.
 hisa_status_t make_shape(const hisa_params_t* p, bool need_indexer, bool need_attn, Shape* s) {
   if (!p) return HISA_ERR_INVALID_ARG;
@@ -52,6 +54,9 @@ hisa_status_t make_shape(const hisa_params_t* p, bool need_indexer, bool need_at
     if (p->d_idx != 64 && p->d_idx != 128 && p->d_idx != 256) return p->d_idx < 1 ? HISA_ERR_INVALID_ARG : HISA_ERR_UNSUPPORTED;
     s->n_blk = (p->n_kv + p->block - 1) / p->block;
     if ((int64_t)p->top_m * p->block > (int64_t)1 << 24) return HISA_ERR_UNSUPPORTED;
+    if (p->n_idx_heads < 0) return HISA_ERR_INVALID_ARG;
+    if (p->n_idx_heads > 16) return HISA_ERR_UNSUPPORTED;
+    s->HI = p->n_idx_heads;
   } else {
     s->n_blk = p->block >= 1 ? (p->n_kv + p->block - 1) / p->block : 0;
   }
@@ -65,6 +70,15 @@ hisa_status_t make_shape(const hisa_params_t* p, bool need_indexer, bool need_at
   }
   return HISA_OK;
 }
+
+hisa_status_t set_idx_weights(Shape* s, const float* idx_weights) {
+  if ((s->HI == 0) != (idx_weights == nullptr)) return HISA_ERR_INVALID_ARG;
+  if (idx_weights && ((uintptr_t)idx_weights & 3u) != 0) return HISA_ERR_INVALID_ARG;
+  s->w_idx = idx_weights;
+  return HISA_OK;
+}
+
+namespace {
 
 size_t topm_ws(const Shape& s) {
   size_t b = align_up((size_t)s.n_query * s.n_blk * sizeof(float));
@@ -182,11 +196,12 @@ hisa_status_t hisa_block_topm_workspace_size(const hisa_params_t* params, size_t
   return HISA_OK;
 }
 
-hisa_status_t hisa_block_topm(const hisa_params_t* params, const void* q_idx, const float* block_keys,
-                              int32_t* block_idx, float* block_scores, int32_t* dev_status, void* workspace,
-                              size_t workspace_bytes, cudaStream_t stream) {
+hisa_status_t hisa_block_topm(const hisa_params_t* params, const void* q_idx, const float* idx_weights,
+                              const float* block_keys, int32_t* block_idx, float* block_scores, int32_t* dev_status,
+                              void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   Shape s;
   hisa_status_t rc = hisa::make_shape(params, true, false, &s);
+  if (rc == HISA_OK) rc = hisa::set_idx_weights(&s, idx_weights);
   if (rc != HISA_OK) return rc;
   if (!q_idx || !block_keys || !block_idx) return HISA_ERR_INVALID_ARG;
   if (!hisa::aligned16(q_idx) || !hisa::aligned16(block_keys) || !hisa::aligned16(block_idx)) return HISA_ERR_INVALID_ARG;
@@ -205,11 +220,12 @@ hisa_status_t hisa_token_topk_workspace_size(const hisa_params_t* params, size_t
   return HISA_OK;
 }
 
-hisa_status_t hisa_token_topk(const hisa_params_t* params, const void* q_idx, const void* k_idx,
-                              const int32_t* block_idx, int32_t* token_idx, float* token_scores, int32_t* dev_status,
-                              void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+hisa_status_t hisa_token_topk(const hisa_params_t* params, const void* q_idx, const float* idx_weights,
+                              const void* k_idx, const int32_t* block_idx, int32_t* token_idx, float* token_scores,
+                              int32_t* dev_status, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   Shape s;
   hisa_status_t rc = hisa::make_shape(params, true, false, &s);
+  if (rc == HISA_OK) rc = hisa::set_idx_weights(&s, idx_weights);
   if (rc != HISA_OK) return rc;
   if (!q_idx || !k_idx || !block_idx || !token_idx) return HISA_ERR_INVALID_ARG;
   if (!hisa::aligned16(q_idx) || !hisa::aligned16(k_idx) || !hisa::aligned16(block_idx) || !hisa::aligned16(token_idx))
@@ -311,12 +327,13 @@ hisa_status_t check_forward_args(const void* q_idx, const void* k_idx, const voi
 }
 }  // namespace
 
-hisa_status_t hisa_forward(const hisa_params_t* params, const void* q_idx, const void* k_idx, const void* q,
-                           const void* k, const void* v, void* o, float* lse, int32_t* block_idx_out,
-                           int32_t* token_idx_out, int32_t* dev_status, void* workspace, size_t workspace_bytes,
-                           cudaStream_t stream) {
+hisa_status_t hisa_forward(const hisa_params_t* params, const void* q_idx, const float* idx_weights,
+                           const void* k_idx, const void* q, const void* k, const void* v, void* o, float* lse,
+                           int32_t* block_idx_out, int32_t* token_idx_out, int32_t* dev_status, void* workspace,
+                           size_t workspace_bytes, cudaStream_t stream) {
   Shape s;
   hisa_status_t rc = hisa::make_shape(params, true, true, &s);
+  if (rc == HISA_OK) rc = hisa::set_idx_weights(&s, idx_weights);
   if (rc != HISA_OK) return rc;
   rc = check_forward_args(q_idx, k_idx, q, k, v, o, lse, block_idx_out, token_idx_out);
   if (rc != HISA_OK) return rc;
@@ -327,12 +344,14 @@ hisa_status_t hisa_forward(const hisa_params_t* params, const void* q_idx, const
                       token_idx_out, dev_status, ws, workspace_bytes, stream);
 }
 
-hisa_status_t hisa_forward_cached(const hisa_params_t* params, const void* q_idx, const void* k_idx,
-                                  float* block_keys, int64_t refresh_begin, const void* q, const void* k,
-                                  const void* v, void* o, float* lse, int32_t* block_idx_out, int32_t* token_idx_out,
-                                  int32_t* dev_status, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+hisa_status_t hisa_forward_cached(const hisa_params_t* params, const void* q_idx, const float* idx_weights,
+                                  const void* k_idx, float* block_keys, int64_t refresh_begin, const void* q,
+                                  const void* k, const void* v, void* o, float* lse, int32_t* block_idx_out,
+                                  int32_t* token_idx_out, int32_t* dev_status, void* workspace,
+                                  size_t workspace_bytes, cudaStream_t stream) {
   Shape s;
   hisa_status_t rc = hisa::make_shape(params, true, true, &s);
+  if (rc == HISA_OK) rc = hisa::set_idx_weights(&s, idx_weights);
   if (rc != HISA_OK) return rc;
   rc = check_forward_args(q_idx, k_idx, q, k, v, o, lse, block_idx_out, token_idx_out);
   if (rc != HISA_OK) return rc;
@@ -355,10 +374,12 @@ hisa_status_t hisa_flat_topk_workspace_size(const hisa_params_t* params, size_t*
   return HISA_OK;
 }
 
-hisa_status_t hisa_flat_topk(const hisa_params_t* params, const void* q_idx, const void* k_idx, int32_t* token_idx,
-                             float* token_scores, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+hisa_status_t hisa_flat_topk(const hisa_params_t* params, const void* q_idx, const float* idx_weights,
+                             const void* k_idx, int32_t* token_idx, float* token_scores, void* workspace,
+                             size_t workspace_bytes, cudaStream_t stream) {
   Shape s;
   hisa_status_t rc = hisa::make_shape(params, true, false, &s);
+  if (rc == HISA_OK) rc = hisa::set_idx_weights(&s, idx_weights);
   if (rc != HISA_OK) return rc;
   if (!q_idx || !k_idx || !token_idx) return HISA_ERR_INVALID_ARG;
   if (!hisa::aligned16(q_idx) || !hisa::aligned16(k_idx) || !hisa::aligned16(token_idx)) return HISA_ERR_INVALID_ARG;
@@ -379,10 +400,12 @@ hisa_status_t hisa_block_candidates_workspace_size(const hisa_params_t* local, s
 }
 
 hisa_status_t hisa_block_candidates(const hisa_params_t* local, int64_t n_kv_global, int64_t first_block,
-                                    const void* q_idx, const float* block_keys, float* cand_scores, int32_t* cand_ids,
-                                    void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+                                    const void* q_idx, const float* idx_weights, const float* block_keys,
+                                    float* cand_scores, int32_t* cand_ids, void* workspace, size_t workspace_bytes,
+                                    cudaStream_t stream) {
   Shape s;
   hisa_status_t rc = hisa::make_shape(local, true, false, &s);
+  if (rc == HISA_OK) rc = hisa::set_idx_weights(&s, idx_weights);
   if (rc != HISA_OK) return rc;
   if (s.n_q != 1) return HISA_ERR_UNSUPPORTED;  // decode: the query is the newest token of the whole context
   if (first_block < 0 || n_kv_global < 1 || first_block * s.B + s.n_kv > n_kv_global) return HISA_ERR_INVALID_ARG;

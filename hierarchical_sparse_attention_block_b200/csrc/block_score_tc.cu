@@ -259,7 +259,7 @@ cudaError_t launch_tc(const Shape& s, const void* q_idx, const float* bk, float*
 }  // namespace
 
 bool block_score_tc_eligible(const Shape& s) {
-  return (s.d_idx == 64 || s.d_idx == 128) && s.n_q >= 64 && s.n_query <= 0x7FFFFFFFLL &&
+  return s.HI == 0 && (s.d_idx == 64 || s.d_idx == 128) && s.n_q >= 64 && s.n_query <= 0x7FFFFFFFLL &&
          (int64_t)s.batch * s.n_blk <= 0x7FFFFFFFLL;
 }
 

@@ -4,7 +4,8 @@
 // "塊級粗過濾" and the forced first/last block remark of "塊內精挑字符".
 //
 // block_score_kernel is the CUDA-core scorer (decode: one query per sequence
-// makes this a GEMV streaming n_blk * d_idx * 4 B of block keys from HBM).
+// makes this a GEMV streaming n_blk * d_idx * 4 B of block keys from HBM);
+// block_score_mh_kernel scores with the multi-head weighted form.
 // block_topm_kernel runs one CTA per query: the scores of blocks 1..c-1 become
 // order-preserving keys in shared memory and a CTA radix selection keeps the
 // best m-2 of them (ties to the lower block id).
@@ -55,6 +56,52 @@ __global__ void __launch_bounds__(256) block_score_kernel(const uint16_t* __rest
     }
     dot = warp_sum(dot);
     if (lane == 0) scores[qg * n_blk + j] = dot;
+  }
+}
+
+// The multi-head indexer score sum_j w_j * max(0, q_j . bk) (n_idx_heads = HI >= 1): the query's
+// HI heads go to shared memory as fp32, a warp takes one block key at a time (lane = D/32
+// dimensions), and the per-head dot products are summed over the warp one head after another.
+template <int D>
+__global__ void __launch_bounds__(256) block_score_mh_kernel(const uint16_t* __restrict__ q_idx,
+                                                             const float* __restrict__ w_idx,
+                                                             const float* __restrict__ bk, float* __restrict__ scores,
+                                                             int64_t n_q, int64_t n_kv, int B, int64_t n_blk,
+                                                             int chunks, int HI) {
+  constexpr int PER = D / 32;
+  extern __shared__ float sq[];  // [HI][D] query heads, then [HI] weights
+  const int64_t qg = blockIdx.x / chunks;
+  const int chunk = blockIdx.x % chunks;
+  const int seq = (int)(qg / n_q);
+  const int64_t p = n_kv - n_q + qg % n_q;
+  const int64_t c = p / B;
+  const int64_t j0 = (int64_t)chunk * kScoreBlocksPerCta;
+  if (j0 > c) return;
+  const int64_t j1 = min(j0 + kScoreBlocksPerCta, c + 1);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint16_t* qrow = q_idx + qg * HI * D;
+  for (int i = threadIdx.x; i < HI * D; i += 256) sq[i] = __uint_as_float((uint32_t)qrow[i] << 16);
+  for (int i = threadIdx.x; i < HI; i += 256) sq[HI * D + i] = w_idx[qg * HI + i];
+  __syncthreads();
+  const float* bks = bk + (int64_t)seq * n_blk * D + lane * PER;
+  for (int64_t j = j0 + warp; j < j1; j += 8) {
+    float b[PER];
+#pragma unroll
+    for (int e = 0; e < PER; e += 2) {
+      const float2 b2 = *reinterpret_cast<const float2*>(bks + j * D + e);
+      b[e] = b2.x;
+      b[e + 1] = b2.y;
+    }
+    float score = 0.f;
+    for (int h = 0; h < HI; ++h) {
+      const float* qh = sq + h * D + lane * PER;
+      float dot = 0.f;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) dot = fmaf(qh[e], b[e], dot);
+      dot = warp_sum(dot);
+      score = fmaf(sq[HI * D + h], fmaxf(dot, 0.f), score);
+    }
+    if (lane == 0) scores[qg * n_blk + j] = score;
   }
 }
 
@@ -114,6 +161,25 @@ cudaError_t launch_block_score(const Shape& s, const void* q_idx, const float* b
   const int64_t grid = s.n_query * chunks;
   if (grid > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
   const uint16_t* qp = static_cast<const uint16_t*>(q_idx);
+  if (s.HI > 0) {
+    const int smem = (s.HI * s.d_idx + s.HI) * (int)sizeof(float);
+    switch (s.d_idx) {
+      case 64:
+        block_score_mh_kernel<64><<<(unsigned)grid, 256, smem, st>>>(qp, s.w_idx, block_keys, scores, s.n_q, s.n_kv,
+                                                                     s.B, s.n_blk, chunks, s.HI);
+        break;
+      case 128:
+        block_score_mh_kernel<128><<<(unsigned)grid, 256, smem, st>>>(qp, s.w_idx, block_keys, scores, s.n_q, s.n_kv,
+                                                                      s.B, s.n_blk, chunks, s.HI);
+        break;
+      case 256:
+        block_score_mh_kernel<256><<<(unsigned)grid, 256, smem, st>>>(qp, s.w_idx, block_keys, scores, s.n_q, s.n_kv,
+                                                                      s.B, s.n_blk, chunks, s.HI);
+        break;
+      default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+  }
   switch (s.d_idx) {
     case 64:
       block_score_kernel<64><<<(unsigned)grid, 256, 0, st>>>(qp, block_keys, scores, s.n_q, s.n_kv, s.B, s.n_blk, chunks);

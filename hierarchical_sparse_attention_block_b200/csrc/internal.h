@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "hisa.h"
+
 namespace hisa {
 
 // Validated problem shape (see hisa_params_t in hisa.h).
@@ -14,7 +16,14 @@ struct Shape {
   float scale;      // softmax scale, already resolved
   int64_t n_blk;    // ceil(n_kv / B)
   int64_t n_query;  // batch * n_q
+  int HI = 0;                    // indexer heads: 0 = one head scored by a dot product
+  const float* w_idx = nullptr;  // [n_query][HI] head weights when HI >= 1
 };
+
+// Shape of a request (the validation every call shares; see hisa.h).  need_attn: the attention
+// fields matter.  with_weights then checks idx_weights against n_idx_heads and keeps it.
+hisa_status_t make_shape(const hisa_params_t* p, bool need_indexer, bool need_attn, Shape* s);
+hisa_status_t set_idx_weights(Shape* s, const float* idx_weights);
 
 // Step 1: block means for blocks [b0, b1) of every sequence.
 cudaError_t launch_block_pool(const Shape& s, const void* k_idx, int64_t b0, int64_t b1, float* block_keys,

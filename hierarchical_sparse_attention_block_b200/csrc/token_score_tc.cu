@@ -268,7 +268,7 @@ cudaError_t launch_ts(const Shape& s, const void* q_idx, const void* k_idx, cons
 }  // namespace
 
 bool token_score_tc_eligible(const Shape& s, int slots) {
-  return (s.d_idx == 64 || s.d_idx == 128) && (s.B == 32 || s.B == 64 || s.B == 128 || s.B == 256) &&
+  return s.HI == 0 && (s.d_idx == 64 || s.d_idx == 128) && (s.B == 32 || s.B == 64 || s.B == 128 || s.B == 256) &&
          s.n_q >= kTileQ && slots < 32767 && s.n_query <= 0x7FFFFFFFLL &&
          (int64_t)s.batch * s.n_kv <= 0x7FFFFFFFLL;
 }

@@ -10,6 +10,8 @@
 // an order-preserving u32 key at [slot * B + offset] of the query's row;
 // positions past the query or in unused slots get key 0 ("empty").
 //
+// token_score_mh_kernel: the same for the multi-head weighted score.
+//
 // token_select_kernel: one CTA per query; the row of keys is staged in shared
 // memory (when it fits) and a CTA radix selection takes the best
 // min(k, candidates), emitted in ascending token order.
@@ -128,6 +130,97 @@ __global__ void __launch_bounds__(kScoreThreads)
   }
 }
 
+// The multi-head indexer score sum_j w_j * max(0, q_j . k_t) (n_idx_heads = HI >= 1).  Same
+// work split and slot rules as token_score_kernel; the query's HI heads sit in shared memory as
+// fp32 and every token row, read once, is scored against each head in turn.
+template <int D>
+__global__ void __launch_bounds__(kScoreThreads)
+    token_score_mh_kernel(const uint16_t* __restrict__ q_idx, const float* __restrict__ w_idx,
+                          const uint16_t* __restrict__ k_idx, const int32_t* __restrict__ block_idx, int slots,
+                          uint32_t* __restrict__ keys, int32_t* __restrict__ status, int64_t n_q, int64_t n_kv, int B,
+                          int spc, int chunks, int64_t q0, int HI) {
+  constexpr int CPL = D / 64;  // 16-byte chunks per lane
+  __shared__ int s_blk[kMaxSlotsPerCta];
+  __shared__ int s_len[kMaxSlotsPerCta];
+  extern __shared__ float sq[];  // [HI][D] query heads, then [HI] weights
+
+  const int64_t lq = blockIdx.x / chunks;
+  const int chunk = blockIdx.x % chunks;
+  const int64_t qg = q0 + lq;
+  const int seq = (int)(qg / n_q);
+  const int64_t p = n_kv - n_q + qg % n_q;
+  const int64_t c = p / B;
+  const int r0 = chunk * spc;
+  const int nr = min(spc, slots - r0);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+
+  for (int rr = warp; rr < nr; rr += kScoreThreads / 32) {
+    const int r = r0 + rr;
+    int blk;
+    bool ok;
+    if (block_idx) {
+      const int32_t* row = block_idx + qg * slots;
+      blk = row[r];
+      int mx = -1;
+      for (int t = lane; t < r; t += 32) {
+        const int v = row[t];
+        if (v >= 0 && v <= c) mx = max(mx, v);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+      ok = blk >= 0 && blk <= c && blk > mx;
+      if (!ok && blk != -1 && lane == 0 && status) atomicOr(status, kStatusBadIndex);
+    } else {
+      blk = r;
+      ok = r <= c;
+    }
+    if (lane == 0) {
+      s_blk[rr] = ok ? blk : -1;
+      s_len[rr] = ok ? visible_len(blk, B, p) : 0;
+    }
+  }
+  const uint16_t* qrow = q_idx + qg * HI * D;
+  for (int i = threadIdx.x; i < HI * D; i += kScoreThreads) sq[i] = __uint_as_float((uint32_t)qrow[i] << 16);
+  for (int i = threadIdx.x; i < HI; i += kScoreThreads) sq[HI * D + i] = w_idx[qg * HI + i];
+  __syncthreads();
+
+  const int grp = threadIdx.x >> 3, sub = threadIdx.x & 7;
+  const unsigned gmask = 0xFFu << (lane & ~7);
+  constexpr int NG = kScoreThreads / 8;  // token rows per CTA step
+  uint32_t* krow = keys + lq * (int64_t)slots * B;
+  for (int rr = 0; rr < nr; ++rr) {
+    const int blk = s_blk[rr], len = s_len[rr];
+    const uint16_t* kb = k_idx + ((int64_t)seq * n_kv + (int64_t)(blk < 0 ? 0 : blk) * B) * D + sub * 8;
+    uint32_t* dst = krow + (int64_t)(r0 + rr) * B;
+    for (int o = grp; o < B; o += NG) {  // warp-uniform trip count: rows o of a lane group
+      float kv[8 * CPL];
+#pragma unroll
+      for (int u = 0; u < CPL; ++u) {
+        const uint4 w = o < len ? ld_nc_v4(kb + (int64_t)o * D + u * 64) : make_uint4(0, 0, 0, 0);
+        kv[8 * u + 0] = bf16_lo(w.x); kv[8 * u + 1] = bf16_hi(w.x);
+        kv[8 * u + 2] = bf16_lo(w.y); kv[8 * u + 3] = bf16_hi(w.y);
+        kv[8 * u + 4] = bf16_lo(w.z); kv[8 * u + 5] = bf16_hi(w.z);
+        kv[8 * u + 6] = bf16_lo(w.w); kv[8 * u + 7] = bf16_hi(w.w);
+      }
+      float score = 0.f;
+      for (int h = 0; h < HI; ++h) {
+        float dot = 0.f;
+#pragma unroll
+        for (int u = 0; u < CPL; ++u) {
+          const float* qq = sq + h * D + (sub + 8 * u) * 8;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) dot = fmaf(qq[e], kv[8 * u + e], dot);
+        }
+        dot += __shfl_xor_sync(gmask, dot, 4);
+        dot += __shfl_xor_sync(gmask, dot, 2);
+        dot += __shfl_xor_sync(gmask, dot, 1);
+        score = fmaf(sq[HI * D + h], fmaxf(dot, 0.f), score);
+      }
+      if (sub == 0) dst[o] = o < len ? score_key(score) : 0u;
+    }
+  }
+}
+
 template <int NT>
 __global__ void __launch_bounds__(NT)
     token_select_kernel(const uint32_t* __restrict__ keys, const int32_t* __restrict__ block_idx, int slots,
@@ -191,6 +284,25 @@ cudaError_t launch_token_score(const Shape& s, const void* q_idx, const void* k_
   if (grid > 0x7FFFFFFFLL) return cudaErrorInvalidConfiguration;
   const uint16_t* qp = static_cast<const uint16_t*>(q_idx);
   const uint16_t* kp = static_cast<const uint16_t*>(k_idx);
+  if (s.HI > 0) {
+    const int smem = (s.HI * s.d_idx + s.HI) * (int)sizeof(float);
+    switch (s.d_idx) {
+      case 64:
+        token_score_mh_kernel<64><<<(unsigned)grid, kScoreThreads, smem, st>>>(
+            qp, s.w_idx, kp, block_idx, slots, keys, status, s.n_q, s.n_kv, s.B, spc, chunks, q0, s.HI);
+        break;
+      case 128:
+        token_score_mh_kernel<128><<<(unsigned)grid, kScoreThreads, smem, st>>>(
+            qp, s.w_idx, kp, block_idx, slots, keys, status, s.n_q, s.n_kv, s.B, spc, chunks, q0, s.HI);
+        break;
+      case 256:
+        token_score_mh_kernel<256><<<(unsigned)grid, kScoreThreads, smem, st>>>(
+            qp, s.w_idx, kp, block_idx, slots, keys, status, s.n_q, s.n_kv, s.B, spc, chunks, q0, s.HI);
+        break;
+      default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+  }
   switch (s.d_idx) {
     case 64:
       token_score_kernel<64><<<(unsigned)grid, kScoreThreads, 0, st>>>(qp, kp, block_idx, slots, keys, status, s.n_q,

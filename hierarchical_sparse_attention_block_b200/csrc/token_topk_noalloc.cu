@@ -57,13 +57,18 @@ cudaError_t scratch_address(void** out) {
 }  // namespace
 }  // namespace hisa
 
-extern "C" hisa_status_t hisa_token_topk_noalloc(const hisa_params_t* params, const void* q_idx, const void* k_idx,
+extern "C" hisa_status_t hisa_token_topk_noalloc(const hisa_params_t* params, const void* q_idx,
+                                                 const float* idx_weights, const void* k_idx,
                                                  const int32_t* block_idx, int32_t* token_idx, float* token_scores,
                                                  int32_t* dev_status, cudaStream_t stream) {
   using namespace hisa;
   // Same argument rules as hisa_token_topk.
   size_t one_query = 0, preferred = 0;
   hisa_status_t rc = hisa_token_topk_workspace_size(params, &one_query, &preferred);
+  if (rc != HISA_OK) return rc;
+  Shape s;
+  rc = make_shape(params, true, false, &s);
+  if (rc == HISA_OK) rc = set_idx_weights(&s, idx_weights);
   if (rc != HISA_OK) return rc;
   if (one_query > kNoAllocScratchBytes) return HISA_ERR_UNSUPPORTED;
   if (!q_idx || !k_idx || !block_idx || !token_idx) return HISA_ERR_INVALID_ARG;
@@ -79,20 +84,6 @@ extern "C" hisa_status_t hisa_token_topk_noalloc(const hisa_params_t* params, co
     return HISA_ERR_CUDA;
   }
   // Queries in chunks that fit the array.
-  Shape s;
-  s.batch = params->batch;
-  s.n_q = params->n_q;
-  s.n_kv = params->n_kv;
-  s.d_idx = params->d_idx;
-  s.B = params->block;
-  s.m = params->top_m;
-  s.k = params->top_k;
-  s.H = params->n_heads;
-  s.Hkv = params->n_kv_heads;
-  s.d = params->d_head;
-  s.scale = 0.f;
-  s.n_blk = (params->n_kv + params->block - 1) / params->block;
-  s.n_query = (int64_t)params->batch * params->n_q;
   const int64_t chunk = (int64_t)(kNoAllocScratchBytes / one_query);
   uint32_t* keys = static_cast<uint32_t*>(scratch);
   for (int64_t q0 = 0; q0 < s.n_query; q0 += chunk) {

@@ -13,7 +13,8 @@
  *
  *   1. cut each sequence's indexer keys into blocks of B tokens and mean-pool
  *      every block into one block key;
- *   2. score each query against the block keys it can see (dot product);
+ *   2. score each query against the block keys it can see with the
+ *      indexer's score (below);
  *   3. keep m blocks: block 0, the query's own block c = floor(p/B), and the
  *      m-2 best of blocks 1..c-1 (all visible blocks when c+1 <= m);
  *   4. score the query against the tokens t <= p of those blocks;
@@ -28,12 +29,25 @@
  *     pointers must be 16-byte aligned.
  *   - Shapes (b = batch, H = n_heads, Hk = n_kv_heads, d = d_head):
  *       q_idx  [b][n_q][d_idx]  bf16     k_idx   [b][n_kv][d_idx] bf16
+ *         ([b][n_q][Hi][d_idx] with an Hi-head indexer, idx_weights
+ *          [b][n_q][Hi] fp32)
  *       block_keys [b][ceil(n_kv/B)][d_idx] fp32
  *       block_idx  [b][n_q][m]  int32    token_idx [b][n_q][k] int32
  *       q [b][n_q][H][d] bf16   k, v [b][n_kv][Hk][d] bf16
  *       o [b][n_q][H][d] bf16   lse [b][n_q][H] fp32 (natural log)
  *     Query i of a sequence sits at position p_i = n_kv - n_q + i
  *     (prefill: n_q = n_kv; decode: n_q = 1, p = n_kv - 1).
+ *   - The indexer's score of a key kv (a block key in step 2, a token's
+ *     k_idx row in step 4) is the original indexer's own score function
+ *     ([IP] 1.2.1 item 2, 1.3 item 4 "Score Function Consistency"):
+ *       n_idx_heads = 0:   q . kv                         (one head);
+ *       n_idx_heads = Hi:  sum_j w_j * max(0, q_j . kv)   (Hi heads q_j with
+ *                          the query's head weights w_j = idx_weights, the
+ *                          multi-head indexer form of DeepSeek-V3.2).
+ *     idx_weights must be NULL when n_idx_heads is 0 and non-NULL otherwise.
+ *     The tensor-core scorers serve the one-head form; the Hi-head form runs
+ *     on CUDA-core scorers.  Integer inputs and integer weights keep it exact
+ *     while |scores| * B < 2^24.
  *   - Index lists are ascending with -1 padding at the tail.  Ties in a
  *     selection go to the lower block / token index.
  *   - Every call validates its arguments on the host before launching
@@ -47,7 +61,8 @@
  *     dereferenced, and bit 0 of *dev_status is set (atomicOr).  No kernel
  *     traps or waits unboundedly: a wait that runs out (1 s) sets bit 1 of
  *     *dev_status and the results of that call are not valid.
- *   - Supported sizes: d_idx in {64, 128, 256}; d_head in {64, 128}; B a
+ *   - Supported sizes: d_idx in {64, 128, 256}; n_idx_heads in [0, 16];
+ *     d_head in {64, 128}; B a
  *     power of two in [1, 4096]; m >= 2; k >= 1; n_heads a multiple of
  *     n_kv_heads; n_kv < 2^31.  Integer-valued indexer inputs (|x| <= 4)
  *     make every block mean and score exact in fp32, so selections are exact.
@@ -72,7 +87,9 @@ typedef enum hisa_status {
   HISA_ERR_CUDA = 4         /* a CUDA call failed; see hisa_last_cuda_error() */
 } hisa_status_t;
 
-/* Problem description.  scale <= 0 selects 1/sqrt(d_head).  flags must be 0. */
+/* Problem description.  scale <= 0 selects 1/sqrt(d_head).  flags must be 0.
+ * n_idx_heads: 0 for a one-head dot-product indexer, Hi in [1, 16] for the
+ * Hi-head weighted form (see the conventions above). */
 typedef struct hisa_params {
   int32_t batch;      /* b: independent sequences of equal length */
   int32_t d_idx;      /* indexer head dimension */
@@ -86,6 +103,7 @@ typedef struct hisa_params {
   int32_t d_head;     /* d: attention head dimension */
   float scale;        /* softmax scale tau */
   int32_t flags;      /* reserved, 0 */
+  int32_t n_idx_heads; /* Hi: indexer query heads (0: one head, plain dot product) */
 } hisa_params_t;
 
 /* Step 1 -- [IP] 1.2.1 item 1; [QB] "塊級粗過濾" bullet 1.
@@ -100,16 +118,16 @@ hisa_status_t hisa_block_pool(const hisa_params_t* params, const void* k_idx, in
 /* Steps 2-3 -- [IP] 1.2.1 items 2-3; [QB] "塊級粗過濾" bullets 2-3 and the
  * forced first/last block remark of "塊內精挑字符".
  * block_idx[s][i][0..m): the min(m, c+1) kept blocks, ascending, -1 padded.
- * block_scores (nullable) [b][n_q][m] fp32: q . block_key of each kept block
+ * block_scores (nullable) [b][n_q][m] fp32: the indexer score of each kept block
  * (NaN for padding).  dev_status (nullable): see conventions.  Workspace:
  * hisa_block_topm_workspace_size bytes.  With many queries per sequence the
  * scores come from a tcgen05 tensor-core kernel that splits each fp32 block
  * key into three bf16 terms (fp32-faithful; exact on integer inputs), with
  * few queries from a CUDA-core kernel. */
 hisa_status_t hisa_block_topm_workspace_size(const hisa_params_t* params, size_t* bytes);
-hisa_status_t hisa_block_topm(const hisa_params_t* params, const void* q_idx, const float* block_keys,
-                              int32_t* block_idx, float* block_scores, int32_t* dev_status, void* workspace,
-                              size_t workspace_bytes, cudaStream_t stream);
+hisa_status_t hisa_block_topm(const hisa_params_t* params, const void* q_idx, const float* idx_weights,
+                              const float* block_keys, int32_t* block_idx, float* block_scores, int32_t* dev_status,
+                              void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* Steps 4-5 -- [IP] 1.2.2 items 1-2; [QB] "塊內精挑字符".
  * token_idx[s][i][0..k): the min(k, candidates) best tokens t <= p_i of the
@@ -119,8 +137,8 @@ hisa_status_t hisa_block_topm(const hisa_params_t* params, const void* q_idx, co
  * the reported minimum works; more lets more queries run per launch. */
 hisa_status_t hisa_token_topk_workspace_size(const hisa_params_t* params, size_t* min_bytes,
                                              size_t* preferred_bytes);
-hisa_status_t hisa_token_topk(const hisa_params_t* params, const void* q_idx, const void* k_idx,
-                              const int32_t* block_idx, int32_t* token_idx, float* token_scores,
+hisa_status_t hisa_token_topk(const hisa_params_t* params, const void* q_idx, const float* idx_weights,
+                              const void* k_idx, const int32_t* block_idx, int32_t* token_idx, float* token_scores,
                               int32_t* dev_status, void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* Step 6 -- [QB] "HISA的關鍵優勢在於" (the downstream attention is unchanged).
@@ -140,10 +158,10 @@ hisa_status_t sparse_attn_fwd(const hisa_params_t* params, const void* q, const 
 /* Steps 1-6 in one call.  block_idx_out and token_idx_out (nullable) receive
  * the intermediate selections.  Workspace: hisa_forward_workspace_size. */
 hisa_status_t hisa_forward_workspace_size(const hisa_params_t* params, size_t* bytes);
-hisa_status_t hisa_forward(const hisa_params_t* params, const void* q_idx, const void* k_idx, const void* q,
-                           const void* k, const void* v, void* o, float* lse, int32_t* block_idx_out,
-                           int32_t* token_idx_out, int32_t* dev_status, void* workspace, size_t workspace_bytes,
-                           cudaStream_t stream);
+hisa_status_t hisa_forward(const hisa_params_t* params, const void* q_idx, const float* idx_weights,
+                           const void* k_idx, const void* q, const void* k, const void* v, void* o, float* lse,
+                           int32_t* block_idx_out, int32_t* token_idx_out, int32_t* dev_status, void* workspace,
+                           size_t workspace_bytes, cudaStream_t stream);
 
 /* Steps 1-6 with caller-owned block keys that persist between calls (decode
  * serving, [QB] "HISA的關鍵優勢在於": the KV cache is unchanged, so the pooled
@@ -152,10 +170,11 @@ hisa_status_t hisa_forward(const hisa_params_t* params, const void* q_idx, const
  * [refresh_begin, ceil(n_kv/B)): 0 pools everything (e.g. after a prefill),
  * (n_kv - 1) / B refreshes only the block the newest token entered.  Results
  * equal hisa_forward's.  Workspace: hisa_forward_workspace_size bytes. */
-hisa_status_t hisa_forward_cached(const hisa_params_t* params, const void* q_idx, const void* k_idx,
-                                  float* block_keys, int64_t refresh_begin, const void* q, const void* k,
-                                  const void* v, void* o, float* lse, int32_t* block_idx_out, int32_t* token_idx_out,
-                                  int32_t* dev_status, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+hisa_status_t hisa_forward_cached(const hisa_params_t* params, const void* q_idx, const float* idx_weights,
+                                  const void* k_idx, float* block_keys, int64_t refresh_begin, const void* q,
+                                  const void* k, const void* v, void* o, float* lse, int32_t* block_idx_out,
+                                  int32_t* token_idx_out, int32_t* dev_status, void* workspace,
+                                  size_t workspace_bytes, cudaStream_t stream);
 
 /* The flat token indexer the two-level one replaces ([IP] 1.1 item 1; [QB]
  * "兩步消除上下文索引瓶頸"): token_idx[s][i] = the min(k, p_i+1) best tokens
@@ -163,9 +182,9 @@ hisa_status_t hisa_forward_cached(const hisa_params_t* params, const void* q_idx
  * used as the speed comparator and for the degeneration check. */
 hisa_status_t hisa_flat_topk_workspace_size(const hisa_params_t* params, size_t* min_bytes,
                                             size_t* preferred_bytes);
-hisa_status_t hisa_flat_topk(const hisa_params_t* params, const void* q_idx, const void* k_idx,
-                             int32_t* token_idx, float* token_scores, void* workspace, size_t workspace_bytes,
-                             cudaStream_t stream);
+hisa_status_t hisa_flat_topk(const hisa_params_t* params, const void* q_idx, const float* idx_weights,
+                             const void* k_idx, int32_t* token_idx, float* token_scores, void* workspace,
+                             size_t workspace_bytes, cudaStream_t stream);
 
 /* The token stage (steps 4-5) for callers that cannot allocate device memory.
  * The pages have no counterpart of this call; it exists for users of the
@@ -182,9 +201,9 @@ hisa_status_t hisa_flat_topk(const hisa_params_t* params, const void* q_idx, con
  * each device looks up the array's device address; make that first call
  * before any stream capture.  All calls share the array: calls that overlap
  * on the GPU (other streams or host threads) race, so serialize them. */
-hisa_status_t hisa_token_topk_noalloc(const hisa_params_t* params, const void* q_idx, const void* k_idx,
-                                      const int32_t* block_idx, int32_t* token_idx, float* token_scores,
-                                      int32_t* dev_status, cudaStream_t stream);
+hisa_status_t hisa_token_topk_noalloc(const hisa_params_t* params, const void* q_idx, const float* idx_weights,
+                                      const void* k_idx, const int32_t* block_idx, int32_t* token_idx,
+                                      float* token_scores, int32_t* dev_status, cudaStream_t stream);
 
 /* ---- Decode with the context split across ranks (context parallelism) ----
  * Rank r owns tokens [t0, t0 + n_loc) of every sequence, t0 = first_block * B
@@ -212,8 +231,9 @@ hisa_status_t hisa_block_candidates_workspace_size(const hisa_params_t* local, s
  * be 1 (HISA_ERR_UNSUPPORTED otherwise); block_keys are this rank's pooled
  * keys [batch][ceil(n_loc / B)][d_idx]. */
 hisa_status_t hisa_block_candidates(const hisa_params_t* local, int64_t n_kv_global, int64_t first_block,
-                                    const void* q_idx, const float* block_keys, float* cand_scores,
-                                    int32_t* cand_ids, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+                                    const void* q_idx, const float* idx_weights, const float* block_keys,
+                                    float* cand_scores, int32_t* cand_ids, void* workspace, size_t workspace_bytes,
+                                    cudaStream_t stream);
 /* The best k (score descending, id ascending) of each row's candidates, given
  * as n_parts parts of [rows][n_per] each (the rank-major all-gather layout
  * [n_parts][rows][n_per]; entries with id -1 are empty).  Ties are resolved by

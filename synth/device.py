@@ -12,7 +12,7 @@ import subprocess
 import numpy as np
 
 from . import T_K, T_KIDX, T_Q, T_QIDX, T_V
-from .workloads import Workload, needle_table, probe_signs
+from .workloads import Workload, needle_table, probe_signs, w_idx_rows
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libsynth.so")
@@ -71,11 +71,16 @@ def device_inputs(w: Workload, device="cuda", with_attention: bool = True, strea
     import torch
 
     bf = torch.bfloat16
+    q_shape = (w.batch, w.n_q, w.d_idx) if w.n_idx_heads == 0 else (w.batch, w.n_q, w.n_idx_heads, w.d_idx)
     out = {
-        "q_idx": torch.empty((w.batch, w.n_q, w.d_idx), dtype=bf, device=device),
+        "q_idx": torch.empty(q_shape, dtype=bf, device=device),
         "k_idx": torch.empty((w.batch, w.n_kv, w.d_idx), dtype=bf, device=device),
     }
     fill_int(out["q_idx"], w.seed, T_QIDX, 0, stream)
+    if w.n_idx_heads:
+        # the indexer's head weights: few values, generated on the host half of the generator
+        wts = np.stack([w_idx_rows(w, s, 0, w.n_q) for s in range(w.batch)])
+        out["w_idx"] = torch.from_numpy(wts).to(device)
     fill_int(out["k_idx"], w.seed, T_KIDX, 0, stream)
     if w.needles > 0:
         tables = np.stack([needle_table(w, s) for s in range(w.batch)]).astype(np.int32)

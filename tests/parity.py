@@ -13,6 +13,18 @@ from synth.workloads import Workload, k_idx_rows, k_rows, q_idx_rows, q_rows, v_
 ATOL, RTOL = 2e-3, 1e-2
 
 
+def dev_inputs(inp: dict, device="cuda") -> dict:
+    """Host inputs on the device: bf16 bit arrays as bf16 tensors, the fp32 head weights as fp32."""
+    import torch
+
+    out = {}
+    for k, v in inp.items():
+        if k.startswith("_"):
+            continue
+        out[k] = torch.from_numpy(np.ascontiguousarray(v)).to(device) if v.dtype == np.float32 else to_dev(v, device)
+    return out
+
+
 def to_dev(a_u16: np.ndarray, device="cuda"):
     import torch
 
@@ -48,10 +60,11 @@ def run_stages(hs, w: Workload, dev: dict, attention=True):
     status = torch.zeros(1, dtype=torch.int32, device=d)
     blk = torch.empty((w.batch, w.n_q, w.top_m), dtype=torch.int32, device=d)
     bsc = torch.empty((w.batch, w.n_q, w.top_m), dtype=torch.float32, device=d)
-    hs.hisa_block_topm(p, dev["q_idx"], bk, blk, bsc, status)
+    wi = dev.get("w_idx")  # the indexer's head weights (multi-head indexer only)
+    hs.hisa_block_topm(p, dev["q_idx"], bk, blk, bsc, status, idx_weights=wi)
     tok = torch.empty((w.batch, w.n_q, w.top_k), dtype=torch.int32, device=d)
     tsc = torch.empty((w.batch, w.n_q, w.top_k), dtype=torch.float32, device=d)
-    hs.hisa_token_topk(p, dev["q_idx"], dev["k_idx"], blk, tok, tsc, status)
+    hs.hisa_token_topk(p, dev["q_idx"], dev["k_idx"], blk, tok, tsc, status, idx_weights=wi)
     out = {"block_keys": bk, "block_idx": blk, "block_scores": bsc, "token_idx": tok, "token_scores": tsc,
            "status": status}
     if attention:
@@ -73,7 +86,8 @@ def run_forward(hs, w: Workload, dev: dict):
     blk = torch.empty((w.batch, w.n_q, w.top_m), dtype=torch.int32, device=d)
     tok = torch.empty((w.batch, w.n_q, w.top_k), dtype=torch.int32, device=d)
     status = torch.zeros(1, dtype=torch.int32, device=d)
-    hs.hisa_forward(p, dev["q_idx"], dev["k_idx"], dev["q"], dev["k"], dev["v"], o, lse, blk, tok, status)
+    hs.hisa_forward(p, dev["q_idx"], dev["k_idx"], dev["q"], dev["k"], dev["v"], o, lse, blk, tok, status,
+                    idx_weights=dev.get("w_idx"))
     torch.cuda.synchronize()
     return {"o": o, "lse": lse, "block_idx": blk, "token_idx": tok, "status": status}
 

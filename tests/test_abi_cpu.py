@@ -97,16 +97,36 @@ def test_workspace_checks_before_launch():
     a = ctypes.c_void_p(4096)
     need = hs.hisa_block_topm_workspace_size(p)
     assert need >= 1024 * 16 * 4
-    assert lib.hisa_block_topm(ctypes.byref(p), a, a, a, None, None, a, need - 1, None) == hs.HISA_ERR_WORKSPACE
-    assert lib.hisa_block_topm(ctypes.byref(p), a, a, a, None, None, None, need, None) == hs.HISA_ERR_WORKSPACE
+    assert lib.hisa_block_topm(ctypes.byref(p), a, None, a, a, None, None, a, need - 1, None) == hs.HISA_ERR_WORKSPACE
+    assert lib.hisa_block_topm(ctypes.byref(p), a, None, a, a, None, None, None, need, None) == hs.HISA_ERR_WORKSPACE
     mn, pref = hs.hisa_token_topk_workspace_size(p)
     assert mn == p.top_m * p.block * 4 and pref == mn * p.n_q
-    assert lib.hisa_token_topk(ctypes.byref(p), a, a, a, a, None, None, a, mn - 4, None) == hs.HISA_ERR_WORKSPACE
+    assert lib.hisa_token_topk(ctypes.byref(p), a, None, a, a, a, None, None, a, mn - 4, None) == hs.HISA_ERR_WORKSPACE
     fmin, fpref = hs.hisa_flat_topk_workspace_size(p)
     assert fmin == 16 * 64 * 4
     need_f = hs.hisa_forward_workspace_size(p)
-    assert lib.hisa_forward(ctypes.byref(p), a, a, a, a, a, a, None, None, None, None, a, need_f - 1,
+    assert lib.hisa_forward(ctypes.byref(p), a, None, a, a, a, a, a, None, None, None, None, a, need_f - 1,
                             None) == hs.HISA_ERR_WORKSPACE
+
+
+def test_indexer_heads_and_weights_go_together():
+    """n_idx_heads = 0 takes no head weights; n_idx_heads >= 1 requires them; more than 16 heads
+    are outside the supported range.  All rejected on the host, before any launch."""
+    lib = hs.lib()
+    a = ctypes.c_void_p(4096)
+    p = _p()
+    need = hs.hisa_block_topm_workspace_size(p)
+    assert lib.hisa_block_topm(ctypes.byref(p), a, a, a, a, None, None, a, need, None) == hs.HISA_ERR_INVALID_ARG
+    p.n_idx_heads = 4
+    assert lib.hisa_block_topm(ctypes.byref(p), a, None, a, a, None, None, a, need, None) == hs.HISA_ERR_INVALID_ARG
+    mn, _ = hs.hisa_token_topk_workspace_size(p)
+    assert lib.hisa_token_topk(ctypes.byref(p), a, None, a, a, a, None, None, a, mn, None) == hs.HISA_ERR_INVALID_ARG
+    assert lib.hisa_token_topk(ctypes.byref(p), a, ctypes.c_void_p(4098), a, a, a, None, None, a, mn,
+                               None) == hs.HISA_ERR_INVALID_ARG  # weights not 4-byte aligned
+    p.n_idx_heads = 17
+    assert lib.hisa_block_topm(ctypes.byref(p), a, a, a, a, None, None, a, need, None) == hs.HISA_ERR_UNSUPPORTED
+    p.n_idx_heads = -1
+    assert lib.hisa_block_topm(ctypes.byref(p), a, a, a, a, None, None, a, need, None) == hs.HISA_ERR_INVALID_ARG
 
 
 def test_workspace_sizes_follow_the_shapes():

@@ -39,7 +39,7 @@ class OraclePhases:
     def __init__(self, oracle, w):
         self.O, self.w = oracle, w
 
-    def blocks(self, pl, shard, q_idx, k_idx):
+    def blocks(self, pl, shard, q_idx, k_idx, idx_weights=None):
         w = self.w
         m, c = w.top_m, (shard.n_kv_global - 1) // w.block
         scores = np.full((w.batch, m), np.nan, dtype=np.float32)
@@ -67,7 +67,7 @@ class OraclePhases:
             out[r, : len(order)] = np.sort(ids[r][v][order])
         return torch.from_numpy(out), None
 
-    def tokens(self, pl, shard, q_idx, k_idx, block_idx, status=None):
+    def tokens(self, pl, shard, q_idx, k_idx, block_idx, status=None, idx_weights=None):
         w = self.w
         scores = np.full((w.batch, w.top_k), np.nan, dtype=np.float32)
         ids = np.full((w.batch, w.top_k), -1, dtype=np.int32)

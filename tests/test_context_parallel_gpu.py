@@ -12,7 +12,7 @@ import pytest
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
-from parity import assert_close, run_stages, to_dev  # noqa: E402
+from parity import assert_close, dev_inputs, run_stages, to_dev  # noqa: E402
 from synth.workloads import Workload, full_inputs  # noqa: E402
 
 
@@ -53,7 +53,9 @@ def _run_ranks(hs, w, inp, world):
             bk = torch.empty((w.batch, sh.n_blk, w.d_idx), dtype=torch.float32, device="cuda")
             hs.hisa_block_pool(pl, k_idx, bk)
             status = torch.zeros(1, dtype=torch.int32, device="cuda")
-            blk, tok, o, lse = cp.decode_step(p, sh, q_idx, k_idx, bk, q, k, v, exchange_of(r), status=status)
+            wi = torch.from_numpy(inp["w_idx"]).cuda() if w.n_idx_heads else None
+            blk, tok, o, lse = cp.decode_step(p, sh, q_idx, k_idx, bk, q, k, v, exchange_of(r), status=status,
+                                              idx_weights=wi)
             torch.cuda.synchronize()
             results[r] = (blk.cpu().numpy(), tok.cpu().numpy(), o.float().cpu().numpy(), lse.cpu().numpy(),
                           int(status.item()))
@@ -77,6 +79,7 @@ CASES = [
     (Workload("cp_gqa", 3, 1, 9000, 128, 128, 6, 500, 8, 2, 128), 2),
     (Workload("cp_all_blocks", 1, 1, 2500, 64, 64, 64, 2000, 2, 2, 64), 4),
     (Workload("cp_one_rank", 2, 1, 5000, 64, 64, 8, 300, 4, 4, 64), 1),
+    (Workload("cp_multihead_indexer", 2, 1, 7000, 64, 64, 8, 300, 4, 4, 64, n_idx_heads=4), 3),
 ]
 
 
@@ -84,7 +87,7 @@ CASES = [
 def test_split_context_decode_matches_oracle(hs, oracle_lib, w, world):
     inp = full_inputs(w)
     ref = oracle_lib.run(w, inp)
-    one = run_stages(hs, w, {k: to_dev(v) for k, v in inp.items() if not k.startswith("_")})
+    one = run_stages(hs, w, dev_inputs(inp))
     n = w.batch
     for blk, tok, o, lse, status in _run_ranks(hs, w, inp, world):
         assert status == 0

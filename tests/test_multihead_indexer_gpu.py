@@ -1,0 +1,77 @@
+"""GPU parity of the indexer's multi-head weighted score, sum_j w_j * ReLU(q_j . k), the original
+indexer's own score function that the pages ask to keep ("北大HISA稀疏注意力机制" section 1.3
+item 4).  The block and token stages must select exactly what the oracle selects, the token
+scores must equal an exact integer recomputation, and attention over the selection stays within
+the parity tolerance.  Integer inputs and integer weights keep every score exact: each case
+keeps log2(heads * 3 * 16 * d_idx) + log2(B) below 24 bits."""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+from parity import assert_close, dev_inputs, run_forward, run_stages  # noqa: E402
+from synth.workloads import Workload, full_inputs  # noqa: E402
+
+
+@pytest.fixture(scope="module")
+def hs():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import hierarchical_sparse_attention_block_b200 as m
+
+    return m
+
+
+CASES = [
+    # name, batch, n_q, n_kv, d_idx, block, top_m, top_k, n_heads, n_kv_heads, d_head, needles, seed, n_idx_heads
+    Workload("mh1_prefill", 1, 600, 600, 64, 32, 6, 120, 2, 2, 64, 0, 0, 1),
+    Workload("mh4_prefill", 2, 300, 900, 128, 64, 5, 200, 4, 4, 128, 2, 0, 4),
+    Workload("mh16_prefill", 1, 257, 700, 64, 32, 4, 150, 2, 1, 64, 0, 0, 16),
+    Workload("mh2_d256", 1, 300, 800, 256, 64, 5, 100, 2, 2, 64, 0, 0, 2),
+    Workload("mh8_decode", 3, 1, 5000, 64, 64, 8, 300, 2, 2, 64, 0, 0, 8),
+]
+
+
+def _exact_token_scores(inp, w, r, tok):
+    """sum_j w_j * max(0, q_j . k_t) in int64 for the tokens of query row r."""
+    seq, i = divmod(r, w.n_q)
+    q = (inp["q_idx"][seq, i].astype(np.uint32) << 16).view(np.float32).astype(np.int64)  # [H][d]
+    k = (inp["k_idx"][seq][tok].astype(np.uint32) << 16).view(np.float32).astype(np.int64)  # [n][d]
+    wts = inp["w_idx"][seq, i].astype(np.int64)
+    return (np.maximum(k @ q.T, 0) * wts).sum(axis=1)
+
+
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+def test_multihead_stages_match_oracle(hs, oracle_lib, w):
+    inp = full_inputs(w)
+    ref = oracle_lib.run(w, inp)
+    got = run_stages(hs, w, dev_inputs(inp))
+    n = w.batch * w.n_q
+    assert np.array_equal(got["block_idx"].cpu().numpy().reshape(n, w.top_m), ref["block_idx"])
+    tok = got["token_idx"].cpu().numpy().reshape(n, w.top_k)
+    assert np.array_equal(tok, ref["token_idx"]), np.argwhere(tok != ref["token_idx"])[:5]
+    assert int(got["status"].item()) == 0
+    ts = got["token_scores"].cpu().numpy().reshape(n, w.top_k)
+    for r in range(0, n, max(1, n // 40)):
+        v = tok[r] >= 0
+        assert np.array_equal(ts[r][v], _exact_token_scores(inp, w, r, tok[r][v]).astype(np.float32))
+    assert_close(got["o"].float().cpu().numpy().reshape(n, w.n_heads, w.d_head), ref["o"], "o")
+    assert_close(got["lse"].cpu().numpy().reshape(n, w.n_heads), ref["lse"], "lse")
+
+
+@pytest.mark.parametrize("w", [CASES[1], CASES[4]], ids=lambda w: w.name)
+def test_multihead_forward_and_flat(hs, oracle_lib, w):
+    inp = full_inputs(w)
+    dev = dev_inputs(inp)
+    ref = oracle_lib.run(w, inp)
+    got = run_forward(hs, w, dev)
+    n = w.batch * w.n_q
+    assert np.array_equal(got["token_idx"].cpu().numpy().reshape(n, w.top_k), ref["token_idx"])
+    assert_close(got["o"].float().cpu().numpy().reshape(n, w.n_heads, w.d_head), ref["o"], "o")
+    # the flat comparator scores every visible token with the same function
+    flat_ref = oracle_lib.run(w, inp, flat=True, attention=False)
+    p = hs.params_of(w)
+    tok = torch.empty((w.batch, w.n_q, w.top_k), dtype=torch.int32, device="cuda")
+    hs.hisa_flat_topk(p, dev["q_idx"], dev["k_idx"], tok, idx_weights=dev["w_idx"])
+    assert np.array_equal(tok.cpu().numpy().reshape(n, w.top_k), flat_ref["token_idx"])

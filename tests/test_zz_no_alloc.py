@@ -37,7 +37,7 @@ def _call_noalloc(hs, w, dev, blk):
     sc = torch.full((w.batch, w.n_q, w.top_k), 7.0, dtype=torch.float32, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-    rc = hs.lib().hisa_token_topk_noalloc(ctypes.byref(p), ctypes.c_void_p(dev["q_idx"].data_ptr()),
+    rc = hs.lib().hisa_token_topk_noalloc(ctypes.byref(p), ctypes.c_void_p(dev["q_idx"].data_ptr()), None,
                                           ctypes.c_void_p(dev["k_idx"].data_ptr()), ctypes.c_void_p(blk.data_ptr()),
                                           ctypes.c_void_p(tok.data_ptr()), ctypes.c_void_p(sc.data_ptr()),
                                           ctypes.c_void_p(status.data_ptr()), stream)
@@ -72,6 +72,6 @@ def test_noalloc_rejects_a_query_larger_than_the_array(hs):
     # one query would need 4096 blocks x 2048 tokens x 4 B = 32 MiB of keys > 16 MiB
     p = hs.params(1, 1, 1 << 23, 128, 2048, 4096, 16)
     a = ctypes.c_void_p(1 << 20)
-    rc = hs.lib().hisa_token_topk_noalloc(ctypes.byref(p), a, a, a, a, None, None, None)
+    rc = hs.lib().hisa_token_topk_noalloc(ctypes.byref(p), a, None, a, a, a, None, None, None)
     assert rc == hs.HISA_ERR_UNSUPPORTED
     _ = np
