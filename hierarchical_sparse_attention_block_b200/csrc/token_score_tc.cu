@@ -40,7 +40,9 @@ struct TsLayout {
   static constexpr int K_OFF = Q_OFF + Q_BYTES;
   static constexpr int MAP_OFF = K_OFF + STAGES * K_BYTES;  // int16 [kTileQ][kRun]
   static constexpr int BAR_OFF = MAP_OFF + kTileQ * kRun * 2;
-  static constexpr int SMEM = BAR_OFF + 8 * (2 + STAGES) + 16 + 1024;
+  static constexpr int NBAR = 3 + STAGES;  // q, MMA done x 2 accumulators, K stages
+  static constexpr int SMEM = BAR_OFF + 8 * NBAR + 16 + 1024;
+  static constexpr uint32_t TMEM_COLS = 2 * B;  // two B-column accumulators
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
   static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(B >> 3) << 17) |
                                     ((uint32_t)(kTileQ >> 4) << 24);
@@ -53,23 +55,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     token_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                           const int32_t* __restrict__ block_idx, int slots, uint32_t* __restrict__ keys,
                           int32_t* __restrict__ status, int64_t n_q, int64_t n_kv, int q_tiles, int runs, int64_t q0,
-                          int64_t nq) {
+                          int64_t nq, const float* __restrict__ w_idx, int HI) {
   using L = TsLayout<D, B>;
   constexpr int kKStages = L::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
 
+  // Rows of the tile are (query, indexer head) pairs: QT queries x HE heads.
+  const int HE = HI > 0 ? HI : 1;
+  const int QT = kTileQ / HE;
   // Tiles are enumerated over the queries of the chunk [q0, q0 + nq).
   const int run = blockIdx.x % runs;
   const int64_t tile_lin = blockIdx.x / runs;
   const int64_t seq_first = q0 / n_q;
-  const int64_t tile0 = (q0 % n_q) / kTileQ;  // first tile of the first sequence touched
+  const int64_t tile0 = (q0 % n_q) / QT;      // first tile of the first sequence touched
   const int64_t tile_abs = tile0 + tile_lin;  // tile counted from the first sequence's start
   const int64_t seq = seq_first + tile_abs / q_tiles;
   const int64_t ti = tile_abs % q_tiles;
-  const int64_t tq0 = seq * n_q + ti * kTileQ;                 // first global query of the tile
+  const int64_t tq0 = seq * n_q + ti * QT;                     // first global query of the tile
   const int64_t t_lo = max(tq0, q0);
-  const int64_t t_hi = min(min(tq0 + kTileQ, (seq + 1) * n_q), q0 + nq);  // exclusive
+  const int64_t t_hi = min(min(tq0 + QT, (seq + 1) * n_q), q0 + nq);  // exclusive
   if (t_lo >= t_hi) return;
   const int64_t c_max = (n_kv - n_q + (t_hi - 1 - seq * n_q)) / B;
   const int64_t jb0 = (int64_t)run * kRun;
@@ -80,16 +85,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sQ = smem + L::Q_OFF;
   uint8_t* sK = smem + L::K_OFF;
   int16_t* smap = reinterpret_cast<int16_t*>(smem + L::MAP_OFF);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);  // [0] q, [1] mma, [2..] k stages
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::BAR_OFF + 8 * (2 + kKStages));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);  // [0] q, [1..2] mma done, [3..] k stages
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::BAR_OFF + 8 * L::NBAR);
 
   if (warp == 0) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                 "r"((uint32_t)(B < 32 ? 32 : B)));
+                 "r"(L::TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   if (tid == 0) {
-    for (int i = 0; i < 2 + kKStages; ++i)
+    for (int i = 0; i < L::NBAR; ++i)
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars[i])));
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -103,9 +108,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t bq = smem_u32(&bars[0]);
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bq), "r"((uint32_t)L::Q_BYTES)
                  : "memory");
-    for (int hh = 0; hh < L::HALVES; ++hh) tma_load_2d(smem_u32(sQ + hh * kTileQ * 128), &tmap_q, hh * 64, (int)tq0, bq);
+    for (int hh = 0; hh < L::HALVES; ++hh)
+      tma_load_2d(smem_u32(sQ + hh * kTileQ * 128), &tmap_q, hh * 64, (int)(tq0 * HE), bq);
     for (int s = 0; s < kKStages && s < nb; ++s) {
-      const uint32_t bk = smem_u32(&bars[2 + s]);
+      const uint32_t bk = smem_u32(&bars[3 + s]);
       asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bk), "r"((uint32_t)L::K_BYTES)
                    : "memory");
       const int krow = (int)(seq * n_kv + (jb0 + s) * B);
@@ -114,13 +120,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  // Slot map of this thread's query row for blocks jb0 .. jb0+nb-1.
-  const int64_t qrow = tq0 + tid;  // global query id of this thread's row
-  const bool row_ok = qrow >= t_lo && qrow < t_hi;
+  // Slot map of query tid of the tile (threads tid < QT) for blocks jb0 .. jb0+nb-1.
+  {
+  const int64_t qrow = tq0 + tid;  // global query id
+  const bool row_ok = tid < QT && qrow >= t_lo && qrow < t_hi;
   const int64_t p = n_kv - n_q + (qrow - seq * n_q);
   const int64_t c = p / B;
   uint32_t* krow_keys = keys + (qrow - q0) * (int64_t)slots * B;
-  for (int jj = 0; jj < kRun; ++jj) smap[tid * kRun + jj] = -1;
+  if (tid < QT)
+    for (int jj = 0; jj < kRun; ++jj) smap[tid * kRun + jj] = -1;
   if (row_ok) {
     if (block_idx) {
       const int32_t* lst = block_idx + qrow * slots;
@@ -148,37 +156,51 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   }
+  }
+
+  // This thread's TMEM lane = tile row tid: query tq0 + tid / HE, indexer head tid % HE.
+  const int qi = tid / HE, head = tid % HE;
+  const int64_t qrow = tq0 + qi;
+  const bool row_ok = qrow >= t_lo && qrow < t_hi;
+  const int64_t p = n_kv - n_q + (qrow - seq * n_q);
+  uint32_t* krow_keys = keys + (qrow - q0) * (int64_t)slots * B;
+  const float wgt = (HI > 0 && row_ok) ? w_idx[qrow * HI + head] : 1.f;
+  __syncthreads();  // the slot maps are complete
 
   bool ok = mbar_wait(smem_u32(&bars[0]), 0);
   ok = __syncthreads_and(ok) != 0;
   const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK);
-  for (int b = 0; b < nb && ok; ++b) {
-    const int stage = b % kKStages;
-    const uint32_t phase = (uint32_t)((b / kKStages) & 1);
-    if (tid == 0) {
-      if (mbar_wait(smem_u32(&bars[2 + stage]), phase)) {
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  // Thread 0: once block bb's K stage has landed, its scores go to accumulator bb & 1 (B columns).
+  auto issue_mma = [&](int bb) -> bool {
+    const int stage = bb % kKStages;
+    if (!mbar_wait(smem_u32(&bars[3 + stage]), (uint32_t)((bb / kKStages) & 1))) return false;
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t acc_col = tmem + (uint32_t)((bb & 1) * B);
 #pragma unroll
-        for (int hh = 0; hh < L::HALVES; ++hh) {
+    for (int hh = 0; hh < L::HALVES; ++hh) {
 #pragma unroll
-          for (int s = 0; s < 4; ++s) {
-            const uint64_t ad = desc_kmajor_sw128(q_base + hh * kTileQ * 128 + s * 32);
-            const uint64_t bd = desc_kmajor_sw128(k_base + stage * L::K_BYTES + hh * B * 128 + s * 32);
-            const uint32_t acc = (hh | s) ? 1u : 0u;
-            asm volatile(
-                "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-                " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem),
-                "l"(ad), "l"(bd), "r"(L::IDESC), "r"(acc));
-          }
-        }
-        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                         smem_u32(&bars[1]))
-                     : "memory");
-      } else {
-        if (status) atomicOr(status, kStatusTimeout);
+      for (int s = 0; s < 4; ++s) {
+        const uint64_t ad = desc_kmajor_sw128(q_base + hh * kTileQ * 128 + s * 32);
+        const uint64_t bd = desc_kmajor_sw128(k_base + stage * L::K_BYTES + hh * B * 128 + s * 32);
+        const uint32_t acc = (hh | s) ? 1u : 0u;
+        asm volatile(
+            "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+            " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(acc_col),
+            "l"(ad), "l"(bd), "r"(L::IDESC), "r"(acc));
       }
     }
-    bool done = mbar_wait(smem_u32(&bars[1]), (uint32_t)(b & 1));
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(&bars[1 + (bb & 1)]))
+                 : "memory");
+    return true;
+  };
+  if (ok && tid == 0 && nb > 0 && !issue_mma(0) && status) atomicOr(status, kStatusTimeout);
+  for (int b = 0; b < nb && ok; ++b) {
+    const int stage = b % kKStages;
+    // The next block's scores are computed while this block's are read: its accumulator was last
+    // read in iteration b - 1, which every warp finished before that iteration's closing barrier.
+    if (tid == 0 && b + 1 < nb && !issue_mma(b + 1) && status) atomicOr(status, kStatusTimeout);
+    bool done = mbar_wait(smem_u32(&bars[1 + (b & 1)]), (uint32_t)((b >> 1) & 1));
     done = __syncthreads_and(done) != 0;
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     if (!done) {
@@ -188,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // The MMA has consumed this K stage: refill it with block b + kKStages.
     if (tid == 0 && b + kKStages < nb) {
-      const uint32_t bk = smem_u32(&bars[2 + stage]);
+      const uint32_t bk = smem_u32(&bars[3 + stage]);
       asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bk), "r"((uint32_t)L::K_BYTES)
                    : "memory");
       const int krow = (int)(seq * n_kv + (jb0 + b + kKStages) * B);
@@ -196,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_2d(smem_u32(sK + stage * L::K_BYTES + hh * B * 128), &tmap_k, hh * 64, krow, bk);
     }
     // Epilogue: rows whose query kept block jb0 + b.
-    const int slot = row_ok ? smap[tid * kRun + b] : -1;
+    const int slot = row_ok ? smap[qi * kRun + b] : -1;
     if (__any_sync(0xFFFFFFFFu, slot >= 0)) {
       const int64_t j = jb0 + b;
       const int64_t tok0 = j * B;
@@ -204,7 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
       for (int cc = 0; cc < B / 32; ++cc) {
         uint32_t v[32];
-        const uint32_t addr = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(cc * 32);
+        const uint32_t addr = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)((b & 1) * B + cc * 32);
         asm volatile(
             "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
             "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
@@ -215,16 +237,52 @@ __global__ void __launch_bounds__(kThreads, 1)
               "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
             : "r"(addr));
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-        if (slot >= 0) {
+        if (HI == 0) {
+          if (slot >= 0) {
 #pragma unroll
-          for (int t = 0; t < 32; t += 4) {
-            const int64_t tk = tok0 + cc * 32 + t;
-            uint4 w;
-            w.x = tk <= p ? score_key(__uint_as_float(v[t])) : 0u;
-            w.y = tk + 1 <= p ? score_key(__uint_as_float(v[t + 1])) : 0u;
-            w.z = tk + 2 <= p ? score_key(__uint_as_float(v[t + 2])) : 0u;
-            w.w = tk + 3 <= p ? score_key(__uint_as_float(v[t + 3])) : 0u;
-            *reinterpret_cast<uint4*>(dst + cc * 32 + t) = w;
+            for (int t = 0; t < 32; t += 4) {
+              const int64_t tk = tok0 + cc * 32 + t;
+              uint4 w;
+              w.x = tk <= p ? score_key(__uint_as_float(v[t])) : 0u;
+              w.y = tk + 1 <= p ? score_key(__uint_as_float(v[t + 1])) : 0u;
+              w.z = tk + 2 <= p ? score_key(__uint_as_float(v[t + 2])) : 0u;
+              w.w = tk + 3 <= p ? score_key(__uint_as_float(v[t + 3])) : 0u;
+              *reinterpret_cast<uint4*>(dst + cc * 32 + t) = w;
+            }
+          }
+        } else {
+          // Multi-head score w_j * max(0, q_j . k) per row, summed over the HE rows of a query
+          // with a transposing reduction: after it, the lane of head h holds the sums of tokens
+          // h * (32 / HE) .. (h + 1) * (32 / HE) - 1 of this chunk.
+          float x[32];
+#pragma unroll
+          for (int t = 0; t < 32; ++t) x[t] = wgt * fmaxf(__uint_as_float(v[t]), 0.f);
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            if ((1 << m) < HE) {  // warp-uniform
+              constexpr int kHalfMax = 16;
+              const int half = 16 >> m;
+              const int o = HE >> (m + 1);
+              const bool up = (head & o) != 0;
+#pragma unroll
+              for (int t = 0; t < kHalfMax; ++t) {
+                if (t < half) {
+                  const float send = up ? x[t] : x[t + half];
+                  const float keep = up ? x[t + half] : x[t];
+                  x[t] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, o);
+                }
+              }
+            }
+          }
+          if (slot >= 0) {
+            const int n = 32 / HE, t0 = head * n;
+#pragma unroll
+            for (int t = 0; t < 32; ++t) {
+              if (t < n) {
+                const int64_t tk = tok0 + cc * 32 + t0 + t;
+                dst[cc * 32 + t0 + t] = tk <= p ? score_key(x[t]) : 0u;
+              }
+            }
           }
         }
       }
@@ -237,8 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
   if (warp == 0) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                 "r"((uint32_t)(B < 32 ? 32 : B)));
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(L::TMEM_COLS));
   }
 }
 
@@ -247,28 +304,32 @@ cudaError_t launch_ts(const Shape& s, const void* q_idx, const void* k_idx, cons
                       uint32_t* keys, int32_t* status, int64_t q0, int64_t nq, cudaStream_t st) {
   using L = TsLayout<D, B>;
   CUtensorMap mq, mk;
-  if (!map_bf16_sw128(&mq, q_idx, D, (uint64_t)s.n_query, kTileQ)) return cudaErrorNotSupported;
+  const int HE = s.HI > 0 ? s.HI : 1;
+  const int QT = kTileQ / HE;
+  if (!map_bf16_sw128(&mq, q_idx, D, (uint64_t)s.n_query * HE, kTileQ)) return cudaErrorNotSupported;
   if (!map_bf16_sw128(&mk, k_idx, D, (uint64_t)s.batch * s.n_kv, B)) return cudaErrorNotSupported;
   auto kern = token_score_tc_kernel<D, B>;
   cudaError_t e = ensure_smem((const void*)kern, L::SMEM);
   if (e != cudaSuccess) return e;
-  const int q_tiles = (int)((s.n_q + kTileQ - 1) / kTileQ);
+  const int q_tiles = (int)((s.n_q + QT - 1) / QT);
   const int runs = (int)((s.n_blk + kRun - 1) / kRun);
   // tiles from the chunk's first tile to its last
-  const int64_t first = (q0 / s.n_q) * q_tiles + (q0 % s.n_q) / kTileQ;
+  const int64_t first = (q0 / s.n_q) * q_tiles + (q0 % s.n_q) / QT;
   const int64_t lastq = q0 + nq - 1;
-  const int64_t last = (lastq / s.n_q) * q_tiles + (lastq % s.n_q) / kTileQ;
+  const int64_t last = (lastq / s.n_q) * q_tiles + (lastq % s.n_q) / QT;
   const int64_t grid = (last - first + 1) * runs;
   if (grid > 0x7FFFFFFFLL) return cudaErrorNotSupported;
   kern<<<(unsigned)grid, kThreads, L::SMEM, st>>>(mq, mk, block_idx, slots, keys, status, s.n_q, s.n_kv, q_tiles,
-                                                  runs, q0, nq);
+                                                  runs, q0, nq, s.w_idx, s.HI);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 bool token_score_tc_eligible(const Shape& s, int slots) {
-  return s.HI == 0 && (s.d_idx == 64 || s.d_idx == 128) && (s.B == 32 || s.B == 64 || s.B == 128 || s.B == 256) &&
+  // a query's indexer heads are consecutive rows of a warp: 1, 2, 4, 8 or 16 of them
+  const bool heads_ok = s.HI == 0 || (s.HI <= 16 && (s.HI & (s.HI - 1)) == 0);
+  return heads_ok && (s.d_idx == 64 || s.d_idx == 128) && (s.B == 32 || s.B == 64 || s.B == 128 || s.B == 256) &&
          s.n_q >= kTileQ && slots < 32767 && s.n_query <= 0x7FFFFFFFLL &&
          (int64_t)s.batch * s.n_kv <= 0x7FFFFFFFLL;
 }
