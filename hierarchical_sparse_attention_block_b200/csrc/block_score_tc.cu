@@ -59,8 +59,11 @@ template <int D>
 __global__ void __launch_bounds__(kTcThreads, 1)
     block_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_bk,
                           float* __restrict__ scores, int32_t* __restrict__ status, int64_t n_q, int64_t n_kv,
-                          int B, int64_t n_blk, int q_tiles, int n_tiles) {
+                          int B, int64_t n_blk, int q_tiles, int n_tiles, const float* __restrict__ w_idx, int HI) {
   using L = TcLayout<D>;
+  // Rows of the tile are (query, indexer head) pairs: QT queries x HE heads.
+  const int HE = HI > 0 ? HI : 1;
+  const int QT = kTileM / HE;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
 
@@ -68,8 +71,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int qt_all = blockIdx.x / n_tiles;
   const int seq = qt_all / q_tiles;
   const int qt = qt_all % q_tiles;
-  const int64_t q0 = (int64_t)qt * kTileM;
-  const int64_t q_last = min(q0 + kTileM, n_q) - 1;
+  const int64_t q0 = (int64_t)qt * QT;
+  const int64_t q_last = min(q0 + QT, n_q) - 1;
   const int64_t c_max = (n_kv - n_q + q_last) / B;
   const int64_t j0 = (int64_t)nt * kTileN;
   if (j0 > c_max) return;  // whole tile above the causal diagonal
@@ -100,7 +103,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (tid == 0) {
     const uint32_t tx = (uint32_t)(L::A_BYTES + L::S_BYTES);
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar_tma), "r"(tx) : "memory");
-    const int32_t qrow = (int32_t)((int64_t)seq * n_q + q0);
+    const int32_t qrow = (int32_t)(((int64_t)seq * n_q + q0) * HE);
 #pragma unroll
     for (int h = 0; h < L::HALVES; ++h) {
       asm volatile(
@@ -189,10 +192,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   ok = done;
 
   if (ok) {
-    const int64_t qi = q0 + warp * 32 + lane;  // this thread's query row within the sequence
-    const bool row_ok = qi < n_q;
+    // this thread's TMEM lane = tile row tid: query q0 + tid / HE (within the sequence), head tid % HE
+    const int head = tid % HE;
+    const int64_t qi = q0 + tid / HE;
+    const bool row_ok = tid / HE < QT && qi < n_q;
     const int64_t c = row_ok ? (n_kv - n_q + qi) / B : -1;
     float* out = scores + ((int64_t)seq * n_q + qi) * n_blk;
+    const float wgt = (HI > 0 && row_ok) ? w_idx[((int64_t)seq * n_q + qi) * HI + head] : 1.f;
 #pragma unroll
     for (int cc = 0; cc < kTileN / 32; ++cc) {
       uint32_t v[32];
@@ -208,7 +214,35 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           : "r"(addr));
       asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
       const int64_t jb = j0 + cc * 32;
-      if (row_ok && jb <= c) {
+      if (HI > 0) {
+        // w_j * max(0, q_j . bk) per row, summed over a query's HE rows by a transposing reduction:
+        // the lane of head h ends with the scores of blocks jb + h * (32 / HE) .. + 32 / HE - 1.
+        float x[32];
+#pragma unroll
+        for (int t = 0; t < 32; ++t) x[t] = wgt * fmaxf(__uint_as_float(v[t]), 0.f);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          if ((1 << m) < HE) {  // warp-uniform
+            const int half = 16 >> m;
+            const int o = HE >> (m + 1);
+            const bool up = (head & o) != 0;
+#pragma unroll
+            for (int t = 0; t < 16; ++t) {
+              if (t < half) {
+                const float send = up ? x[t] : x[t + half];
+                const float keep = up ? x[t + half] : x[t];
+                x[t] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, o);
+              }
+            }
+          }
+        }
+        const int n = 32 / HE, t0 = head * n;
+        if (row_ok) {
+#pragma unroll
+          for (int t = 0; t < 32; ++t)
+            if (t < n && jb + t0 + t <= c) out[jb + t0 + t] = x[t];
+        }
+      } else if (row_ok && jb <= c) {
         if (jb + 31 <= c && (n_blk & 3) == 0) {  // 16-byte aligned rows only
 #pragma unroll
           for (int t = 0; t < 32; t += 4)
@@ -238,7 +272,9 @@ cudaError_t launch_tc(const Shape& s, const void* q_idx, const float* bk, float*
                       cudaStream_t st) {
   using L = TcLayout<D>;
   CUtensorMap mq, mb;
-  if (!make_map_2d(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q_idx, D, (uint64_t)s.n_query, 64, kTileM,
+  const int HE = s.HI > 0 ? s.HI : 1;
+  const int QT = kTileM / HE;
+  if (!make_map_2d(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, q_idx, D, (uint64_t)s.n_query * HE, 64, kTileM,
                    CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorNotSupported;
   if (!make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, bk, D, (uint64_t)s.batch * s.n_blk, D, kTileN,
@@ -247,19 +283,22 @@ cudaError_t launch_tc(const Shape& s, const void* q_idx, const float* bk, float*
   auto kern = block_score_tc_kernel<D>;
   cudaError_t e = ensure_smem((const void*)kern, L::SMEM);
   if (e != cudaSuccess) return e;
-  const int q_tiles = (int)((s.n_q + kTileM - 1) / kTileM);
+  const int q_tiles = (int)((s.n_q + QT - 1) / QT);
   const int n_tiles = (int)((s.n_blk + kTileN - 1) / kTileN);
   const int64_t grid = (int64_t)s.batch * q_tiles * n_tiles;
   if (grid > 0x7FFFFFFFLL) return cudaErrorNotSupported;
   kern<<<(unsigned)grid, kTcThreads, L::SMEM, st>>>(mq, mb, scores, status, s.n_q, s.n_kv, s.B, s.n_blk, q_tiles,
-                                                    n_tiles);
+                                                    n_tiles, s.w_idx, s.HI);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 bool block_score_tc_eligible(const Shape& s) {
-  return s.HI == 0 && (s.d_idx == 64 || s.d_idx == 128) && s.n_q >= 64 && s.n_query <= 0x7FFFFFFFLL &&
+  // a query's indexer heads are consecutive rows of a warp: 1, 2, 4, 8 or 16 of them
+  const bool heads_ok = s.HI == 0 || (s.HI <= 16 && (s.HI & (s.HI - 1)) == 0);
+  return heads_ok && (s.d_idx == 64 || s.d_idx == 128) && s.n_q >= 64 &&
+         s.n_query * (s.HI > 0 ? s.HI : 1) <= 0x7FFFFFFFLL &&
          (int64_t)s.batch * s.n_blk <= 0x7FFFFFFFLL;
 }
 
