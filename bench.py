@@ -178,35 +178,66 @@ def attention_bytes(w, counts):
 
 def indexer_bytes(w, counts):
     nq = w.batch * w.n_q
+    hi = max(1, w.n_idx_heads)
     return (counts["n_cand"] * w.d_idx * 2            # token gather
             + w.batch * w.n_kv * w.d_idx * 2            # pooling read
-            + nq * w.d_idx * 2 + nq * (w.top_m + w.top_k) * 4)
+            + nq * hi * w.d_idx * 2 + nq * (w.top_m + w.top_k) * 4)
+
+
+def compulsory_bytes(w):
+    """The floor of any schedule: every input read once (indexer keys and queries, head weights,
+    Q, K, V) and every output written once (O, LSE); the index lists are intermediates."""
+    nq = w.batch * w.n_q
+    hi = max(1, w.n_idx_heads)
+    return (w.batch * w.n_kv * w.d_idx * 2 + nq * hi * w.d_idx * 2 + (nq * hi * 4 if w.n_idx_heads else 0)
+            + w.batch * w.n_kv * w.n_kv_heads * w.d_head * 2 * 2
+            + nq * w.n_heads * w.d_head * 2 * 2 + nq * w.n_heads * 4)
+
+
+def needle_recall(w, block_idx):
+    """Fraction of the planted needle blocks among the probe query's kept blocks (the last query
+    of each sequence: the query whose signs the needles follow), over all sequences."""
+    from synth.workloads import needle_table
+
+    if w.needles <= 0:
+        return None
+    sel = block_idx[:, w.n_q - 1].cpu().numpy()
+    hits = total = 0
+    for seq in range(w.batch):
+        nb = set(needle_table(w, seq).tolist())
+        hits += len(nb & set(sel[seq][sel[seq] >= 0].tolist()))
+        total += len(nb)
+    return hits / total if total else None
 
 
 def l2_gather_peak(hs, dev, st, row_bytes=256, region_bytes=32 << 20, n_gathers=8 << 20):
     """Measured ceiling of the attention kernel's gathers (GB/s): hisa_gather_probe copying
     hashed 256-byte rows of a 32 MiB region (one head's K and V at 64K, L2-resident) into shared
-    memory with the kernel's cp.async pattern and nothing else.  Best of 5 event-timed launches."""
+    memory with the kernel's cp.async pattern and nothing else.  The best of 5 event-timed
+    launches at each of 2 and 3 CTAs (8 and 12 warps) per SM; returns (GB/s, CTAs per SM)."""
     import torch
 
     rows = torch.zeros(region_bytes, dtype=torch.uint8, device=dev)
     sink = torch.zeros(1, dtype=torch.int32, device=dev)
-    for _ in range(2):
-        hs.hisa_gather_probe(rows, row_bytes, n_gathers, sink, stream=st)
-    ts = []
-    for _ in range(5):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(st)
-        hs.hisa_gather_probe(rows, row_bytes, n_gathers, sink, stream=st)
-        e1.record(st)
-        e1.synchronize()
-        ts.append(e0.elapsed_time(e1))
-    return n_gathers * row_bytes / (min(ts) * 1e-3) / 1e9
+    best = (0.0, 0)
+    for ctas in (2, 3):
+        for _ in range(2):
+            hs.hisa_gather_probe(rows, row_bytes, n_gathers, sink, ctas_per_sm=ctas, stream=st)
+        ts = []
+        for _ in range(5):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(st)
+            hs.hisa_gather_probe(rows, row_bytes, n_gathers, sink, ctas_per_sm=ctas, stream=st)
+            e1.record(st)
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        best = max(best, (n_gathers * row_bytes / (min(ts) * 1e-3) / 1e9, ctas))
+    return best
 
 
-def _profile_traffic(kernel_file: str, summary_name: str, workload_name: str):
-    """DRAM bytes per launch from the committed ncu summary of this workload, or None when there
-    is none or the kernel changed since it was taken."""
+def _profile_record(kernel_file: str, summary_name: str, workload_name: str):
+    """The committed ncu record of this kernel on this workload (DRAM bytes per launch, L2 hit
+    rate), or None when there is none or the kernel changed since it was taken."""
     path = os.path.join(ROOT, "profiles", summary_name)
     src = os.path.join(ROOT, "hierarchical_sparse_attention_block_b200", "csrc", kernel_file)
     try:
@@ -215,7 +246,7 @@ def _profile_traffic(kernel_file: str, summary_name: str, workload_name: str):
         sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
         if j.get("source_sha256_16") != sha or j.get("workload") != workload_name:
             return None
-        return j.get("dram_bytes_per_launch_full_workload")
+        return j
     except Exception:
         return None
 
@@ -399,7 +430,7 @@ def run_ours(a, rank, world, local_rank):
                      "frac": achieved / hbm_gbs, "peak_kind": peak_kind,
                      "frac_of_nominal_8tbs": achieved / 8000.0,
                      "algorithmic_bytes_per_launch": a_bytes,
-                     "traffic": _profile_traffic("sparse_attn.cu", f"sparse_attn_{w.name}.json", w.name)},
+                     "traffic": None},
         "stages_ms": {n: statistics.mean(v) for n, v in stage_ms.items()},
         "pool_in_step": "newest block only (cache block keys persist)" if decode else "every block",
         "cuda_graph": use_graph,
@@ -407,19 +438,32 @@ def run_ours(a, rank, world, local_rank):
         "indexer_ms": idx_ms, "indexer_queries_per_s": nq / (idx_ms * 1e-3),
         "tokens_per_s": counts["k_eff"] / (ms * 1e-3),
         "end_to_end_hbm_roofline_frac_8tbs": ((a_bytes + indexer_bytes(w, counts)) / 8e12) / (ms * 1e-3),
+        "compulsory_bytes": None if decode else compulsory_bytes(w),
+        "compulsory_ms_at_8tbs": None if decode else compulsory_bytes(w) / 8e12 * 1e3,
+        "needle_recall": needle_recall(w, blk),
         "region_ms_incl_l2_flush": region_ms,
         "gpu_launches": launches * a.steps,
         "clocks": clk.summary(),
     }
+    rec = _profile_record("sparse_attn.cu", f"sparse_attn_{w.name}.json", w.name)
+    if rec is not None:
+        # DRAM bytes of one launch from the committed ncu record (the same kernel source)
+        t = rec.get("dram_bytes_per_launch_full_workload")
+        result["roofline"]["traffic"] = t
+        result["roofline"]["dram_gbs"] = t / (attn_ms * 1e-3) / 1e9
+        result["roofline"]["dram_frac_8tbs"] = t / (attn_ms * 1e-3) / 8e12
+        if rec.get("l2_hit_rate_pct") is not None:
+            result["roofline"]["l2_hit_rate_pct"] = rec["l2_hit_rate_pct"]
     if not decode:
         # Prefill gathers are served by the L2 (each head's K/V is reused by many queries): the
         # HBM fraction above exceeds 1, so the kernel is also set against a measured L2 gather
         # ceiling of the same access pattern.
-        pk = l2_gather_peak(hs, dev, st)
+        pk, ctas = l2_gather_peak(hs, dev, st)
         result["roofline"]["l2_gather"] = {
             "peak_gbs": pk, "frac": achieved / pk,
-            "probe": "hisa_gather_probe: 16-byte cp.async gathers of hashed 256-byte rows of a 32 MiB "
-                     "L2-resident region into shared memory, 12 warps per SM, 4 stages, no arithmetic"}
+            "probe": f"hisa_gather_probe: 16-byte cp.async gathers of hashed 256-byte rows of a 32 MiB "
+                     f"L2-resident region into shared memory, 4 stages, no arithmetic; best of 8 and 12 "
+                     f"warps per SM ({4 * ctas} here)"}
     if comp:
         result["flat_indexer_ms"] = comp["flat_indexer_ms"]
         result["speedup_vs_flat_indexer"] = comp["flat_indexer_ms"] / idx_ms

@@ -70,7 +70,7 @@ def _load():
         "hisa_flat_topk": [pp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
         "hisa_token_topk_noalloc": [pp, vp, vp, vp, vp, vp, vp, vp, vp],
         "hisa_forward_cached": [pp, vp, vp, vp, vp, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
-        "hisa_gather_probe": [vp, i64, ctypes.c_int32, i64, ctypes.c_uint32, vp, vp],
+        "hisa_gather_probe": [vp, i64, ctypes.c_int32, i64, ctypes.c_uint32, vp, ctypes.c_int32, vp],
         "hisa_block_candidates_workspace_size": [pp, sz],
         "hisa_block_candidates": [pp, i64, i64, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
         "hisa_topk_merge": [vp, vp, ctypes.c_int32, i64, ctypes.c_int32, ctypes.c_int32, vp, vp, vp],
@@ -278,12 +278,12 @@ def hisa_lse_merge(o_parts, lse_parts, o, lse=None, stream=None):
                                                  _stream(stream)))
 
 
-def hisa_gather_probe(rows, row_bytes, n_gathers, sink, seed=1, stream=None):
+def hisa_gather_probe(rows, row_bytes, n_gathers, sink, seed=1, ctas_per_sm=0, stream=None):
     """Measurement helper: n_gathers copies of hashed rows of `rows` into shared memory, the
     attention kernel's gather pattern without its arithmetic (see include/hisa.h)."""
     n_rows = rows.numel() * rows.element_size() // row_bytes
     _check("hisa_gather_probe", _lib.hisa_gather_probe(_ptr(rows), n_rows, row_bytes, n_gathers, seed, _ptr(sink),
-                                                       _stream(stream)))
+                                                       ctas_per_sm, _stream(stream)))
 
 
 def hisa_version() -> str:

@@ -446,11 +446,13 @@ hisa_status_t hisa_lse_merge(const void* o_parts, const float* lse_parts, int32_
 }
 
 hisa_status_t hisa_gather_probe(const void* rows, int64_t n_rows, int32_t row_bytes, int64_t n_gathers, uint32_t seed,
-                                uint32_t* sink, cudaStream_t stream) {
+                                uint32_t* sink, int32_t ctas_per_sm, cudaStream_t stream) {
   if (!rows || !sink || n_rows < 1 || n_rows > 0x7FFFFFFFLL || n_gathers < 0) return HISA_ERR_INVALID_ARG;
+  if (ctas_per_sm < 0 || ctas_per_sm > 3) return HISA_ERR_INVALID_ARG;
   if (!hisa::gather_probe_row_bytes_ok(row_bytes) || !hisa::aligned16(rows)) return HISA_ERR_INVALID_ARG;
   if (n_gathers == 0) return HISA_OK;
-  return hisa::cuda_fail(hisa::launch_gather_probe(rows, n_rows, row_bytes, n_gathers, seed, sink, stream));
+  return hisa::cuda_fail(hisa::launch_gather_probe(rows, n_rows, row_bytes, n_gathers, seed, sink,
+                                                     ctas_per_sm ? ctas_per_sm : 3, stream));
 }
 
 }  // extern "C"

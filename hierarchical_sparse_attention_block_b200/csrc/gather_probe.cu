@@ -6,7 +6,7 @@
 //
 // Every warp walks tiles of kRows gathers, copies the rows into its own ring
 // of kStages shared-memory stages and keeps kStages - 1 tiles in flight; 4
-// warps per CTA and 64 KB of shared memory per CTA, three CTAs per SM.  The
+// warps per CTA and 64 KB of shared memory per CTA, one to three CTAs per SM.  The
 // row of gather e is the top bits of a multiplicative hash of e (over the
 // largest power of two of rows the buffer holds), computed in registers, so
 // no index read or division stands between two copies.
@@ -53,13 +53,13 @@ __global__ void __launch_bounds__(kWarps * 32) gather_probe_kernel(const uint8_t
 
 template <int CHUNKS>
 cudaError_t launch_chunks(const void* rows, int row_shift, int64_t n_gathers, uint32_t seed, uint32_t* sink,
-                          cudaStream_t st) {
+                          int ctas_per_sm, cudaStream_t st) {
   auto kern = gather_probe_kernel<CHUNKS>;
   cudaError_t e = ensure_smem((const void*)kern, kSmem);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  kern<<<(unsigned)(3 * sms), kWarps * 32, kSmem, st>>>(static_cast<const uint8_t*>(rows), row_shift, n_gathers, seed,
+  kern<<<(unsigned)(ctas_per_sm * sms), kWarps * 32, kSmem, st>>>(static_cast<const uint8_t*>(rows), row_shift, n_gathers, seed,
                                                         sink);
   return cudaGetLastError();
 }
@@ -67,16 +67,16 @@ cudaError_t launch_chunks(const void* rows, int row_shift, int64_t n_gathers, ui
 }  // namespace
 
 cudaError_t launch_gather_probe(const void* rows, int64_t n_rows, int row_bytes, int64_t n_gathers, uint32_t seed,
-                                uint32_t* sink, cudaStream_t st) {
+                                uint32_t* sink, int ctas_per_sm, cudaStream_t st) {
   int bits = 0;  // rows used: the largest power of two <= n_rows
   while (bits < 31 && ((int64_t)2 << bits) <= n_rows) ++bits;
   const int shift = 32 - bits;  // 32 (one row) leaves row 0
   switch (row_bytes / 16) {
-    case 16: return launch_chunks<16>(rows, shift, n_gathers, seed, sink, st);
-    case 8: return launch_chunks<8>(rows, shift, n_gathers, seed, sink, st);
-    case 4: return launch_chunks<4>(rows, shift, n_gathers, seed, sink, st);
-    case 2: return launch_chunks<2>(rows, shift, n_gathers, seed, sink, st);
-    default: return launch_chunks<1>(rows, shift, n_gathers, seed, sink, st);
+    case 16: return launch_chunks<16>(rows, shift, n_gathers, seed, sink, ctas_per_sm, st);
+    case 8: return launch_chunks<8>(rows, shift, n_gathers, seed, sink, ctas_per_sm, st);
+    case 4: return launch_chunks<4>(rows, shift, n_gathers, seed, sink, ctas_per_sm, st);
+    case 2: return launch_chunks<2>(rows, shift, n_gathers, seed, sink, ctas_per_sm, st);
+    default: return launch_chunks<1>(rows, shift, n_gathers, seed, sink, ctas_per_sm, st);
   }
 }
 

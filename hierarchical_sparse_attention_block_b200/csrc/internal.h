@@ -84,7 +84,7 @@ cudaError_t launch_lse_merge(const void* o_parts, const float* lse_parts, int G,
 // Measurement helper: gathers of hashed rows into shared memory (see hisa_gather_probe).
 bool gather_probe_row_bytes_ok(int row_bytes);
 cudaError_t launch_gather_probe(const void* rows, int64_t n_rows, int row_bytes, int64_t n_gathers, uint32_t seed,
-                                uint32_t* sink, cudaStream_t st);
+                                uint32_t* sink, int ctas_per_sm, cudaStream_t st);
 
 // cudaError_t value behind the last HISA_ERR_CUDA on this host thread.
 extern thread_local int32_t g_last_cuda_error;

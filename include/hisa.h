@@ -262,10 +262,11 @@ hisa_status_t hisa_lse_merge(const void* o_parts, const float* lse_parts, int32_
  * measured ceiling for rows the L2 serves.  rows: device, [n_rows][row_bytes],
  * 16-byte aligned, n_rows < 2^31; row_bytes a multiple of 16, at most 256,
  * with 32 / (row_bytes / 16) integral; sink: one device word the kernel adds a
- * copied word to, so the copies cannot be optimised away.  Returns
- * HISA_ERR_INVALID_ARG for bad arguments; asynchronous on stream. */
+ * copied word to, so the copies cannot be optimised away; ctas_per_sm: CTAs
+ * of 4 warps launched per SM, 1..3 (64 KB of shared memory each), 0 = 3.
+ * Returns HISA_ERR_INVALID_ARG for bad arguments; asynchronous on stream. */
 hisa_status_t hisa_gather_probe(const void* rows, int64_t n_rows, int32_t row_bytes, int64_t n_gathers,
-                                uint32_t seed, uint32_t* sink, cudaStream_t stream);
+                                uint32_t seed, uint32_t* sink, int32_t ctas_per_sm, cudaStream_t stream);
 
 /* Static text for a status code. */
 const char* hisa_status_string(hisa_status_t status);

@@ -138,3 +138,27 @@ def test_workspace_sizes_follow_the_shapes():
     assert hs.hisa_sparse_attn_workspace_size(p) > 0
     big = hs.params(1, 65536, 65536, 128, 128, 64, 2048, 16, 16, 128)
     assert hs.hisa_sparse_attn_workspace_size(big) == 0
+
+
+def test_gather_probe_validation():
+    """The measurement probe rejects bad arguments on the host: null or misaligned rows, row
+    sizes that are not 16..256 bytes in whole 16-byte chunks dividing a warp, and launch shapes
+    outside 0..3 CTAs per SM; zero gathers launch nothing."""
+    lib = hs.lib()
+    a = ctypes.c_void_p(4096)
+    ok = dict(n_rows=1024, row_bytes=256, n=64, seed=1, ctas=0)
+
+    def call(rows=a, sink=a, **kw):
+        k = {**ok, **kw}
+        return lib.hisa_gather_probe(rows, k["n_rows"], k["row_bytes"], k["n"], k["seed"], sink, k["ctas"], None)
+
+    assert call(rows=None) == hs.HISA_ERR_INVALID_ARG
+    assert call(sink=None) == hs.HISA_ERR_INVALID_ARG
+    assert call(rows=ctypes.c_void_p(4104)) == hs.HISA_ERR_INVALID_ARG
+    for rb in (0, 8, 24, 48, 272, 512):
+        assert call(row_bytes=rb) == hs.HISA_ERR_INVALID_ARG, rb
+    for c in (-1, 4):
+        assert call(ctas=c) == hs.HISA_ERR_INVALID_ARG, c
+    assert call(n_rows=0) == hs.HISA_ERR_INVALID_ARG
+    assert call(n=-1) == hs.HISA_ERR_INVALID_ARG
+    assert call(n=0) == hs.HISA_OK
