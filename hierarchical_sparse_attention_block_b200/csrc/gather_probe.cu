@@ -26,6 +26,7 @@ __global__ void __launch_bounds__(kWarps * 32) gather_probe_kernel(const uint8_t
                                                                    uint32_t* __restrict__ sink) {
   constexpr int kRowBytes = CHUNKS * 16;
   constexpr int kPerStep = 32 / CHUNKS;  // rows one warp instruction moves
+  static_assert(kPerStep <= kRows && kRows % kPerStep == 0, "a copy step stays inside its tile");
   extern __shared__ __align__(128) uint8_t smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int r_lane = lane / CHUNKS, c_lane = lane % CHUNKS;
@@ -76,12 +77,13 @@ cudaError_t launch_gather_probe(const void* rows, int64_t n_rows, int row_bytes,
     case 8: return launch_chunks<8>(rows, shift, n_gathers, seed, sink, ctas_per_sm, st);
     case 4: return launch_chunks<4>(rows, shift, n_gathers, seed, sink, ctas_per_sm, st);
     case 2: return launch_chunks<2>(rows, shift, n_gathers, seed, sink, ctas_per_sm, st);
-    default: return launch_chunks<1>(rows, shift, n_gathers, seed, sink, ctas_per_sm, st);
+    default: return cudaErrorInvalidValue;
   }
 }
 
+// One warp instruction moves 32 / (row_bytes / 16) rows, at most a tile (kRows): rows of 32 to 256 bytes.
 bool gather_probe_row_bytes_ok(int row_bytes) {
-  return row_bytes >= 16 && row_bytes <= kMaxRowBytes && row_bytes % 16 == 0 && 32 % (row_bytes / 16) == 0;
+  return row_bytes >= 32 && row_bytes <= kMaxRowBytes && row_bytes % 16 == 0 && 32 % (row_bytes / 16) == 0;
 }
 
 }  // namespace hisa

@@ -260,8 +260,7 @@ hisa_status_t hisa_lse_merge(const void* o_parts, const float* lse_parts, int32_
  * 16-byte cp.async, the copy pattern of sparse_attn_fwd's gathers without any
  * of its arithmetic or index reads, so that timing it gives that kernel a
  * measured ceiling for rows the L2 serves.  rows: device, [n_rows][row_bytes],
- * 16-byte aligned, n_rows < 2^31; row_bytes a multiple of 16, at most 256,
- * with 32 / (row_bytes / 16) integral; sink: one device word the kernel adds a
+ * 16-byte aligned, n_rows < 2^31; row_bytes 32, 64, 128 or 256; sink: one device word the kernel adds a
  * copied word to, so the copies cannot be optimised away; ctas_per_sm: CTAs
  * of 4 warps launched per SM, 1..3 (64 KB of shared memory each), 0 = 3.
  * Returns HISA_ERR_INVALID_ARG for bad arguments; asynchronous on stream. */

@@ -142,7 +142,7 @@ def test_workspace_sizes_follow_the_shapes():
 
 def test_gather_probe_validation():
     """The measurement probe rejects bad arguments on the host: null or misaligned rows, row
-    sizes that are not 16..256 bytes in whole 16-byte chunks dividing a warp, and launch shapes
+    sizes other than 32, 64, 128 and 256 bytes, and launch shapes
     outside 0..3 CTAs per SM; zero gathers launch nothing."""
     lib = hs.lib()
     a = ctypes.c_void_p(4096)
@@ -155,7 +155,7 @@ def test_gather_probe_validation():
     assert call(rows=None) == hs.HISA_ERR_INVALID_ARG
     assert call(sink=None) == hs.HISA_ERR_INVALID_ARG
     assert call(rows=ctypes.c_void_p(4104)) == hs.HISA_ERR_INVALID_ARG
-    for rb in (0, 8, 24, 48, 272, 512):
+    for rb in (0, 8, 16, 24, 48, 96, 272, 512):
         assert call(row_bytes=rb) == hs.HISA_ERR_INVALID_ARG, rb
     for c in (-1, 4):
         assert call(ctas=c) == hs.HISA_ERR_INVALID_ARG, c

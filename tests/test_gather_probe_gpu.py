@@ -6,7 +6,7 @@ torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("row_bytes", [16, 64, 256])
+@pytest.mark.parametrize("row_bytes", [32, 64, 128, 256])
 @pytest.mark.parametrize("ctas", [1, 2, 3])
 def test_gather_probe_copies_rows(row_bytes, ctas):
     if not torch.cuda.is_available():
