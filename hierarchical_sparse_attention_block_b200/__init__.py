@@ -25,7 +25,7 @@ EXPORTS = (
     "hisa_forward", "hisa_flat_topk_workspace_size", "hisa_flat_topk", "hisa_status_string",
     "hisa_last_cuda_error", "hisa_version", "hisa_token_topk_noalloc", "hisa_forward_cached", "hisa_gather_probe",
     "hisa_block_candidates_workspace_size", "hisa_block_candidates", "hisa_topk_merge", "hisa_remap_ids",
-    "hisa_lse_merge",
+    "hisa_lse_merge", "hisa_forward_host_workspace_size", "hisa_forward_host",
 )
 
 
@@ -70,6 +70,8 @@ def _load():
         "hisa_flat_topk": [pp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
         "hisa_token_topk_noalloc": [pp, vp, vp, vp, vp, vp, vp, vp, vp],
         "hisa_forward_cached": [pp, vp, vp, vp, vp, i64, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
+        "hisa_forward_host_workspace_size": [pp, sz],
+        "hisa_forward_host": [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp, vp],
         "hisa_gather_probe": [vp, i64, ctypes.c_int32, i64, ctypes.c_uint32, vp, ctypes.c_int32, vp],
         "hisa_block_candidates_workspace_size": [pp, sz],
         "hisa_block_candidates": [pp, i64, i64, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp],
@@ -214,6 +216,26 @@ def hisa_forward_cached(p, q_idx, k_idx, block_keys, refresh_begin, q, k, v, o, 
                                     _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(block_idx_out),
                                     _ptr(token_idx_out), _ptr(dev_status), _ptr(workspace), workspace.numel(),
                                     _stream(stream)))
+
+
+def hisa_forward_host_workspace_size(p):
+    return _size(_lib.hisa_forward_host_workspace_size, p)
+
+
+def hisa_forward_host(p, q_idx, k_idx, q, k, v, o, lse=None, dev_status=None, workspace=None, stream=None,
+                      copy_stream=None, idx_weights=None):
+    """Steps 1-6 with host inputs and outputs (CPU tensors, pinned for asynchronous copies) and a
+    device workspace; the copies overlap the work when copy_stream is given (see include/hisa.h).
+    Returns when the work is enqueued on stream."""
+    import torch
+
+    if workspace is None:
+        workspace = _workspace(hisa_forward_host_workspace_size(p), torch.device("cuda", torch.cuda.current_device()))
+    cs = ctypes.c_void_p(copy_stream.cuda_stream) if copy_stream is not None else None
+    _check("hisa_forward_host",
+           _lib.hisa_forward_host(ctypes.byref(p), _ptr(q_idx), _ptr(idx_weights), _ptr(k_idx), _ptr(q), _ptr(k),
+                                  _ptr(v), _ptr(o), _ptr(lse), _ptr(dev_status), _ptr(workspace), workspace.numel(),
+                                  _stream(stream), cs))
 
 
 def hisa_flat_topk_workspace_size(p):

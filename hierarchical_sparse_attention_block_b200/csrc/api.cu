@@ -4,7 +4,9 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <mutex>
+#include <vector>
 
 #include "hisa.h"
 #include "internal.h"
@@ -361,6 +363,230 @@ hisa_status_t hisa_forward_cached(const hisa_params_t* params, const void* q_idx
   if (!workspace || !hisa::aligned16(workspace) || workspace_bytes < L.total) return HISA_ERR_WORKSPACE;
   return forward_impl(s, L, q_idx, k_idx, block_keys, refresh_begin, q, k, v, o, lse, block_idx_out, token_idx_out,
                       dev_status, static_cast<uint8_t*>(workspace), workspace_bytes, stream);
+}
+
+namespace {
+// hisa_forward_host: the queries are taken in units whose attention can start as soon as the
+// unit's rows are on the device.  A long sequence (n_q > kHostChunk) is cut into query chunks of
+// at least kHostChunk queries, at most kHostMaxChunks per sequence: chunk [i0, i1) needs the K/V
+// rows [0, n_kv - n_q + i1) only, so each chunk copies just the rows the earlier ones did not.
+// Short sequences (decode) go in up to kHostGroups groups of whole sequences.
+constexpr int64_t kHostChunk = 8192;
+constexpr int64_t kHostMaxChunks = 16;
+constexpr int kHostGroups = 8;
+
+struct HostUnit {
+  int s0, s1;      // sequences [s0, s1)
+  int64_t i0, i1;  // queries [i0, i1) of each of them
+  int64_t kv0;     // first K/V row of the sequence this unit copies (query chunks only)
+};
+
+std::vector<HostUnit> host_units(const Shape& s) {
+  std::vector<HostUnit> u;
+  if (s.n_q > kHostChunk) {
+    const int64_t len = std::max(kHostChunk, (s.n_q + kHostMaxChunks - 1) / kHostMaxChunks);
+    for (int seq = 0; seq < s.batch; ++seq)
+      for (int64_t i0 = 0; i0 < s.n_q; i0 += len)
+        u.push_back({seq, seq + 1, i0, std::min(i0 + len, s.n_q), i0 == 0 ? 0 : s.n_kv - s.n_q + i0});
+  } else {
+    const int g = std::min(s.batch, kHostGroups);
+    for (int j = 0; j < g; ++j) u.push_back({s.batch * j / g, s.batch * (j + 1) / g, 0, s.n_q, 0});
+  }
+  return u;
+}
+
+// The attention problem of a unit: its sequences and queries, positions as in the full problem
+// (p = n_kv - n_q + i), keys the prefix [0, n_kv - n_q + i1) of each sequence.  A query chunk is
+// one sequence, so the shorter key range changes no stride.
+Shape unit_shape(const Shape& s, const HostUnit& u) {
+  Shape c = s;
+  c.batch = u.s1 - u.s0;
+  c.n_q = u.i1 - u.i0;
+  if (u.i0 > 0 || u.i1 < s.n_q) c.n_kv = s.n_kv - s.n_q + u.i1;
+  c.n_query = (int64_t)c.batch * c.n_q;
+  c.n_blk = (c.n_kv + s.B - 1) / s.B;
+  return c;
+}
+
+struct HostFwdLayout {
+  FwdLayout f;
+  size_t part, q_idx, w, k_idx, q, k, v, o, lse, total;
+};
+
+HostFwdLayout host_fwd_layout(const Shape& s) {
+  HostFwdLayout L;
+  L.f = fwd_layout(s);
+  size_t part = 0;
+  for (const HostUnit& u : host_units(s)) {
+    const Shape c = unit_shape(s, u);
+    part = std::max(part, hisa::attn_partial_bytes(c, hisa::attn_pick_splits(c)));
+  }
+  size_t off = L.f.total;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += hisa::align_up(bytes);
+    return at;
+  };
+  const int64_t he = s.HI > 0 ? s.HI : 1;
+  L.part = take(part);
+  L.q_idx = take((size_t)s.n_query * he * s.d_idx * 2);
+  L.w = take(s.HI > 0 ? (size_t)s.n_query * s.HI * sizeof(float) : 0);
+  L.k_idx = take((size_t)s.batch * s.n_kv * s.d_idx * 2);
+  L.q = take((size_t)s.n_query * s.H * s.d * 2);
+  L.k = take((size_t)s.batch * s.n_kv * s.Hkv * s.d * 2);
+  L.v = take((size_t)s.batch * s.n_kv * s.Hkv * s.d * 2);
+  L.o = take((size_t)s.n_query * s.H * s.d * 2);
+  L.lse = take((size_t)s.n_query * s.H * sizeof(float));
+  L.total = off;
+  return L;
+}
+
+bool is_device_memory(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    (void)cudaGetLastError();  // an unknown host pointer: not device memory
+    return false;
+  }
+  return a.type == cudaMemoryTypeDevice;
+}
+
+// Events of one call, destroyed when it returns (a pending event is released once it completes).
+struct EventSet {
+  std::vector<cudaEvent_t> ev;
+  cudaError_t make(cudaEvent_t* e) {
+    const cudaError_t r = cudaEventCreateWithFlags(e, cudaEventDisableTiming);
+    if (r == cudaSuccess) ev.push_back(*e);
+    return r;
+  }
+  ~EventSet() {
+    for (cudaEvent_t e : ev) cudaEventDestroy(e);
+  }
+};
+}  // namespace
+
+hisa_status_t hisa_forward_host_workspace_size(const hisa_params_t* params, size_t* bytes) {
+  Shape s;
+  hisa_status_t rc = hisa::make_shape(params, true, true, &s);
+  if (rc != HISA_OK) return rc;
+  if (!bytes) return HISA_ERR_INVALID_ARG;
+  *bytes = host_fwd_layout(s).total;
+  return HISA_OK;
+}
+
+hisa_status_t hisa_forward_host(const hisa_params_t* params, const void* q_idx, const float* idx_weights,
+                                const void* k_idx, const void* q, const void* k, const void* v, void* o, float* lse,
+                                int32_t* dev_status, void* workspace, size_t workspace_bytes, cudaStream_t stream,
+                                cudaStream_t copy_stream) {
+  Shape s;
+  hisa_status_t rc = hisa::make_shape(params, true, true, &s);
+  if (rc != HISA_OK) return rc;
+  if ((s.HI == 0) != (idx_weights == nullptr)) return HISA_ERR_INVALID_ARG;
+  if (!q_idx || !k_idx || !q || !k || !v || !o) return HISA_ERR_INVALID_ARG;
+  const HostFwdLayout L = host_fwd_layout(s);
+  if (!workspace || !hisa::aligned16(workspace) || workspace_bytes < L.total) return HISA_ERR_WORKSPACE;
+  const void* host_ptrs[] = {q_idx, idx_weights, k_idx, q, k, v, o, lse};
+  for (const void* p : host_ptrs)
+    if (p && is_device_memory(p)) return HISA_ERR_INVALID_ARG;
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* d_q_idx = ws + L.q_idx;
+  float* d_w = s.HI > 0 ? reinterpret_cast<float*>(ws + L.w) : nullptr;
+  uint8_t* d_k_idx = ws + L.k_idx;
+  uint8_t* d_q = ws + L.q;
+  uint8_t* d_k = ws + L.k;
+  uint8_t* d_v = ws + L.v;
+  uint8_t* d_o = ws + L.o;
+  float* d_lse = reinterpret_cast<float*>(ws + L.lse);
+  float* bk = reinterpret_cast<float*>(ws + L.f.bk);
+  int32_t* blk = reinterpret_cast<int32_t*>(ws + L.f.block_idx);
+  int32_t* tok = reinterpret_cast<int32_t*>(ws + L.f.token_idx);
+  rc = hisa::set_idx_weights(&s, d_w);
+  if (rc != HISA_OK) return rc;
+
+  const bool overlap = copy_stream != nullptr && copy_stream != stream;
+  cudaStream_t cs = overlap ? copy_stream : stream;
+  EventSet events;
+  cudaError_t e = cudaSuccess;
+  auto ok = [&](cudaError_t r) {
+    if (e == cudaSuccess) e = r;
+    return e == cudaSuccess;
+  };
+  // the copy stream starts after the caller's earlier work on stream (which may use the workspace)
+  if (overlap) {
+    cudaEvent_t start;
+    if (!ok(events.make(&start)) || !ok(cudaEventRecord(start, stream)) || !ok(cudaStreamWaitEvent(cs, start, 0)))
+      return hisa::cuda_fail(e);
+  }
+
+  // Indexer inputs first, then steps 1-5 on stream while the attention inputs stream in.
+  const int64_t he = s.HI > 0 ? s.HI : 1;
+  const size_t qrow = (size_t)s.H * s.d * 2, kvrow = (size_t)s.Hkv * s.d * 2;
+  ok(cudaMemcpyAsync(d_q_idx, q_idx, (size_t)s.n_query * he * s.d_idx * 2, cudaMemcpyHostToDevice, stream));
+  if (d_w) ok(cudaMemcpyAsync(d_w, idx_weights, (size_t)s.n_query * s.HI * sizeof(float), cudaMemcpyHostToDevice,
+                              stream));
+  ok(cudaMemcpyAsync(d_k_idx, k_idx, (size_t)s.batch * s.n_kv * s.d_idx * 2, cudaMemcpyHostToDevice, stream));
+  if (e != cudaSuccess) return hisa::cuda_fail(e);
+  if (!ok(hisa::launch_block_pool(s, d_k_idx, 0, s.n_blk, bk, stream))) return hisa::cuda_fail(e);
+  rc = hisa::run_block_stage(s, d_q_idx, bk, blk, nullptr, dev_status, ws + L.f.blk_stage, stream);
+  if (rc != HISA_OK) return rc;
+  rc = hisa::run_token_stage(s, d_q_idx, d_k_idx, blk, s.m, tok, nullptr, dev_status, ws + L.f.keys,
+                             L.f.total - L.f.keys, stream);
+  if (rc != HISA_OK) return rc;
+
+  const std::vector<HostUnit> units = host_units(s);
+  std::vector<cudaEvent_t> in(units.size()), done(units.size());
+  auto h2d = [&](uint8_t* dst, const void* src, size_t off, size_t bytes) {
+    return ok(cudaMemcpyAsync(dst + off, static_cast<const uint8_t*>(src) + off, bytes, cudaMemcpyHostToDevice, cs));
+  };
+  for (size_t j = 0; j < units.size() && e == cudaSuccess; ++j) {
+    const HostUnit& u = units[j];
+    const Shape c = unit_shape(s, u);
+    // K/V rows [kv0, c.n_kv) of each of the unit's sequences; its Q rows
+    for (int seq = u.s0; seq < u.s1; ++seq) {
+      const size_t off = ((size_t)seq * s.n_kv + u.kv0) * kvrow, bytes = (size_t)(c.n_kv - u.kv0) * kvrow;
+      h2d(d_k, k, off, bytes);
+      h2d(d_v, v, off, bytes);
+    }
+    if (u.i0 == 0 && u.i1 == s.n_q)
+      h2d(d_q, q, (size_t)u.s0 * s.n_q * qrow, (size_t)(u.s1 - u.s0) * s.n_q * qrow);
+    else
+      h2d(d_q, q, ((size_t)u.s0 * s.n_q + u.i0) * qrow, (size_t)(u.i1 - u.i0) * qrow);
+    if (overlap && ok(events.make(&in[j]))) ok(cudaEventRecord(in[j], cs));
+  }
+  if (e != cudaSuccess) return hisa::cuda_fail(e);
+
+  // Step 6 per unit, as soon as its rows are in.
+  for (size_t j = 0; j < units.size(); ++j) {
+    const HostUnit& u = units[j];
+    const Shape c = unit_shape(s, u);
+    if (overlap && !ok(cudaStreamWaitEvent(stream, in[j], 0))) return hisa::cuda_fail(e);
+    const size_t q0 = (size_t)u.s0 * s.n_q + u.i0;  // first query row of the unit
+    const size_t kv_off = (size_t)u.s0 * s.n_kv * kvrow;
+    const int splits = hisa::attn_pick_splits(c);
+    if (!ok(hisa::launch_sparse_attn(c, d_q + q0 * qrow, d_k + kv_off, d_v + kv_off, tok + q0 * s.k, d_o + q0 * qrow,
+                                     d_lse + q0 * s.H, dev_status, splits, ws + L.part, stream)))
+      return hisa::cuda_fail(e);
+    if (overlap && ok(events.make(&done[j]))) ok(cudaEventRecord(done[j], stream));
+    if (e != cudaSuccess) return hisa::cuda_fail(e);
+  }
+
+  // O and LSE of each unit back to the host once its attention is done.
+  for (size_t j = 0; j < units.size() && e == cudaSuccess; ++j) {
+    const HostUnit& u = units[j];
+    const size_t q0 = (size_t)u.s0 * s.n_q + u.i0;
+    const size_t rows = (size_t)(u.s1 - u.s0) * (u.i1 - u.i0);  // contiguous: several sequences only whole
+    if (overlap) ok(cudaStreamWaitEvent(cs, done[j], 0));
+    ok(cudaMemcpyAsync(static_cast<uint8_t*>(o) + q0 * qrow, d_o + q0 * qrow, rows * qrow, cudaMemcpyDeviceToHost,
+                       cs));
+    if (lse)
+      ok(cudaMemcpyAsync(lse + q0 * s.H, d_lse + q0 * s.H, rows * s.H * sizeof(float), cudaMemcpyDeviceToHost, cs));
+  }
+  // stream's later work sees the copies back complete
+  if (overlap && e == cudaSuccess) {
+    cudaEvent_t end;
+    if (ok(events.make(&end)) && ok(cudaEventRecord(end, cs))) ok(cudaStreamWaitEvent(stream, end, 0));
+  }
+  return hisa::cuda_fail(e);
 }
 
 hisa_status_t hisa_flat_topk_workspace_size(const hisa_params_t* params, size_t* min_bytes, size_t* preferred_bytes) {

@@ -163,6 +163,30 @@ hisa_status_t hisa_forward(const hisa_params_t* params, const void* q_idx, const
                            int32_t* block_idx_out, int32_t* token_idx_out, int32_t* dev_status, void* workspace,
                            size_t workspace_bytes, cudaStream_t stream);
 
+/* Steps 1-6 with the inputs and outputs in HOST memory: q_idx, idx_weights,
+ * k_idx, q, k, v are read from the host and o, lse (nullable) written back
+ * there, in the layouts above.  Pinned host memory (cudaHostAlloc /
+ * cudaHostRegister) lets the copies run asynchronously; pageable memory works
+ * but the copies then stall the calling thread.  The device copies of the
+ * inputs and outputs live in the caller's device workspace
+ * (hisa_forward_host_workspace_size bytes, 16-byte aligned).
+ *
+ * The copies overlap the work: the indexer inputs go first (on stream) and
+ * the indexer runs while copy_stream brings in Q, K and V in query chunks of
+ * each sequence (a chunk of queries [i0, i1) needs the K/V rows up to its last
+ * position only); attention of a chunk starts as soon as its rows have
+ * arrived, and its O/LSE rows go back on copy_stream while the next chunk
+ * runs.  Results equal hisa_forward's on the same inputs.  copy_stream
+ * (nullable, or equal to stream) runs the copies; without one everything is
+ * serialised on stream.  On return the work is enqueued; stream's later work
+ * (and a cudaStreamSynchronize(stream)) sees o and lse complete.  Returns
+ * HISA_ERR_INVALID_ARG when a host argument is device memory. */
+hisa_status_t hisa_forward_host_workspace_size(const hisa_params_t* params, size_t* bytes);
+hisa_status_t hisa_forward_host(const hisa_params_t* params, const void* q_idx, const float* idx_weights,
+                                const void* k_idx, const void* q, const void* k, const void* v, void* o, float* lse,
+                                int32_t* dev_status, void* workspace, size_t workspace_bytes, cudaStream_t stream,
+                                cudaStream_t copy_stream);
+
 /* Steps 1-6 with caller-owned block keys that persist between calls (decode
  * serving, [QB] "HISA的關鍵優勢在於": the KV cache is unchanged, so the pooled
  * block keys of the cache can be kept).  block_keys [b][ceil(n_kv/B)][d_idx]

@@ -162,3 +162,29 @@ def test_gather_probe_validation():
     assert call(n_rows=0) == hs.HISA_ERR_INVALID_ARG
     assert call(n=-1) == hs.HISA_ERR_INVALID_ARG
     assert call(n=0) == hs.HISA_OK
+
+
+def test_forward_host_validation():
+    """hisa_forward_host checks its arguments on the host before any copy: every input and o
+    present, head weights iff n_idx_heads > 0, a 16-byte aligned device workspace of at least
+    hisa_forward_host_workspace_size bytes, which covers hisa_forward's workspace plus device
+    copies of every input and output."""
+    lib = hs.lib()
+    p = _p()
+    a = ctypes.c_void_p(4096)
+    need = hs.hisa_forward_host_workspace_size(p)
+    fwd = hs.hisa_forward_workspace_size(p)
+    io = (p.batch * p.n_q * p.d_idx * 2 + p.batch * p.n_kv * p.d_idx * 2
+          + 2 * p.batch * p.n_q * p.n_heads * p.d_head * 2 + 2 * p.batch * p.n_kv * p.n_kv_heads * p.d_head * 2
+          + p.batch * p.n_q * p.n_heads * 4)
+    assert need >= fwd + io
+
+    def call(qi=a, w=None, ki=a, q=a, k=a, v=a, o=a, ws=a, nbytes=need):
+        return lib.hisa_forward_host(ctypes.byref(p), qi, w, ki, q, k, v, o, None, None, ws, nbytes, None, None)
+
+    for kw in ("qi", "ki", "q", "k", "v", "o"):
+        assert call(**{kw: None}) == hs.HISA_ERR_INVALID_ARG, kw
+    assert call(w=a) == hs.HISA_ERR_INVALID_ARG  # weights without indexer heads
+    assert call(nbytes=need - 1) == hs.HISA_ERR_WORKSPACE
+    assert call(ws=None) == hs.HISA_ERR_WORKSPACE
+    assert call(ws=ctypes.c_void_p(4104)) == hs.HISA_ERR_WORKSPACE
