@@ -212,8 +212,9 @@ def needle_recall(w, block_idx):
 
 def l2_gather_peak(hs, dev, st, row_bytes=256, region_bytes=32 << 20, n_gathers=8 << 20):
     """Measured ceiling of the attention kernel's gathers (GB/s): hisa_gather_probe copying
-    hashed 256-byte rows of a 32 MiB region (one head's K and V at 64K, L2-resident) into shared
-    memory with the kernel's cp.async pattern and nothing else.  The best of 5 event-timed
+    hashed 256-byte rows of a region into shared memory with the kernel's cp.async pattern and
+    nothing else; a 32 MiB region (one head's K and V at 64K) stays in L2, a region of GiBs
+    measures gathers from HBM.  The best of 5 event-timed
     launches at each of 2 and 3 CTAs (8 and 12 warps) per SM; returns (GB/s, CTAs per SM)."""
     import torch
 
@@ -454,6 +455,15 @@ def run_ours(a, rank, world, local_rank):
         result["roofline"]["dram_frac_8tbs"] = t / (attn_ms * 1e-3) / 8e12
         if rec.get("l2_hit_rate_pct") is not None:
             result["roofline"]["l2_hit_rate_pct"] = rec["l2_hit_rate_pct"]
+    if decode:
+        # Decode gathers come from HBM with no reuse: the same probe over a 4 GiB region (far
+        # larger than L2) gives the gather ceiling of random 256-byte rows from DRAM.
+        pk, ctas = l2_gather_peak(hs, dev, st, region_bytes=4 << 30)
+        result["roofline"]["hbm_gather"] = {
+            "peak_gbs": pk, "frac": achieved / pk,
+            "probe": f"hisa_gather_probe: 16-byte cp.async gathers of hashed 256-byte rows of a 4 GiB region "
+                     f"(HBM) into shared memory, 4 stages, no arithmetic; best of 8 and 12 warps per SM "
+                     f"({4 * ctas} here)"}
     if not decode:
         # Prefill gathers are served by the L2 (each head's K/V is reused by many queries): the
         # HBM fraction above exceeds 1, so the kernel is also set against a measured L2 gather
