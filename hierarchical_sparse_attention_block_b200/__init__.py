@@ -226,7 +226,7 @@ def hisa_forward_host(p, q_idx, k_idx, q, k, v, o, lse=None, dev_status=None, wo
                       copy_stream=None, idx_weights=None):
     """Steps 1-6 with host inputs and outputs (CPU tensors, pinned for asynchronous copies) and a
     device workspace; the copies overlap the work when copy_stream is given (see include/hisa.h).
-    Returns when the work is enqueued on stream."""
+    Synchronous: returns when o and lse hold the results."""
     import torch
 
     if workspace is None:

@@ -581,11 +581,13 @@ hisa_status_t hisa_forward_host(const hisa_params_t* params, const void* q_idx, 
     if (lse)
       ok(cudaMemcpyAsync(lse + q0 * s.H, d_lse + q0 * s.H, rows * s.H * sizeof(float), cudaMemcpyDeviceToHost, cs));
   }
-  // stream's later work sees the copies back complete
+  // The outputs are in host memory when the call returns: stream waits for the copies back and
+  // is synchronised (the events of the call are then complete before they are destroyed).
   if (overlap && e == cudaSuccess) {
     cudaEvent_t end;
     if (ok(events.make(&end)) && ok(cudaEventRecord(end, cs))) ok(cudaStreamWaitEvent(stream, end, 0));
   }
+  ok(cudaStreamSynchronize(stream));
   return hisa::cuda_fail(e);
 }
 

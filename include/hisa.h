@@ -22,7 +22,8 @@
  *   6. softmax attention of every head over just those tokens.
  *
  * Conventions shared by every call
- *   - Tensors are dense, row-major, in DEVICE memory, owned by the caller.
+ *   - Tensors are dense, row-major, in DEVICE memory, owned by the caller
+ *     (hisa_forward_host alone takes its inputs and outputs in host memory).
  *     The library allocates nothing; calls that need scratch take a caller
  *     workspace whose size the matching *_workspace_size call reports.
  *   - bf16 tensors are passed as void* (__nv_bfloat16 elements).  Base
@@ -45,15 +46,17 @@
  *                          the query's head weights w_j = idx_weights, the
  *                          multi-head indexer form of DeepSeek-V3.2).
  *     idx_weights must be NULL when n_idx_heads is 0 and non-NULL otherwise.
- *     The tensor-core scorers serve the one-head form; the Hi-head form runs
- *     on CUDA-core scorers.  Integer inputs and integer weights keep it exact
- *     while |scores| * B < 2^24.
+ *     With many queries per sequence both forms are scored on the tensor
+ *     cores (the Hi-head form for Hi in {1, 2, 4, 8, 16}); other Hi and
+ *     decode run on CUDA-core scorers.  Integer inputs and integer weights
+ *     keep every score exact while |scores| * B < 2^24.
  *   - Index lists are ascending with -1 padding at the tail.  Ties in a
  *     selection go to the lower block / token index.
  *   - Every call validates its arguments on the host before launching
  *     anything (HISA_ERR_INVALID_ARG / HISA_ERR_UNSUPPORTED /
  *     HISA_ERR_WORKSPACE) and then only enqueues work on `stream`; results
- *     are ready when the stream reaches them.  A launch failure returns
+ *     are ready when the stream reaches them (hisa_forward_host returns with
+ *     its results in host memory).  A launch failure returns
  *     HISA_ERR_CUDA; hisa_last_cuda_error() gives the cudaError_t value.
  *   - Index lists given as INPUT are checked on the device: an entry that is
  *     out of range (below -1, beyond the query's own block / position, or not
@@ -178,9 +181,9 @@ hisa_status_t hisa_forward(const hisa_params_t* params, const void* q_idx, const
  * arrived, and its O/LSE rows go back on copy_stream while the next chunk
  * runs.  Results equal hisa_forward's on the same inputs.  copy_stream
  * (nullable, or equal to stream) runs the copies; without one everything is
- * serialised on stream.  On return the work is enqueued; stream's later work
- * (and a cudaStreamSynchronize(stream)) sees o and lse complete.  Returns
- * HISA_ERR_INVALID_ARG when a host argument is device memory. */
+ * serialised on stream.  The call is synchronous: it returns when o and lse
+ * are in host memory (it synchronises stream).  Returns HISA_ERR_INVALID_ARG
+ * when a host argument is device memory. */
 hisa_status_t hisa_forward_host_workspace_size(const hisa_params_t* params, size_t* bytes);
 hisa_status_t hisa_forward_host(const hisa_params_t* params, const void* q_idx, const float* idx_weights,
                                 const void* k_idx, const void* q, const void* k, const void* v, void* o, float* lse,
