@@ -4,21 +4,30 @@
 //
 // A kept block is a contiguous B x d_idx tile of k_idx, and 128 consecutive
 // queries keep overlapping sets of blocks.  So instead of gathering rows per
-// query, a CTA takes a tile of 128 queries of one sequence and a run of up to
-// kRun key blocks at or below the tile's causal limit, and for each block j:
-//   * TMA brings K_j (B rows, 128-byte swizzle: the K-major UMMA operand) into
-//     one of 2-3 shared-memory stages (the 128 query rows came once);
-//   * one thread issues d_idx/16 tcgen05.mma (kind::f16, M=128, N=B) writing
-//     all 128 x B scores to TMEM (fp32; exact on integer-valued inputs);
-//   * each warp reads its 32 query rows back (tcgen05.ld) -- only when one of
-//     its queries kept block j -- and writes that query's B order-preserving
-//     keys to its slot of the key buffer (0 for tokens after the query).
-// The slot of block j in each query's kept list comes from a per-CTA map
-// built by scanning the lists once (same acceptance rule as the CUDA-core
-// scorer: in range and above every earlier in-range entry).  The CTA holding
-// the first run also zero-fills unused slots and flags malformed entries.
-// With no list (the flat indexer) slot = block id.  Waits are bounded (1 s);
-// a timeout sets status bit 1.
+// query, a CTA takes a tile of 128 query rows of one sequence and a run of up
+// to kRun key blocks at or below the tile's causal limit, and scores every
+// block of the run against the whole tile with one group of tcgen05.mma
+// (kind::f16, M = 128 rows, N = B, fp32 in TMEM; exact on integer-valued
+// inputs).  The CTA is split by role, the roles handing work over through
+// mbarriers:
+//   * warp 8 (one thread): TMA of the query tile once, then of each key block
+//     (B rows, 128-byte swizzle: the K-major UMMA operand) into a ring of
+//     2-4 shared-memory stages;
+//   * warp 9 (one thread): the MMAs of block b into TMEM accumulator b & 1,
+//     once its stage has landed and that accumulator has been read out;
+//   * warps 0-7, two groups of four (group g reads accumulator g, so the
+//     blocks alternate between the groups): each warp reads its 32 rows back
+//     (tcgen05.ld) -- only when one of its queries kept the block -- and
+//     writes that query's B order-preserving keys to its slot of the key
+//     buffer (0 for tokens after the query).
+// With a multi-head indexer the 128 rows are 128 / H queries x H heads and
+// the readout applies w_j * max(0, .) and sums a query's rows.  The slot of
+// block j in each query's kept list comes from a per-CTA map built by
+// scanning the lists once (same acceptance rule as the CUDA-core scorer: in
+// range and above every earlier in-range entry).  The CTA holding the first
+// run also zero-fills unused slots and flags malformed entries.  With no list
+// (the flat indexer) slot = block id.  Waits are bounded (1 s): a role that
+// gives up sets status bit 1 and an abort flag the other roles poll.
 #include "common.cuh"
 #include "internal.h"
 #include "tc_common.cuh"
@@ -26,23 +35,31 @@
 namespace hisa {
 namespace {
 
-constexpr int kThreads = 128;
+constexpr int kEpiWarps = 8;  // two groups of four, one per TMEM accumulator
+constexpr int kWarpTma = 8, kWarpMma = 9;
+constexpr int kThreads = (kEpiWarps + 2) * 32;
 constexpr int kTileQ = 128;
-constexpr int kRun = 64;      // key blocks per CTA
+constexpr int kRun = 64;  // key blocks per CTA
 
 template <int D, int B>
 struct TsLayout {
   static constexpr int HALVES = D / 64;
   static constexpr int Q_BYTES = HALVES * kTileQ * 128;
   static constexpr int K_BYTES = HALVES * B * 128;
-  static constexpr int STAGES = K_BYTES >= 65536 ? 2 : 3;  // K tiles in flight
+  static constexpr int MAP_BYTES = kTileQ * kRun * 2;  // int16 [kTileQ][kRun]
+  static constexpr int AVAIL = 227 * 1024 - 1024 - Q_BYTES - MAP_BYTES - 256;
+  static constexpr int STAGES = AVAIL / K_BYTES >= 4 ? 4 : AVAIL / K_BYTES;  // K tiles in flight
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = Q_OFF + Q_BYTES;
-  static constexpr int MAP_OFF = K_OFF + STAGES * K_BYTES;  // int16 [kTileQ][kRun]
-  static constexpr int BAR_OFF = MAP_OFF + kTileQ * kRun * 2;
-  static constexpr int NBAR = 3 + STAGES;  // q, MMA done x 2 accumulators, K stages
-  static constexpr int SMEM = BAR_OFF + 8 * NBAR + 16 + 1024;
+  static constexpr int MAP_OFF = K_OFF + STAGES * K_BYTES;
+  static constexpr int BAR_OFF = MAP_OFF + MAP_BYTES;
+  // mbarriers: q full | accumulator full x 2 | accumulator empty x 2 | K full x S | K empty x S
+  static constexpr int B_Q = 0, B_AFULL = 1, B_AEMPTY = 3, B_KFULL = 5, B_KEMPTY = 5 + STAGES;
+  static constexpr int NBAR = 5 + 2 * STAGES;
+  static constexpr int MISC_OFF = BAR_OFF + 8 * NBAR;  // TMEM base, abort flag
+  static constexpr int SMEM = MISC_OFF + 16 + 1024;
   static constexpr uint32_t TMEM_COLS = 2 * B;  // two B-column accumulators
+  static_assert(STAGES >= 2, "two key stages at least");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
   static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(B >> 3) << 17) |
                                     ((uint32_t)(kTileQ >> 4) << 24);
@@ -57,7 +74,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                           int32_t* __restrict__ status, int64_t n_q, int64_t n_kv, int q_tiles, int runs, int64_t q0,
                           int64_t nq, const float* __restrict__ w_idx, int HI) {
   using L = TsLayout<D, B>;
-  constexpr int kKStages = L::STAGES;
+  constexpr int S = L::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
 
@@ -81,220 +98,233 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (jb0 > c_max) return;
   const int nb = (int)min((int64_t)kRun, c_max + 1 - jb0);
 
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint8_t* sQ = smem + L::Q_OFF;
   uint8_t* sK = smem + L::K_OFF;
   int16_t* smap = reinterpret_cast<int16_t*>(smem + L::MAP_OFF);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);  // [0] q, [1..2] mma done, [3..] k stages
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::BAR_OFF + 8 * L::NBAR);
+  const uint32_t bar0 = smem_u32(smem + L::BAR_OFF);
+  auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
+  auto fail = [&]() {
+    *abort_flag = 1;
+    if (status) atomicOr(status, kStatusTimeout);
+  };
 
-  if (warp == 0) {
+  if (warp == kWarpMma) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                  "r"(L::TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   if (tid == 0) {
-    for (int i = 0; i < L::NBAR; ++i)
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars[i])));
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    mbar_init(bar(L::B_Q), 1);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(bar(L::B_AFULL + a), 1);
+      mbar_init(bar(L::B_AEMPTY + a), 4);  // the four warps of group a
+    }
+    for (int st = 0; st < S; ++st) {
+      mbar_init(bar(L::B_KFULL + st), 1);
+      mbar_init(bar(L::B_KEMPTY + st), 1);
+    }
+    *abort_flag = 0;
+    mbar_init_fence();
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = *tmem_slot;
 
-  // Producer: the query tile and the first K stages.
-  if (tid == 0) {
-    const uint32_t bq = smem_u32(&bars[0]);
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bq), "r"((uint32_t)L::Q_BYTES)
-                 : "memory");
-    for (int hh = 0; hh < L::HALVES; ++hh)
-      tma_load_2d(smem_u32(sQ + hh * kTileQ * 128), &tmap_q, hh * 64, (int)(tq0 * HE), bq);
-    for (int s = 0; s < kKStages && s < nb; ++s) {
-      const uint32_t bk = smem_u32(&bars[3 + s]);
-      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bk), "r"((uint32_t)L::K_BYTES)
-                   : "memory");
-      const int krow = (int)(seq * n_kv + (jb0 + s) * B);
+  if (warp == kWarpTma) {
+    // ---------------- producer: the query tile, then the key blocks into the stage ring ----------------
+    if (lane == 0) {
+      mbar_expect_tx(bar(L::B_Q), (uint32_t)L::Q_BYTES);
       for (int hh = 0; hh < L::HALVES; ++hh)
-        tma_load_2d(smem_u32(sK + s * L::K_BYTES + hh * B * 128), &tmap_k, hh * 64, krow, bk);
-    }
-  }
-
-  // Slot map of query tid of the tile (threads tid < QT) for blocks jb0 .. jb0+nb-1.
-  {
-  const int64_t qrow = tq0 + tid;  // global query id
-  const bool row_ok = tid < QT && qrow >= t_lo && qrow < t_hi;
-  const int64_t p = n_kv - n_q + (qrow - seq * n_q);
-  const int64_t c = p / B;
-  uint32_t* krow_keys = keys + (qrow - q0) * (int64_t)slots * B;
-  if (tid < QT)
-    for (int jj = 0; jj < kRun; ++jj) smap[tid * kRun + jj] = -1;
-  if (row_ok) {
-    if (block_idx) {
-      const int32_t* lst = block_idx + qrow * slots;
-      int mx = -1;
-      for (int r = 0; r < slots; ++r) {
-        const int b = lst[r];
-        const bool in_range = b >= 0 && b <= c;
-        const bool ok = in_range && b > mx;
-        if (ok && b >= jb0 && b < jb0 + nb) smap[tid * kRun + (b - jb0)] = (int16_t)r;
-        if (run == 0 && !ok) {
-          if (b != -1 && status) atomicOr(status, kStatusBadIndex);
-          uint4* z = reinterpret_cast<uint4*>(krow_keys + (int64_t)r * B);
-          for (int i = 0; i < B / 4; ++i) z[i] = make_uint4(0, 0, 0, 0);
+        tma_load_2d(smem_u32(sQ + hh * kTileQ * 128), &tmap_q, hh * 64, (int)(tq0 * HE), bar(L::B_Q));
+      int issued = 0;
+      for (int b = 0; b < nb; ++b) {
+        const int st = b % S;
+        if (!mbar_wait_or_abort(bar(L::B_KEMPTY + st), (uint32_t)(((b / S) & 1) ^ 1), abort_flag)) {
+          fail();
+          break;
         }
-        if (in_range) mx = max(mx, b);
+        mbar_expect_tx(bar(L::B_KFULL + st), (uint32_t)L::K_BYTES);
+        const int krow = (int)(seq * n_kv + (jb0 + b) * B);
+        for (int hh = 0; hh < L::HALVES; ++hh)
+          tma_load_2d(smem_u32(sK + st * L::K_BYTES + hh * B * 128), &tmap_k, hh * 64, krow, bar(L::B_KFULL + st));
+        issued = b + 1;
       }
-    } else {
-      for (int jj = 0; jj < nb; ++jj)
-        if (jb0 + jj <= c) smap[tid * kRun + jj] = (int16_t)(jb0 + jj);
-      if (run == 0) {  // blocks after the query's own block hold no candidate
-        for (int64_t r = c + 1; r < slots; ++r) {
-          uint4* z = reinterpret_cast<uint4*>(krow_keys + r * B);
-          for (int i = 0; i < B / 4; ++i) z[i] = make_uint4(0, 0, 0, 0);
+      // copies still in flight land before the CTA exits (all of them have, unless a role gave up)
+      mbar_wait(bar(L::B_Q), 0);
+      for (int b = max(0, issued - S); b < issued; ++b) mbar_wait(bar(L::B_KFULL + b % S), (uint32_t)((b / S) & 1));
+    }
+  } else if (warp == kWarpMma) {
+    // ---------------- MMA issuer: block b into accumulator b & 1 ----------------
+    if (lane == 0) {
+      const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK);
+      bool ok = mbar_wait_or_abort(bar(L::B_Q), 0, abort_flag);
+      int issued = 0;
+      for (int b = 0; b < nb && ok; ++b) {
+        const int st = b % S, a = b & 1;
+        ok = mbar_wait_or_abort(bar(L::B_KFULL + st), (uint32_t)((b / S) & 1), abort_flag) &&
+             mbar_wait_or_abort(bar(L::B_AEMPTY + a), (uint32_t)(((b >> 1) & 1) ^ 1), abort_flag);
+        if (!ok) break;
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint32_t acc_col = tmem + (uint32_t)(a * B);
+#pragma unroll
+        for (int hh = 0; hh < L::HALVES; ++hh) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t ad = desc_kmajor_sw128(q_base + hh * kTileQ * 128 + k * 32);
+            const uint64_t bd = desc_kmajor_sw128(k_base + st * L::K_BYTES + hh * B * 128 + k * 32);
+            umma_bf16(acc_col, ad, bd, L::IDESC, (hh | k) ? 1u : 0u);
+          }
         }
+        umma_commit(bar(L::B_KEMPTY + st));  // the stage may be refilled once these MMAs have read it
+        umma_commit(bar(L::B_AFULL + a));    // and the accumulator read out
+        issued = b + 1;
       }
+      if (!ok) fail();
+      // every MMA issued has completed before the TMEM is released
+      if (issued > 0) mbar_wait(bar(L::B_AFULL + ((issued - 1) & 1)), (uint32_t)(((issued - 1) >> 1) & 1));
     }
-  }
-  }
-
-  // This thread's TMEM lane = tile row tid: query tq0 + tid / HE, indexer head tid % HE.
-  const int qi = tid / HE, head = tid % HE;
-  const int64_t qrow = tq0 + qi;
-  const bool row_ok = qrow >= t_lo && qrow < t_hi;
-  const int64_t p = n_kv - n_q + (qrow - seq * n_q);
-  uint32_t* krow_keys = keys + (qrow - q0) * (int64_t)slots * B;
-  const float wgt = (HI > 0 && row_ok) ? w_idx[qrow * HI + head] : 1.f;
-  __syncthreads();  // the slot maps are complete
-
-  bool ok = mbar_wait(smem_u32(&bars[0]), 0);
-  ok = __syncthreads_and(ok) != 0;
-  const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK);
-  // Thread 0: once block bb's K stage has landed, its scores go to accumulator bb & 1 (B columns).
-  auto issue_mma = [&](int bb) -> bool {
-    const int stage = bb % kKStages;
-    if (!mbar_wait(smem_u32(&bars[3 + stage]), (uint32_t)((bb / kKStages) & 1))) return false;
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    const uint32_t acc_col = tmem + (uint32_t)((bb & 1) * B);
-#pragma unroll
-    for (int hh = 0; hh < L::HALVES; ++hh) {
-#pragma unroll
-      for (int s = 0; s < 4; ++s) {
-        const uint64_t ad = desc_kmajor_sw128(q_base + hh * kTileQ * 128 + s * 32);
-        const uint64_t bd = desc_kmajor_sw128(k_base + stage * L::K_BYTES + hh * B * 128 + s * 32);
-        const uint32_t acc = (hh | s) ? 1u : 0u;
-        asm volatile(
-            "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-            " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(acc_col),
-            "l"(ad), "l"(bd), "r"(L::IDESC), "r"(acc));
-      }
-    }
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                     smem_u32(&bars[1 + (bb & 1)]))
-                 : "memory");
-    return true;
-  };
-  if (ok && tid == 0 && nb > 0 && !issue_mma(0) && status) atomicOr(status, kStatusTimeout);
-  for (int b = 0; b < nb && ok; ++b) {
-    const int stage = b % kKStages;
-    // The next block's scores are computed while this block's are read: its accumulator was last
-    // read in iteration b - 1, which every warp finished before that iteration's closing barrier.
-    if (tid == 0 && b + 1 < nb && !issue_mma(b + 1) && status) atomicOr(status, kStatusTimeout);
-    bool done = mbar_wait(smem_u32(&bars[1 + (b & 1)]), (uint32_t)((b >> 1) & 1));
-    done = __syncthreads_and(done) != 0;
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    if (!done) {
-      ok = false;
-      if (tid == 0 && status) atomicOr(status, kStatusTimeout);
-      break;
-    }
-    // The MMA has consumed this K stage: refill it with block b + kKStages.
-    if (tid == 0 && b + kKStages < nb) {
-      const uint32_t bk = smem_u32(&bars[3 + stage]);
-      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bk), "r"((uint32_t)L::K_BYTES)
-                   : "memory");
-      const int krow = (int)(seq * n_kv + (jb0 + b + kKStages) * B);
-      for (int hh = 0; hh < L::HALVES; ++hh)
-        tma_load_2d(smem_u32(sK + stage * L::K_BYTES + hh * B * 128), &tmap_k, hh * 64, krow, bk);
-    }
-    // Epilogue: rows whose query kept block jb0 + b.
-    const int slot = row_ok ? smap[qi * kRun + b] : -1;
-    if (__any_sync(0xFFFFFFFFu, slot >= 0)) {
-      const int64_t j = jb0 + b;
-      const int64_t tok0 = j * B;
-      uint32_t* dst = krow_keys + (int64_t)(slot < 0 ? 0 : slot) * B;
-#pragma unroll 1
-      for (int cc = 0; cc < B / 32; ++cc) {
-        uint32_t v[32];
-        const uint32_t addr = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)((b & 1) * B + cc * 32);
-        asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-            "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-              "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
-              "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
-              "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]),
-              "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-            : "r"(addr));
-        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-        if (HI == 0) {
-          if (slot >= 0) {
-#pragma unroll
-            for (int t = 0; t < 32; t += 4) {
-              const int64_t tk = tok0 + cc * 32 + t;
-              uint4 w;
-              w.x = tk <= p ? score_key(__uint_as_float(v[t])) : 0u;
-              w.y = tk + 1 <= p ? score_key(__uint_as_float(v[t + 1])) : 0u;
-              w.z = tk + 2 <= p ? score_key(__uint_as_float(v[t + 2])) : 0u;
-              w.w = tk + 3 <= p ? score_key(__uint_as_float(v[t + 3])) : 0u;
-              *reinterpret_cast<uint4*>(dst + cc * 32 + t) = w;
+  } else {
+    // ---------------- readout warps ----------------
+    // Slot map of query tid of the tile (threads tid < QT) for blocks jb0 .. jb0+nb-1.
+    {
+      const int64_t qrow = tq0 + tid;  // global query id
+      const bool row_ok = tid < QT && qrow >= t_lo && qrow < t_hi;
+      const int64_t p = n_kv - n_q + (qrow - seq * n_q);
+      const int64_t c = p / B;
+      uint32_t* krow_keys = keys + (qrow - q0) * (int64_t)slots * B;
+      if (tid < QT)
+        for (int jj = 0; jj < kRun; ++jj) smap[tid * kRun + jj] = -1;
+      if (row_ok) {
+        if (block_idx) {
+          const int32_t* lst = block_idx + qrow * slots;
+          int mx = -1;
+          for (int r = 0; r < slots; ++r) {
+            const int b = lst[r];
+            const bool in_range = b >= 0 && b <= c;
+            const bool ok = in_range && b > mx;
+            if (ok && b >= jb0 && b < jb0 + nb) smap[tid * kRun + (b - jb0)] = (int16_t)r;
+            if (run == 0 && !ok) {
+              if (b != -1 && status) atomicOr(status, kStatusBadIndex);
+              uint4* z = reinterpret_cast<uint4*>(krow_keys + (int64_t)r * B);
+              for (int i = 0; i < B / 4; ++i) z[i] = make_uint4(0, 0, 0, 0);
             }
+            if (in_range) mx = max(mx, b);
           }
         } else {
-          // Multi-head score w_j * max(0, q_j . k) per row, summed over the HE rows of a query
-          // with a transposing reduction: after it, the lane of head h holds the sums of tokens
-          // h * (32 / HE) .. (h + 1) * (32 / HE) - 1 of this chunk.
-          float x[32];
+          for (int jj = 0; jj < nb; ++jj)
+            if (jb0 + jj <= c) smap[tid * kRun + jj] = (int16_t)(jb0 + jj);
+          if (run == 0) {  // blocks after the query's own block hold no candidate
+            for (int64_t r = c + 1; r < slots; ++r) {
+              uint4* z = reinterpret_cast<uint4*>(krow_keys + r * B);
+              for (int i = 0; i < B / 4; ++i) z[i] = make_uint4(0, 0, 0, 0);
+            }
+          }
+        }
+      }
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");  // the slot maps are complete
+
+    // This thread's TMEM lane = tile row r: query tq0 + r / HE, indexer head r % HE.
+    const int g = warp >> 2, quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int qi = r / HE, head = r % HE;
+    const int64_t qrow = tq0 + qi;
+    const bool row_ok = qrow >= t_lo && qrow < t_hi;
+    const int64_t p = n_kv - n_q + (qrow - seq * n_q);
+    uint32_t* krow_keys = keys + (qrow - q0) * (int64_t)slots * B;
+    const float wgt = (HI > 0 && row_ok) ? w_idx[qrow * HI + head] : 1.f;
+    for (int b = g; b < nb; b += 2) {
+      // the warp leaves together (the shuffles and TMEM loads below are warp-wide)
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait_or_abort(bar(L::B_AFULL + g), (uint32_t)((b >> 1) & 1), abort_flag))) {
+        if (lane == 0) fail();
+        break;
+      }
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      // rows whose query kept block jb0 + b
+      const int slot = row_ok ? smap[qi * kRun + b] : -1;
+      if (__any_sync(0xFFFFFFFFu, slot >= 0)) {
+        const int64_t j = jb0 + b;
+        const int64_t tok0 = j * B;
+        uint32_t* dst = krow_keys + (int64_t)(slot < 0 ? 0 : slot) * B;
+#pragma unroll 1
+        for (int cc = 0; cc < B / 32; ++cc) {
+          uint32_t v[32];
+          const uint32_t addr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(g * B + cc * 32);
+          asm volatile(
+              "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+              "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+              : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+                "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
+                "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
+                "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]),
+                "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+              : "r"(addr));
+          asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+          if (HI == 0) {
+            if (slot >= 0) {
 #pragma unroll
-          for (int t = 0; t < 32; ++t) x[t] = wgt * fmaxf(__uint_as_float(v[t]), 0.f);
+              for (int t = 0; t < 32; t += 4) {
+                const int64_t tk = tok0 + cc * 32 + t;
+                uint4 w;
+                w.x = tk <= p ? score_key(__uint_as_float(v[t])) : 0u;
+                w.y = tk + 1 <= p ? score_key(__uint_as_float(v[t + 1])) : 0u;
+                w.z = tk + 2 <= p ? score_key(__uint_as_float(v[t + 2])) : 0u;
+                w.w = tk + 3 <= p ? score_key(__uint_as_float(v[t + 3])) : 0u;
+                *reinterpret_cast<uint4*>(dst + cc * 32 + t) = w;
+              }
+            }
+          } else {
+            // Multi-head score w_j * max(0, q_j . k) per row, summed over the HE rows of a query
+            // with a transposing reduction: after it, the lane of head h holds the sums of tokens
+            // h * (32 / HE) .. (h + 1) * (32 / HE) - 1 of this chunk.
+            float x[32];
 #pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            if ((1 << m) < HE) {  // warp-uniform
-              constexpr int kHalfMax = 16;
-              const int half = 16 >> m;
-              const int o = HE >> (m + 1);
-              const bool up = (head & o) != 0;
+            for (int t = 0; t < 32; ++t) x[t] = wgt * fmaxf(__uint_as_float(v[t]), 0.f);
 #pragma unroll
-              for (int t = 0; t < kHalfMax; ++t) {
-                if (t < half) {
-                  const float send = up ? x[t] : x[t + half];
-                  const float keep = up ? x[t + half] : x[t];
-                  x[t] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, o);
+            for (int m = 0; m < 4; ++m) {
+              if ((1 << m) < HE) {  // warp-uniform
+                constexpr int kHalfMax = 16;
+                const int half = 16 >> m;
+                const int o = HE >> (m + 1);
+                const bool up = (head & o) != 0;
+#pragma unroll
+                for (int t = 0; t < kHalfMax; ++t) {
+                  if (t < half) {
+                    const float send = up ? x[t] : x[t + half];
+                    const float keep = up ? x[t + half] : x[t];
+                    x[t] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, o);
+                  }
+                }
+              }
+            }
+            if (slot >= 0) {
+              const int n = 32 / HE, t0 = head * n;
+#pragma unroll
+              for (int t = 0; t < 32; ++t) {
+                if (t < n) {
+                  const int64_t tk = tok0 + cc * 32 + t0 + t;
+                  dst[cc * 32 + t0 + t] = tk <= p ? score_key(x[t]) : 0u;
                 }
               }
             }
           }
-          if (slot >= 0) {
-            const int n = 32 / HE, t0 = head * n;
-#pragma unroll
-            for (int t = 0; t < 32; ++t) {
-              if (t < n) {
-                const int64_t tk = tok0 + cc * 32 + t0 + t;
-                dst[cc * 32 + t0 + t] = tk <= p ? score_key(x[t]) : 0u;
-              }
-            }
-          }
         }
       }
+      // the accumulator may be overwritten once all four warps of the group have read it
+      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(L::B_AEMPTY + g));
     }
-    // TMEM is rewritten by the next block's MMA only after every warp has read it.
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-    __syncthreads();
   }
 
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
-  if (warp == 0) {
+  if (warp == kWarpMma) {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(L::TMEM_COLS));
   }
 }
