@@ -47,12 +47,13 @@ struct TsLayout {
   static constexpr int Q_BYTES = HALVES * kTileQ * 128;
   static constexpr int K_BYTES = HALVES * B * 128;
   static constexpr int MAP_BYTES = kTileQ * kRun * 2;  // int16 [kTileQ][kRun]
-  static constexpr int AVAIL = 227 * 1024 - 1024 - Q_BYTES - MAP_BYTES - 256;
+  static constexpr int AVAIL = 227 * 1024 - 1024 - Q_BYTES - MAP_BYTES - kTileQ * 4 - 256;
   static constexpr int STAGES = AVAIL / K_BYTES >= 4 ? 4 : AVAIL / K_BYTES;  // K tiles in flight
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = Q_OFF + Q_BYTES;
   static constexpr int MAP_OFF = K_OFF + STAGES * K_BYTES;
-  static constexpr int BAR_OFF = MAP_OFF + MAP_BYTES;
+  static constexpr int W_OFF = MAP_OFF + MAP_BYTES;  // fp32 [kTileQ] head weights of the tile rows
+  static constexpr int BAR_OFF = W_OFF + kTileQ * 4;
   // mbarriers: q full | accumulator full x 2 | accumulator empty x 2 | K full x S | K empty x S
   static constexpr int B_Q = 0, B_AFULL = 1, B_AEMPTY = 3, B_KFULL = 5, B_KEMPTY = 5 + STAGES;
   static constexpr int NBAR = 5 + 2 * STAGES;
@@ -67,7 +68,11 @@ struct TsLayout {
 
 using namespace tc;
 
-template <int D, int B>
+// HET = 0: TMEM lane = tile row (query, head), columns = the block's tokens.  HET = 8 or 16
+// (token-major, B = 128): the MMA operands swap, so TMEM lane = token and columns = tile rows; a
+// query's HET heads are then consecutive registers of one thread and a warp's 32 lanes write 32
+// consecutive keys of a query.
+template <int D, int B, int HET>
 __global__ void __launch_bounds__(kThreads, 1)
     token_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                           const int32_t* __restrict__ block_idx, int slots, uint32_t* __restrict__ keys,
@@ -75,6 +80,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                           int64_t nq, const float* __restrict__ w_idx, int HI) {
   using L = TsLayout<D, B>;
   constexpr int S = L::STAGES;
+  constexpr bool kTokenMajor = HET > 0;
+  static_assert(!kTokenMajor || (B == kTileQ && 32 % HET == 0), "token-major readout: B = 128, HET divides 32");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
 
@@ -174,9 +181,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int hh = 0; hh < L::HALVES; ++hh) {
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const uint64_t ad = desc_kmajor_sw128(q_base + hh * kTileQ * 128 + k * 32);
-            const uint64_t bd = desc_kmajor_sw128(k_base + st * L::K_BYTES + hh * B * 128 + k * 32);
-            umma_bf16(acc_col, ad, bd, L::IDESC, (hh | k) ? 1u : 0u);
+            const uint64_t qd = desc_kmajor_sw128(q_base + hh * kTileQ * 128 + k * 32);
+            const uint64_t kd = desc_kmajor_sw128(k_base + st * L::K_BYTES + hh * B * 128 + k * 32);
+            if constexpr (kTokenMajor)
+              umma_bf16(acc_col, kd, qd, L::IDESC, (hh | k) ? 1u : 0u);  // D[token][row]
+            else
+              umma_bf16(acc_col, qd, kd, L::IDESC, (hh | k) ? 1u : 0u);  // D[row][token]
           }
         }
         umma_commit(bar(L::B_KEMPTY + st));  // the stage may be refilled once these MMAs have read it
@@ -226,6 +236,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    if constexpr (kTokenMajor) {
+      float* wsm = reinterpret_cast<float*>(smem + L::W_OFF);
+      if (tid < kTileQ) {
+        const int64_t qr = tq0 + tid / HET;
+        wsm[tid] = (qr >= t_lo && qr < t_hi) ? w_idx[qr * HET + tid % HET] : 0.f;
+      }
+    }
     asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");  // the slot maps are complete
 
     // This thread's TMEM lane = tile row r: query tq0 + r / HE, indexer head r % HE.
@@ -244,14 +261,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      // rows whose query kept block jb0 + b
-      const int slot = row_ok ? smap[qi * kRun + b] : -1;
-      if (__any_sync(0xFFFFFFFFu, slot >= 0)) {
-        const int64_t j = jb0 + b;
-        const int64_t tok0 = j * B;
-        uint32_t* dst = krow_keys + (int64_t)(slot < 0 ? 0 : slot) * B;
+      if constexpr (kTokenMajor) {
+        // lane = token jb * B + quarter * 32 + lane; chunk cc holds queries cc * kQpc .. + kQpc - 1
+        constexpr int kQpc = 32 / (HET > 0 ? HET : 1);
+        const float* wsm = reinterpret_cast<const float*>(smem + L::W_OFF);
+        const int64_t tk = (jb0 + b) * B + quarter * 32 + lane;
 #pragma unroll 1
-        for (int cc = 0; cc < B / 32; ++cc) {
+        for (int cc = 0; cc < kTileQ / 32; ++cc) {
+          int sl[kQpc];
+          bool any = false;
+#pragma unroll
+          for (int qq = 0; qq < kQpc; ++qq) {
+            const int ql = cc * kQpc + qq;
+            const int64_t qr = tq0 + ql;
+            sl[qq] = (qr >= t_lo && qr < t_hi) ? smap[ql * kRun + b] : -1;  // the same in every lane
+            any = any || sl[qq] >= 0;
+          }
+          if (!any) continue;  // warp-uniform
           uint32_t v[32];
           const uint32_t addr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(g * B + cc * 32);
           asm volatile(
@@ -264,50 +290,87 @@ __global__ void __launch_bounds__(kThreads, 1)
                 "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
               : "r"(addr));
           asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-          if (HI == 0) {
-            if (slot >= 0) {
 #pragma unroll
-              for (int t = 0; t < 32; t += 4) {
-                const int64_t tk = tok0 + cc * 32 + t;
-                uint4 w;
-                w.x = tk <= p ? score_key(__uint_as_float(v[t])) : 0u;
-                w.y = tk + 1 <= p ? score_key(__uint_as_float(v[t + 1])) : 0u;
-                w.z = tk + 2 <= p ? score_key(__uint_as_float(v[t + 2])) : 0u;
-                w.w = tk + 3 <= p ? score_key(__uint_as_float(v[t + 3])) : 0u;
-                *reinterpret_cast<uint4*>(dst + cc * 32 + t) = w;
-              }
+          for (int qq = 0; qq < kQpc; ++qq) {
+            if (sl[qq] >= 0) {
+              const int ql = cc * kQpc + qq;
+              const int64_t qr = tq0 + ql;
+              float sc = 0.f;
+#pragma unroll
+              for (int jh = 0; jh < HET; ++jh)
+                sc = fmaf(wsm[ql * HET + jh], fmaxf(__uint_as_float(v[qq * HET + jh]), 0.f), sc);
+              const int64_t pq = n_kv - n_q + (qr - seq * n_q);
+              keys[(qr - q0) * (int64_t)slots * B + (int64_t)sl[qq] * B + quarter * 32 + lane] =
+                  tk <= pq ? score_key(sc) : 0u;
             }
-          } else {
-            // Multi-head score w_j * max(0, q_j . k) per row, summed over the HE rows of a query
-            // with a transposing reduction: after it, the lane of head h holds the sums of tokens
-            // h * (32 / HE) .. (h + 1) * (32 / HE) - 1 of this chunk.
-            float x[32];
-#pragma unroll
-            for (int t = 0; t < 32; ++t) x[t] = wgt * fmaxf(__uint_as_float(v[t]), 0.f);
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-              if ((1 << m) < HE) {  // warp-uniform
-                constexpr int kHalfMax = 16;
-                const int half = 16 >> m;
-                const int o = HE >> (m + 1);
-                const bool up = (head & o) != 0;
-#pragma unroll
-                for (int t = 0; t < kHalfMax; ++t) {
-                  if (t < half) {
-                    const float send = up ? x[t] : x[t + half];
-                    const float keep = up ? x[t + half] : x[t];
-                    x[t] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, o);
+          }
+        }
+      } else {
+        // rows whose query kept block jb0 + b
+        const int slot = row_ok ? smap[qi * kRun + b] : -1;
+        if (__any_sync(0xFFFFFFFFu, slot >= 0)) {
+          const int64_t j = jb0 + b;
+          const int64_t tok0 = j * B;
+          uint32_t* dst = krow_keys + (int64_t)(slot < 0 ? 0 : slot) * B;
+  #pragma unroll 1
+          for (int cc = 0; cc < B / 32; ++cc) {
+            uint32_t v[32];
+            const uint32_t addr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(g * B + cc * 32);
+            asm volatile(
+                "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+                "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+                : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+                  "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
+                  "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
+                  "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]),
+                  "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+                : "r"(addr));
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+            if (HI == 0) {
+              if (slot >= 0) {
+  #pragma unroll
+                for (int t = 0; t < 32; t += 4) {
+                  const int64_t tk = tok0 + cc * 32 + t;
+                  uint4 w;
+                  w.x = tk <= p ? score_key(__uint_as_float(v[t])) : 0u;
+                  w.y = tk + 1 <= p ? score_key(__uint_as_float(v[t + 1])) : 0u;
+                  w.z = tk + 2 <= p ? score_key(__uint_as_float(v[t + 2])) : 0u;
+                  w.w = tk + 3 <= p ? score_key(__uint_as_float(v[t + 3])) : 0u;
+                  *reinterpret_cast<uint4*>(dst + cc * 32 + t) = w;
+                }
+              }
+            } else {
+              // Multi-head score w_j * max(0, q_j . k) per row, summed over the HE rows of a query
+              // with a transposing reduction: after it, the lane of head h holds the sums of tokens
+              // h * (32 / HE) .. (h + 1) * (32 / HE) - 1 of this chunk.
+              float x[32];
+  #pragma unroll
+              for (int t = 0; t < 32; ++t) x[t] = wgt * fmaxf(__uint_as_float(v[t]), 0.f);
+  #pragma unroll
+              for (int m = 0; m < 4; ++m) {
+                if ((1 << m) < HE) {  // warp-uniform
+                  constexpr int kHalfMax = 16;
+                  const int half = 16 >> m;
+                  const int o = HE >> (m + 1);
+                  const bool up = (head & o) != 0;
+  #pragma unroll
+                  for (int t = 0; t < kHalfMax; ++t) {
+                    if (t < half) {
+                      const float send = up ? x[t] : x[t + half];
+                      const float keep = up ? x[t + half] : x[t];
+                      x[t] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, o);
+                    }
                   }
                 }
               }
-            }
-            if (slot >= 0) {
-              const int n = 32 / HE, t0 = head * n;
-#pragma unroll
-              for (int t = 0; t < 32; ++t) {
-                if (t < n) {
-                  const int64_t tk = tok0 + cc * 32 + t0 + t;
-                  dst[cc * 32 + t0 + t] = tk <= p ? score_key(x[t]) : 0u;
+              if (slot >= 0) {
+                const int n = 32 / HE, t0 = head * n;
+  #pragma unroll
+                for (int t = 0; t < 32; ++t) {
+                  if (t < n) {
+                    const int64_t tk = tok0 + cc * 32 + t0 + t;
+                    dst[cc * 32 + t0 + t] = tk <= p ? score_key(x[t]) : 0u;
+                  }
                 }
               }
             }
@@ -329,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, int B>
+template <int D, int B, int HET>
 cudaError_t launch_ts(const Shape& s, const void* q_idx, const void* k_idx, const int32_t* block_idx, int slots,
                       uint32_t* keys, int32_t* status, int64_t q0, int64_t nq, cudaStream_t st) {
   using L = TsLayout<D, B>;
@@ -338,7 +401,7 @@ cudaError_t launch_ts(const Shape& s, const void* q_idx, const void* k_idx, cons
   const int QT = kTileQ / HE;
   if (!map_bf16_sw128(&mq, q_idx, D, (uint64_t)s.n_query * HE, kTileQ)) return cudaErrorNotSupported;
   if (!map_bf16_sw128(&mk, k_idx, D, (uint64_t)s.batch * s.n_kv, B)) return cudaErrorNotSupported;
-  auto kern = token_score_tc_kernel<D, B>;
+  auto kern = token_score_tc_kernel<D, B, HET>;
   cudaError_t e = ensure_smem((const void*)kern, L::SMEM);
   if (e != cudaSuccess) return e;
   const int q_tiles = (int)((s.n_q + QT - 1) / QT);
@@ -367,8 +430,16 @@ bool token_score_tc_eligible(const Shape& s, int slots) {
 cudaError_t launch_token_score_tc(const Shape& s, const void* q_idx, const void* k_idx, const int32_t* block_idx,
                                   int slots, uint32_t* keys, int32_t* status, int64_t q0, int64_t nq, cudaStream_t st) {
   if (!token_score_tc_eligible(s, slots)) return cudaErrorNotSupported;
+  // 8 or 16 indexer heads with B = 128: token-major readout (a query's heads in one thread)
+  if (s.B == 128 && (s.HI == 8 || s.HI == 16)) {
+    if (s.d_idx == 64)
+      return s.HI == 8 ? launch_ts<64, 128, 8>(s, q_idx, k_idx, block_idx, slots, keys, status, q0, nq, st)
+                       : launch_ts<64, 128, 16>(s, q_idx, k_idx, block_idx, slots, keys, status, q0, nq, st);
+    return s.HI == 8 ? launch_ts<128, 128, 8>(s, q_idx, k_idx, block_idx, slots, keys, status, q0, nq, st)
+                     : launch_ts<128, 128, 16>(s, q_idx, k_idx, block_idx, slots, keys, status, q0, nq, st);
+  }
 #define HISA_TS_CASE(DD, BB) \
-  if (s.d_idx == DD && s.B == BB) return launch_ts<DD, BB>(s, q_idx, k_idx, block_idx, slots, keys, status, q0, nq, st);
+  if (s.d_idx == DD && s.B == BB) return launch_ts<DD, BB, 0>(s, q_idx, k_idx, block_idx, slots, keys, status, q0, nq, st);
   HISA_TS_CASE(64, 32) HISA_TS_CASE(64, 64) HISA_TS_CASE(64, 128) HISA_TS_CASE(64, 256)
   HISA_TS_CASE(128, 32) HISA_TS_CASE(128, 64) HISA_TS_CASE(128, 128) HISA_TS_CASE(128, 256)
 #undef HISA_TS_CASE

@@ -30,6 +30,9 @@ CASES = [
     Workload("mh16_prefill", 1, 257, 700, 64, 32, 4, 150, 2, 1, 64, 0, 0, 16),
     Workload("mh2_d256", 1, 300, 800, 256, 64, 5, 100, 2, 2, 64, 0, 0, 2),
     Workload("mh8_decode", 3, 1, 5000, 64, 64, 8, 300, 2, 2, 64, 0, 0, 8),
+    # B = 128 with 8 or 16 heads: the token scorer's token-major readout (ragged tiles, a context prefix)
+    Workload("mh16_b128", 1, 700, 700, 128, 128, 4, 150, 2, 1, 64, 0, 0, 16),
+    Workload("mh8_b128_context", 2, 520, 900, 64, 128, 5, 200, 2, 2, 64, 0, 0, 8),
 ]
 
 
