@@ -78,8 +78,9 @@ def test_host_forward_equals_device_forward(hs, w):
     assert torch.equal(o2.view(torch.int16), o.view(torch.int16)) and torch.equal(lse2, lse)
 
 
-def test_host_forward_decode_groups_match_oracle(hs, oracle_lib):
-    w = Workload("host_decode", 5, 1, 7000, 64, 64, 8, 300, 4, 4, 64, needles=3)
+@pytest.mark.parametrize("batch", [5, 11])  # groups of one sequence; groups of one and two
+def test_host_forward_decode_groups_match_oracle(hs, oracle_lib, batch):
+    w = Workload("host_decode", batch, 1, 7000, 64, 64, 8, 300, 4, 4, 64, needles=3)
     inp = full_inputs(w)
     ref = oracle_lib.run(w, inp)
     o, lse = _run_host(hs, w, _host(inp), torch.cuda.Stream())
