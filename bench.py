@@ -592,9 +592,20 @@ def oracle_sample(w, seconds: float, device_inputs=None):
         what = f"{done} query evaluations drawn uniformly over the {nq} positions"
     per_q = elapsed / done
     total_s = pool_s + per_q * nq
+    # the same path on one core: a short sample of queries drawn the same way
+    O.set_threads(1)
+    try:
+        ids = np.sort(rng.choice(nq, size=min(64, nq), replace=False)).astype(np.int64)
+        t0 = time.perf_counter()
+        O.run(w, inp, query_ids=ids, block_keys=bkeys)
+        per_q1 = (time.perf_counter() - t0) / len(ids)
+    finally:
+        O.set_threads(threads)
     return {"value": nq / total_s, "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": f"{what}, full path (top-m, top-k, attention in fp64) plus pooling of every block; "
-                      f"{elapsed + pool_s:.1f} s of CPU time, scaled to the whole workload"}
+                      f"{elapsed + pool_s:.1f} s of CPU time, scaled to the whole workload",
+            "single_core_value": 1.0 / per_q1, "single_core_sample": f"{len(ids)} queries on one thread "
+                                                                     f"(pooling excluded)"}
 
 
 def oracle_sample_rows(w, seconds: float):
