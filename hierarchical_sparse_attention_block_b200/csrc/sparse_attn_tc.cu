@@ -33,6 +33,7 @@
 // (max, sum, O) states of its split.  The scores of tile t+1 are computed
 // while the softmax of tile t runs.  Every wait is bounded (1 s): a timeout
 // sets status bit 1 and the CTA stops.
+#include <atomic>
 #include <math.h>
 
 #include "common.cuh"
@@ -664,15 +665,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 int sm_count() {
-  static int cached[64] = {0};
+  static std::atomic<int> cached[64] = {};  // per device; several host threads may launch at once
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (cached[dev] == 0) {
-    int n = 0;
+  int n = cached[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-    cached[dev] = n;
+    cached[dev].store(n, std::memory_order_relaxed);
   }
-  return cached[dev];
+  return n;
 }
 
 template <int GS>
