@@ -62,6 +62,7 @@ PREFILL = [
     Workload("host_prefill_chunks", 2, 20000, 20000, 64, 64, 8, 256, 2, 2, 64),  # 3 chunks per sequence
     Workload("host_context_gqa", 1, 9000, 12000, 128, 128, 8, 512, 8, 2, 128),  # prefix context, GQA
     Workload("host_multihead_indexer", 1, 9000, 9000, 64, 32, 6, 128, 2, 2, 64, n_idx_heads=4),
+    Workload("host_context_batch2", 2, 9000, 11000, 64, 64, 8, 256, 2, 2, 64),  # chunks of sequence 1
 ]
 
 
@@ -99,3 +100,18 @@ def test_host_forward_rejects_device_buffers(hs):
     with pytest.raises(RuntimeError):
         hs.hisa_forward_host(p, h["q_idx"], dev["k_idx"], h["q"], h["k"], h["v"], o)
     torch.cuda.synchronize()
+
+
+def test_host_forward_one_query_last_chunk(hs, oracle_lib):
+    """8193 queries: the second chunk holds one query, whose 512-entry token list is split across
+    CTAs (two work items only, so the list is cut in four), so it is checked against the oracle's
+    tolerance; the first chunk stays bit-identical to hisa_forward."""
+    w = Workload("host_one_query_chunk", 1, 8193, 8193, 64, 64, 8, 512, 2, 2, 64)
+    inp = full_inputs(w)
+    ref_o, ref_lse = _run_device(hs, w, dev_inputs(inp))
+    o, lse = _run_host(hs, w, _host(inp), torch.cuda.Stream())
+    assert torch.equal(o[:, :8192].view(torch.int16), ref_o[:, :8192].view(torch.int16))
+    assert torch.equal(lse[:, :8192], ref_lse[:, :8192])
+    ref = oracle_lib.run(w, inp, query_ids=np.array([8192], dtype=np.int64))
+    assert_close(o[0, 8192].float().numpy().reshape(1, w.n_heads, w.d_head), ref["o"], "o")
+    assert_close(lse[0, 8192].numpy().reshape(1, w.n_heads), ref["lse"], "lse")
