@@ -41,6 +41,13 @@ constexpr int kThreads = (kEpiWarps + 2) * 32;
 constexpr int kTileQ = 128;
 constexpr int kRun = 64;  // key blocks per CTA
 
+// Fewest indexer heads (1 = the one-head indexer) for which B = 128 takes the token-major readout.
+// Measured on the 64K prefill token stage (row readout / token-major): 1 head 4.0 / 6.2 ms,
+// 2 heads 6.3 / 6.5 ms, 4 heads 8.9 / 7.5 ms.
+#ifndef HISA_TS_TM_MIN_HEADS
+#define HISA_TS_TM_MIN_HEADS 4
+#endif
+
 template <int D, int B>
 struct TsLayout {
   static constexpr int HALVES = D / 64;
@@ -240,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* wsm = reinterpret_cast<float*>(smem + L::W_OFF);
       if (tid < kTileQ) {
         const int64_t qr = tq0 + tid / HET;
-        wsm[tid] = (qr >= t_lo && qr < t_hi) ? w_idx[qr * HET + tid % HET] : 0.f;
+        wsm[tid] = (HI > 0 && qr >= t_lo && qr < t_hi) ? w_idx[qr * HET + tid % HET] : 0.f;
       }
     }
     asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");  // the slot maps are complete
@@ -296,9 +303,13 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int ql = cc * kQpc + qq;
               const int64_t qr = tq0 + ql;
               float sc = 0.f;
+              if (HET == 1 && HI == 0) {
+                sc = __uint_as_float(v[qq]);  // the one-head indexer: the plain dot product
+              } else {
 #pragma unroll
-              for (int jh = 0; jh < HET; ++jh)
-                sc = fmaf(wsm[ql * HET + jh], fmaxf(__uint_as_float(v[qq * HET + jh]), 0.f), sc);
+                for (int jh = 0; jh < HET; ++jh)
+                  sc = fmaf(wsm[ql * HET + jh], fmaxf(__uint_as_float(v[qq * HET + jh]), 0.f), sc);
+              }
               const int64_t pq = n_kv - n_q + (qr - seq * n_q);
               keys[(qr - q0) * (int64_t)slots * B + (int64_t)sl[qq] * B + quarter * 32 + lane] =
                   tk <= pq ? score_key(sc) : 0u;
@@ -430,13 +441,15 @@ bool token_score_tc_eligible(const Shape& s, int slots) {
 cudaError_t launch_token_score_tc(const Shape& s, const void* q_idx, const void* k_idx, const int32_t* block_idx,
                                   int slots, uint32_t* keys, int32_t* status, int64_t q0, int64_t nq, cudaStream_t st) {
   if (!token_score_tc_eligible(s, slots)) return cudaErrorNotSupported;
-  // 8 or 16 indexer heads with B = 128: token-major readout (a query's heads in one thread)
-  if (s.B == 128 && (s.HI == 8 || s.HI == 16)) {
-    if (s.d_idx == 64)
-      return s.HI == 8 ? launch_ts<64, 128, 8>(s, q_idx, k_idx, block_idx, slots, keys, status, q0, nq, st)
-                       : launch_ts<64, 128, 16>(s, q_idx, k_idx, block_idx, slots, keys, status, q0, nq, st);
-    return s.HI == 8 ? launch_ts<128, 128, 8>(s, q_idx, k_idx, block_idx, slots, keys, status, q0, nq, st)
-                     : launch_ts<128, 128, 16>(s, q_idx, k_idx, block_idx, slots, keys, status, q0, nq, st);
+  // B = 128 with at least HISA_TS_TM_MIN_HEADS indexer heads: token-major readout (a query's
+  // heads in one thread, coalesced key stores)
+  const int he = s.HI > 0 ? s.HI : 1;
+  if (s.B == 128 && he >= HISA_TS_TM_MIN_HEADS) {
+#define HISA_TS_TM(DD, HH) \
+  if (s.d_idx == DD && he == HH) return launch_ts<DD, 128, HH>(s, q_idx, k_idx, block_idx, slots, keys, status, q0, nq, st);
+    HISA_TS_TM(64, 1) HISA_TS_TM(64, 2) HISA_TS_TM(64, 4) HISA_TS_TM(64, 8) HISA_TS_TM(64, 16)
+    HISA_TS_TM(128, 1) HISA_TS_TM(128, 2) HISA_TS_TM(128, 4) HISA_TS_TM(128, 8) HISA_TS_TM(128, 16)
+#undef HISA_TS_TM
   }
 #define HISA_TS_CASE(DD, BB) \
   if (s.d_idx == DD && s.B == BB) return launch_ts<DD, BB, 0>(s, q_idx, k_idx, block_idx, slots, keys, status, q0, nq, st);

@@ -33,6 +33,7 @@ CASES = [
     # B = 128 with 8 or 16 heads: the token scorer's token-major readout (ragged tiles, a context prefix)
     Workload("mh16_b128", 1, 700, 700, 128, 128, 4, 150, 2, 1, 64, 0, 0, 16),
     Workload("mh8_b128_context", 2, 520, 900, 64, 128, 5, 200, 2, 2, 64, 0, 0, 8),
+    Workload("mh4_b128", 1, 600, 600, 128, 128, 4, 150, 2, 2, 64, 0, 0, 4),
 ]
 
 
