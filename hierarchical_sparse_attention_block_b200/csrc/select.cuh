@@ -147,11 +147,9 @@ __device__ int emit_selected(KeyFn keys, int n, SelectResult r, SelectShared<NT>
   return total;
 }
 
-// Count of nonzero keys, CTA-wide (all threads get the result).
-template <int NT, class KeyFn>
-__device__ int count_nonzero(KeyFn keys, int n, SelectShared<NT>& sm) {
-  int c = 0;
-  for (int i = threadIdx.x; i < n; i += NT) c += keys(i) != 0u;
+// Sum of one int per thread, CTA-wide (all threads get the result).  All NT threads must call.
+template <int NT>
+__device__ int cta_sum(int c, SelectShared<NT>& sm) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xFFFFFFFFu, c, o);
   if ((threadIdx.x & 31) == 0) sm.warp_cnt[threadIdx.x >> 5][0] = (uint32_t)c;
@@ -161,6 +159,14 @@ __device__ int count_nonzero(KeyFn keys, int n, SelectShared<NT>& sm) {
   for (int w = 0; w < NT / 32; ++w) tot += (int)sm.warp_cnt[w][0];
   __syncthreads();
   return tot;
+}
+
+// Count of nonzero keys, CTA-wide (all threads get the result).
+template <int NT, class KeyFn>
+__device__ int count_nonzero(KeyFn keys, int n, SelectShared<NT>& sm) {
+  int c = 0;
+  for (int i = threadIdx.x; i < n; i += NT) c += keys(i) != 0u;
+  return cta_sum<NT>(c, sm);
 }
 
 }  // namespace hisa

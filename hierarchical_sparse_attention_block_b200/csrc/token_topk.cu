@@ -221,11 +221,13 @@ __global__ void __launch_bounds__(kScoreThreads)
   }
 }
 
-template <int NT>
+// KS: the query's keys are staged in shared memory (else read from global memory each pass).
+template <int NT, bool KS>
 __global__ void __launch_bounds__(NT)
     token_select_kernel(const uint32_t* __restrict__ keys, const int32_t* __restrict__ block_idx, int slots,
                         int32_t* __restrict__ token_idx, float* __restrict__ token_scores, int64_t n_q, int log2B,
-                        int k, int64_t q0, int keys_in_smem) {
+                        int k, int64_t q0) {
+  constexpr bool keys_in_smem = KS;
   __shared__ SelectShared<NT> sm;
   extern __shared__ __align__(16) uint32_t dsm[];
   const int B = 1 << log2B;
@@ -237,18 +239,36 @@ __global__ void __launch_bounds__(NT)
   int32_t* sblk = reinterpret_cast<int32_t*>(dsm + (keys_in_smem ? n : 0));
 
   for (int r = threadIdx.x; r < slots; r += NT) sblk[r] = block_idx ? block_idx[qg * slots + r] : r;
+  int cnt = 0;  // nonzero keys this thread staged
   if (keys_in_smem) {
     if ((n & 3) == 0) {
       const uint4* src = reinterpret_cast<const uint4*>(row);
       uint4* dst = reinterpret_cast<uint4*>(skeys);
-      for (int i = threadIdx.x; i < n / 4; i += NT) dst[i] = src[i];
+      for (int i = threadIdx.x; i < n / 4; i += NT) {
+        const uint4 v = src[i];
+        dst[i] = v;
+        cnt += (v.x != 0u) + (v.y != 0u) + (v.z != 0u) + (v.w != 0u);
+      }
     } else {
-      for (int i = threadIdx.x; i < n; i += NT) skeys[i] = row[i];
+      for (int i = threadIdx.x; i < n; i += NT) {
+        const uint32_t v = row[i];
+        skeys[i] = v;
+        cnt += v != 0u;
+      }
     }
   }
   __syncthreads();
-  auto key = [&](int i) -> uint32_t { return keys_in_smem ? skeys[i] : row[i]; };
-  const int nv = count_nonzero<NT>(key, n, sm);
+  auto key = [&](int i) -> uint32_t {
+    if constexpr (KS)
+      return skeys[i];
+    else
+      return row[i];
+  };
+  int nv;
+  if constexpr (KS)
+    nv = cta_sum<NT>(cnt, sm);  // counted while staging
+  else
+    nv = count_nonzero<NT>(key, n, sm);
   const int K = min(k, nv);
   int32_t* out = token_idx + qg * k;
   float* osc = token_scores ? token_scores + qg * k : nullptr;
@@ -332,11 +352,13 @@ cudaError_t launch_token_select(const Shape& s, const uint32_t* keys, const int3
   while ((1 << log2B) < s.B) ++log2B;
   // Few queries (decode): one wide CTA per query keeps the selection from being latency-bound.
   const bool wide = nq < 2 * 148;
-  auto kern = wide ? token_select_kernel<kSelectThreadsWide> : token_select_kernel<kSelectThreads>;
+  auto kern = wide ? (in_smem ? token_select_kernel<kSelectThreadsWide, true>
+                              : token_select_kernel<kSelectThreadsWide, false>)
+                   : (in_smem ? token_select_kernel<kSelectThreads, true> : token_select_kernel<kSelectThreads, false>);
   const int nt = wide ? kSelectThreadsWide : kSelectThreads;
   cudaError_t e = ensure_smem((const void*)kern, smem);
   if (e != cudaSuccess) return e;
-  kern<<<(unsigned)nq, nt, smem, st>>>(keys, block_idx, slots, token_idx, token_scores, s.n_q, log2B, s.k, q0, in_smem);
+  kern<<<(unsigned)nq, nt, smem, st>>>(keys, block_idx, slots, token_idx, token_scores, s.n_q, log2B, s.k, q0);
   return cudaGetLastError();
 }
 
