@@ -13,6 +13,15 @@ Multi-GPU (torchrun, one rank per GPU): every rank runs its own independent
 copy of the workload (a different seed); there is no collective on the data
 path, so scaling is weak and the value is all ranks' queries over the slowest
 rank's time.
+
+Besides the device-resident step the line carries: `e2e` (the same metric
+through the public API with the inputs in pinned host memory and O/LSE read
+back: hisa_forward_host for prefill, hisa_forward_cached for decode),
+`roofline` (the attention kernel against the measured copy bandwidth, plus the
+measured L2 or HBM gather ceiling of its access pattern, and the DRAM traffic
+of the committed ncu record when its source hash matches), `cpu_baseline`
+(the oracle on the host cores, all cores and one), `clocks`, the flat-indexer
+speedup and the needle recall of the probe query.
 """
 from __future__ import annotations
 
