@@ -1,0 +1,59 @@
+"""The bench's own accounting, on the CPU: its closed-form candidate and kept-token counts (which
+set the attention kernel's algorithmic bytes and the roofline) must equal what the oracle counts
+query by query, and the byte formulas must follow the tensor shapes."""
+import importlib.util
+import os
+
+import numpy as np
+import pytest
+
+from synth.workloads import Workload, full_inputs
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def bench():
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    m = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(m)
+    return m
+
+
+CASES = [
+    Workload("counts_prefill", 1, 700, 700, 64, 32, 5, 100, 2, 2, 64),
+    Workload("counts_context", 2, 300, 1000, 64, 64, 4, 150, 2, 1, 64),  # queries after a context prefix
+    Workload("counts_all_blocks", 1, 200, 200, 64, 16, 64, 64, 1, 1, 64),  # m covers every block
+]
+
+
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+def test_closed_form_counts_match_the_oracle(bench, oracle_lib, w):
+    inp = full_inputs(w)
+    n_cand = k_eff = n_vis = 0
+    for seq in range(w.batch):
+        bk = oracle_lib.block_pool(inp["k_idx"][seq], w.block)
+        for i in range(w.n_q):
+            p = w.n_kv - w.n_q + i
+            sel, _ = oracle_lib.block_topm(inp["q_idx"][seq, i], bk, w.block, p, w.top_m)
+            _, ke, nc = oracle_lib.token_topk(inp["q_idx"][seq, i], inp["k_idx"][seq], w.block, p,
+                                             sel[sel >= 0], w.top_k)
+            n_cand += nc
+            k_eff += ke
+            n_vis += p // w.block + 1
+    counts = bench.closed_form_counts(w)
+    assert counts == {"n_cand": n_cand, "k_eff": k_eff, "n_vis": n_vis}
+
+
+def test_byte_formulas(bench):
+    w = Workload("bytes", 2, 300, 1000, 64, 64, 4, 150, 8, 2, 128)
+    c = bench.closed_form_counts(w)
+    nq = w.batch * w.n_q
+    # every kept token's K and V rows once per KV head, plus Q and O rows, LSE and the index lists
+    assert bench.attention_bytes(w, c) == (c["k_eff"] * 2 * 128 * 2 * 2 + nq * 8 * 128 * 2 * 2 + nq * 8 * 4
+                                           + nq * 150 * 4)
+    # every input once, every output once
+    assert bench.compulsory_bytes(w) == (2 * 1000 * 64 * 2 + nq * 64 * 2 + 2 * 1000 * 2 * 128 * 2 * 2
+                                         + nq * 8 * 128 * 2 * 2 + nq * 8 * 4)
+    wm = w.with_(n_idx_heads=4)
+    assert bench.compulsory_bytes(wm) - bench.compulsory_bytes(w) == nq * 3 * 64 * 2 + nq * 4 * 4
