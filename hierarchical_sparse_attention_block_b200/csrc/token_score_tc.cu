@@ -41,6 +41,11 @@ constexpr int kThreads = (kEpiWarps + 2) * 32;
 constexpr int kTileQ = 128;
 constexpr int kRun = 64;  // key blocks per CTA
 
+// Key stages in flight per CTA (fewer stages, less shared memory: more CTAs per SM).
+#ifndef HISA_TS_MAX_STAGES
+#define HISA_TS_MAX_STAGES 4
+#endif
+
 // Fewest indexer heads (1 = the one-head indexer) for which B = 128 takes the token-major readout.
 // Measured on the 64K prefill token stage (row readout / token-major): 1 head 4.0 / 6.2 ms,
 // 2 heads 6.3 / 6.5 ms, 4 heads 8.9 / 7.5 ms.
@@ -55,7 +60,7 @@ struct TsLayout {
   static constexpr int K_BYTES = HALVES * B * 128;
   static constexpr int MAP_BYTES = kTileQ * kRun * 2;  // int16 [kTileQ][kRun]
   static constexpr int AVAIL = 227 * 1024 - 1024 - Q_BYTES - MAP_BYTES - kTileQ * 4 - 256;
-  static constexpr int STAGES = AVAIL / K_BYTES >= 4 ? 4 : AVAIL / K_BYTES;  // K tiles in flight
+  static constexpr int STAGES = AVAIL / K_BYTES >= HISA_TS_MAX_STAGES ? HISA_TS_MAX_STAGES : AVAIL / K_BYTES;
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = Q_OFF + Q_BYTES;
   static constexpr int MAP_OFF = K_OFF + STAGES * K_BYTES;
