@@ -364,3 +364,31 @@ def test_decode_step_in_a_cuda_graph(hs, oracle_lib):
         torch.cuda.synchronize()
         assert torch.equal(got_tok, tok) and torch.equal(got_o, o)
     del g
+
+
+# Candidate lists longer than the selection kernel stages in shared memory (49152 keys): the keys
+# are then read from global memory in every pass.
+LONG_LISTS = [
+    Workload("flat_long_lists", 1, 4, 60000, 64, 64, 8, 512, 2, 2, 64),             # flat: 60032 keys
+    Workload("hier_long_lists", 2, 1, 70000, 64, 256, 200, 1024, 2, 2, 64, needles=5),  # m * B = 51200
+]
+
+
+@pytest.mark.parametrize("w", LONG_LISTS, ids=lambda w: w.name)
+def test_selection_from_global_memory(hs, oracle_lib, w):
+    inp = full_inputs(w)
+    dev = _dev(inp)
+    n = w.batch * w.n_q
+    if w.name.startswith("flat"):
+        ref = oracle_lib.run(w, inp, flat=True, attention=False)
+        p = hs.params_of(w)
+        tok = torch.empty((w.batch, w.n_q, w.top_k), dtype=torch.int32, device="cuda")
+        hs.hisa_flat_topk(p, dev["q_idx"], dev["k_idx"], tok)
+        assert np.array_equal(tok.cpu().numpy().reshape(n, w.top_k), ref["token_idx"])
+    else:
+        ref = oracle_lib.run(w, inp)
+        got = run_stages(hs, w, dev)
+        assert np.array_equal(got["block_idx"].cpu().numpy().reshape(n, w.top_m), ref["block_idx"])
+        assert np.array_equal(got["token_idx"].cpu().numpy().reshape(n, w.top_k), ref["token_idx"])
+        assert_close(got["o"].float().cpu().numpy().reshape(n, w.n_heads, w.d_head), ref["o"], "o")
+        assert int(got["status"].item()) == 0
