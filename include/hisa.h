@@ -179,11 +179,14 @@ hisa_status_t hisa_forward(const hisa_params_t* params, const void* q_idx, const
  * each sequence (a chunk of queries [i0, i1) needs the K/V rows up to its last
  * position only); attention of a chunk starts as soon as its rows have
  * arrived, and its O/LSE rows go back on copy_stream while the next chunk
- * runs.  Results equal hisa_forward's on the same inputs.  copy_stream
- * (nullable, or equal to stream) runs the copies; without one everything is
- * serialised on stream.  The call is synchronous: it returns when o and lse
- * are in host memory (it synchronises stream).  Returns HISA_ERR_INVALID_ARG
- * when a host argument is device memory. */
+ * runs.  The selections equal hisa_forward's on the same inputs, and so do o
+ * and lse bit for bit, except for a chunk or group with so few queries that
+ * its token lists are split across CTAs differently (then they differ by the
+ * rounding of the split merge).  copy_stream (nullable, or equal to stream)
+ * runs the copies; without one everything is serialised on stream.  The call
+ * is synchronous: it returns when o and lse are in host memory (it
+ * synchronises stream), so it cannot be captured in a CUDA graph.  Returns
+ * HISA_ERR_INVALID_ARG when a host argument is device memory. */
 hisa_status_t hisa_forward_host_workspace_size(const hisa_params_t* params, size_t* bytes);
 hisa_status_t hisa_forward_host(const hisa_params_t* params, const void* q_idx, const float* idx_weights,
                                 const void* k_idx, const void* q, const void* k, const void* v, void* o, float* lse,
