@@ -506,89 +506,97 @@ hisa_status_t hisa_forward_host(const hisa_params_t* params, const void* q_idx, 
   const bool overlap = copy_stream != nullptr && copy_stream != stream;
   cudaStream_t cs = overlap ? copy_stream : stream;
   EventSet events;
-  cudaError_t e = cudaSuccess;
-  auto ok = [&](cudaError_t r) {
-    if (e == cudaSuccess) e = r;
-    return e == cudaSuccess;
-  };
-  // the copy stream starts after the caller's earlier work on stream (which may use the workspace)
-  if (overlap) {
-    cudaEvent_t start;
-    if (!ok(events.make(&start)) || !ok(cudaEventRecord(start, stream)) || !ok(cudaStreamWaitEvent(cs, start, 0)))
-      return hisa::cuda_fail(e);
-  }
-
-  // Indexer inputs first, then steps 1-5 on stream while the attention inputs stream in.
-  const int64_t he = s.HI > 0 ? s.HI : 1;
-  const size_t qrow = (size_t)s.H * s.d * 2, kvrow = (size_t)s.Hkv * s.d * 2;
-  ok(cudaMemcpyAsync(d_q_idx, q_idx, (size_t)s.n_query * he * s.d_idx * 2, cudaMemcpyHostToDevice, stream));
-  if (d_w) ok(cudaMemcpyAsync(d_w, idx_weights, (size_t)s.n_query * s.HI * sizeof(float), cudaMemcpyHostToDevice,
-                              stream));
-  ok(cudaMemcpyAsync(d_k_idx, k_idx, (size_t)s.batch * s.n_kv * s.d_idx * 2, cudaMemcpyHostToDevice, stream));
-  if (e != cudaSuccess) return hisa::cuda_fail(e);
-  if (!ok(hisa::launch_block_pool(s, d_k_idx, 0, s.n_blk, bk, stream))) return hisa::cuda_fail(e);
-  rc = hisa::run_block_stage(s, d_q_idx, bk, blk, nullptr, dev_status, ws + L.f.blk_stage, stream);
-  if (rc != HISA_OK) return rc;
-  rc = hisa::run_token_stage(s, d_q_idx, d_k_idx, blk, s.m, tok, nullptr, dev_status, ws + L.f.keys,
-                             L.f.total - L.f.keys, stream);
-  if (rc != HISA_OK) return rc;
-
-  const std::vector<HostUnit> units = host_units(s);
-  std::vector<cudaEvent_t> in(units.size()), done(units.size());
-  auto h2d = [&](uint8_t* dst, const void* src, size_t off, size_t bytes) {
-    return ok(cudaMemcpyAsync(dst + off, static_cast<const uint8_t*>(src) + off, bytes, cudaMemcpyHostToDevice, cs));
-  };
-  for (size_t j = 0; j < units.size() && e == cudaSuccess; ++j) {
-    const HostUnit& u = units[j];
-    const Shape c = unit_shape(s, u);
-    // K/V rows [kv0, c.n_kv) of each of the unit's sequences; its Q rows
-    for (int seq = u.s0; seq < u.s1; ++seq) {
-      const size_t off = ((size_t)seq * s.n_kv + u.kv0) * kvrow, bytes = (size_t)(c.n_kv - u.kv0) * kvrow;
-      h2d(d_k, k, off, bytes);
-      h2d(d_v, v, off, bytes);
+  // Everything enqueued (on success or after an error) completes before the call returns, so
+  // the host buffers and the events are free afterwards.
+  auto enqueue = [&]() -> hisa_status_t {
+    cudaError_t e = cudaSuccess;
+    auto ok = [&](cudaError_t r) {
+      if (e == cudaSuccess) e = r;
+      return e == cudaSuccess;
+    };
+    // the copy stream starts after the caller's earlier work on stream (which may use the workspace)
+    if (overlap) {
+      cudaEvent_t start;
+      if (!ok(events.make(&start)) || !ok(cudaEventRecord(start, stream)) || !ok(cudaStreamWaitEvent(cs, start, 0)))
+        return hisa::cuda_fail(e);
     }
-    if (u.i0 == 0 && u.i1 == s.n_q)
-      h2d(d_q, q, (size_t)u.s0 * s.n_q * qrow, (size_t)(u.s1 - u.s0) * s.n_q * qrow);
-    else
-      h2d(d_q, q, ((size_t)u.s0 * s.n_q + u.i0) * qrow, (size_t)(u.i1 - u.i0) * qrow);
-    if (overlap && ok(events.make(&in[j]))) ok(cudaEventRecord(in[j], cs));
-  }
-  if (e != cudaSuccess) return hisa::cuda_fail(e);
 
-  // Step 6 per unit, as soon as its rows are in.
-  for (size_t j = 0; j < units.size(); ++j) {
-    const HostUnit& u = units[j];
-    const Shape c = unit_shape(s, u);
-    if (overlap && !ok(cudaStreamWaitEvent(stream, in[j], 0))) return hisa::cuda_fail(e);
-    const size_t q0 = (size_t)u.s0 * s.n_q + u.i0;  // first query row of the unit
-    const size_t kv_off = (size_t)u.s0 * s.n_kv * kvrow;
-    const int splits = hisa::attn_pick_splits(c);
-    if (!ok(hisa::launch_sparse_attn(c, d_q + q0 * qrow, d_k + kv_off, d_v + kv_off, tok + q0 * s.k, d_o + q0 * qrow,
-                                     d_lse + q0 * s.H, dev_status, splits, ws + L.part, stream)))
-      return hisa::cuda_fail(e);
-    if (overlap && ok(events.make(&done[j]))) ok(cudaEventRecord(done[j], stream));
+    // Indexer inputs first, then steps 1-5 on stream while the attention inputs stream in.
+    const int64_t he = s.HI > 0 ? s.HI : 1;
+    const size_t qrow = (size_t)s.H * s.d * 2, kvrow = (size_t)s.Hkv * s.d * 2;
+    ok(cudaMemcpyAsync(d_q_idx, q_idx, (size_t)s.n_query * he * s.d_idx * 2, cudaMemcpyHostToDevice, stream));
+    if (d_w) ok(cudaMemcpyAsync(d_w, idx_weights, (size_t)s.n_query * s.HI * sizeof(float), cudaMemcpyHostToDevice,
+                                stream));
+    ok(cudaMemcpyAsync(d_k_idx, k_idx, (size_t)s.batch * s.n_kv * s.d_idx * 2, cudaMemcpyHostToDevice, stream));
     if (e != cudaSuccess) return hisa::cuda_fail(e);
-  }
+    if (!ok(hisa::launch_block_pool(s, d_k_idx, 0, s.n_blk, bk, stream))) return hisa::cuda_fail(e);
+    rc = hisa::run_block_stage(s, d_q_idx, bk, blk, nullptr, dev_status, ws + L.f.blk_stage, stream);
+    if (rc != HISA_OK) return rc;
+    rc = hisa::run_token_stage(s, d_q_idx, d_k_idx, blk, s.m, tok, nullptr, dev_status, ws + L.f.keys,
+                               L.f.total - L.f.keys, stream);
+    if (rc != HISA_OK) return rc;
 
-  // O and LSE of each unit back to the host once its attention is done.
-  for (size_t j = 0; j < units.size() && e == cudaSuccess; ++j) {
-    const HostUnit& u = units[j];
-    const size_t q0 = (size_t)u.s0 * s.n_q + u.i0;
-    const size_t rows = (size_t)(u.s1 - u.s0) * (u.i1 - u.i0);  // contiguous: several sequences only whole
-    if (overlap) ok(cudaStreamWaitEvent(cs, done[j], 0));
-    ok(cudaMemcpyAsync(static_cast<uint8_t*>(o) + q0 * qrow, d_o + q0 * qrow, rows * qrow, cudaMemcpyDeviceToHost,
-                       cs));
-    if (lse)
-      ok(cudaMemcpyAsync(lse + q0 * s.H, d_lse + q0 * s.H, rows * s.H * sizeof(float), cudaMemcpyDeviceToHost, cs));
-  }
-  // The outputs are in host memory when the call returns: stream waits for the copies back and
-  // is synchronised (the events of the call are then complete before they are destroyed).
-  if (overlap && e == cudaSuccess) {
-    cudaEvent_t end;
-    if (ok(events.make(&end)) && ok(cudaEventRecord(end, cs))) ok(cudaStreamWaitEvent(stream, end, 0));
-  }
-  ok(cudaStreamSynchronize(stream));
-  return hisa::cuda_fail(e);
+    const std::vector<HostUnit> units = host_units(s);
+    std::vector<cudaEvent_t> in(units.size()), done(units.size());
+    auto h2d = [&](uint8_t* dst, const void* src, size_t off, size_t bytes) {
+      return ok(cudaMemcpyAsync(dst + off, static_cast<const uint8_t*>(src) + off, bytes, cudaMemcpyHostToDevice, cs));
+    };
+    for (size_t j = 0; j < units.size() && e == cudaSuccess; ++j) {
+      const HostUnit& u = units[j];
+      const Shape c = unit_shape(s, u);
+      // K/V rows [kv0, c.n_kv) of each of the unit's sequences; its Q rows
+      for (int seq = u.s0; seq < u.s1; ++seq) {
+        const size_t off = ((size_t)seq * s.n_kv + u.kv0) * kvrow, bytes = (size_t)(c.n_kv - u.kv0) * kvrow;
+        h2d(d_k, k, off, bytes);
+        h2d(d_v, v, off, bytes);
+      }
+      if (u.i0 == 0 && u.i1 == s.n_q)
+        h2d(d_q, q, (size_t)u.s0 * s.n_q * qrow, (size_t)(u.s1 - u.s0) * s.n_q * qrow);
+      else
+        h2d(d_q, q, ((size_t)u.s0 * s.n_q + u.i0) * qrow, (size_t)(u.i1 - u.i0) * qrow);
+      if (overlap && ok(events.make(&in[j]))) ok(cudaEventRecord(in[j], cs));
+    }
+    if (e != cudaSuccess) return hisa::cuda_fail(e);
+
+    // Step 6 per unit, as soon as its rows are in.
+    for (size_t j = 0; j < units.size(); ++j) {
+      const HostUnit& u = units[j];
+      const Shape c = unit_shape(s, u);
+      if (overlap && !ok(cudaStreamWaitEvent(stream, in[j], 0))) return hisa::cuda_fail(e);
+      const size_t q0 = (size_t)u.s0 * s.n_q + u.i0;  // first query row of the unit
+      const size_t kv_off = (size_t)u.s0 * s.n_kv * kvrow;
+      const int splits = hisa::attn_pick_splits(c);
+      if (!ok(hisa::launch_sparse_attn(c, d_q + q0 * qrow, d_k + kv_off, d_v + kv_off, tok + q0 * s.k, d_o + q0 * qrow,
+                                       d_lse + q0 * s.H, dev_status, splits, ws + L.part, stream)))
+        return hisa::cuda_fail(e);
+      if (overlap && ok(events.make(&done[j]))) ok(cudaEventRecord(done[j], stream));
+      if (e != cudaSuccess) return hisa::cuda_fail(e);
+    }
+
+    // O and LSE of each unit back to the host once its attention is done.
+    for (size_t j = 0; j < units.size() && e == cudaSuccess; ++j) {
+      const HostUnit& u = units[j];
+      const size_t q0 = (size_t)u.s0 * s.n_q + u.i0;
+      const size_t rows = (size_t)(u.s1 - u.s0) * (u.i1 - u.i0);  // contiguous: several sequences only whole
+      if (overlap) ok(cudaStreamWaitEvent(cs, done[j], 0));
+      ok(cudaMemcpyAsync(static_cast<uint8_t*>(o) + q0 * qrow, d_o + q0 * qrow, rows * qrow, cudaMemcpyDeviceToHost,
+                         cs));
+      if (lse)
+        ok(cudaMemcpyAsync(lse + q0 * s.H, d_lse + q0 * s.H, rows * s.H * sizeof(float), cudaMemcpyDeviceToHost, cs));
+    }
+    // The outputs are in host memory when the call returns: stream waits for the copies back and
+    // is synchronised (the events of the call are then complete before they are destroyed).
+    if (overlap && e == cudaSuccess) {
+      cudaEvent_t end;
+      if (ok(events.make(&end)) && ok(cudaEventRecord(end, cs))) ok(cudaStreamWaitEvent(stream, end, 0));
+    }
+    return hisa::cuda_fail(e);
+  };
+  const hisa_status_t st = enqueue();
+  if (overlap) (void)cudaStreamSynchronize(cs);
+  const cudaError_t se = cudaStreamSynchronize(stream);
+  if (st != HISA_OK) return st;
+  return hisa::cuda_fail(se);
 }
 
 hisa_status_t hisa_flat_topk_workspace_size(const hisa_params_t* params, size_t* min_bytes, size_t* preferred_bytes) {
