@@ -41,7 +41,8 @@ struct TcLayout {
   static constexpr int B_OFF = A_OFF + A_BYTES;
   static constexpr int S_OFF = B_OFF + B_BYTES;
   static constexpr int BAR_OFF = S_OFF + S_BYTES;      // 2 mbarriers + TMEM address
-  static constexpr int SMEM = BAR_OFF + 64 + 1024;     // + slack for 1024-byte alignment
+  static constexpr int W_OFF = BAR_OFF + 64;           // fp32 [kTileM] head weights of the tile rows
+  static constexpr int SMEM = W_OFF + kTileM * 4 + 1024;  // + slack for 1024-byte alignment
 };
 
 using namespace tc;
@@ -55,7 +56,10 @@ __device__ __forceinline__ uint32_t bf16_bits(float x) {
   return (uint32_t)(*reinterpret_cast<uint16_t*>(&h));
 }
 
-template <int D>
+// HET = 0: TMEM lane = tile row (query, head), columns = blocks.  HET = 4, 8 or 16 (token-major):
+// the MMA operands swap, so TMEM lane = block and columns = tile rows; a query's HET heads are then
+// consecutive registers of one thread and a warp writes 32 consecutive blocks of a query's row.
+template <int D, int HET>
 __global__ void __launch_bounds__(kTcThreads, 1)
     block_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_bk,
                           float* __restrict__ scores, int32_t* __restrict__ status, int64_t n_q, int64_t n_kv,
@@ -119,6 +123,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         "l"(reinterpret_cast<uint64_t>(&tmap_bk)), "r"(0), "r"(brow), "r"(bar_tma)
         : "memory");
   }
+  if constexpr (HET > 0) {
+    float* wsm = reinterpret_cast<float*>(smem + L::W_OFF);
+    const int64_t qr = q0 + tid / HET;
+    wsm[tid] = qr < n_q ? w_idx[((int64_t)seq * n_q + qr) * HET + tid % HET] : 0.f;
+  }
   bool ok = mbar_wait(bar_tma, 0);
   ok = __syncthreads_and(ok) != 0;
 
@@ -172,9 +181,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int h = 0; h < L::HALVES; ++h) {
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
-          const uint64_t ad = desc_kmajor_sw128(a0 + h * kTileM * 128 + s * 32);
-          const uint64_t bd = desc_kmajor_sw128(b0 + pl * L::B_PLANE + h * kTileN * 128 + s * 32);
+          const uint64_t qd = desc_kmajor_sw128(a0 + h * kTileM * 128 + s * 32);
+          const uint64_t kd = desc_kmajor_sw128(b0 + pl * L::B_PLANE + h * kTileN * 128 + s * 32);
           const uint32_t acc = first ? 0u : 1u;
+          // D[row][block], or D[block][row] for the token-major readout
+          const uint64_t ad = HET > 0 ? kd : qd, bd = HET > 0 ? qd : kd;
           asm volatile(
               "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
               " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem),
@@ -191,7 +202,42 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   ok = done;
 
-  if (ok) {
+  if (ok && HET > 0) {
+    // this thread's TMEM lane = block j0 + tid; chunk cc of the columns holds queries cc * kQpc ..
+    constexpr int kQpc = 32 / (HET > 0 ? HET : 1);
+    const float* wsm = reinterpret_cast<const float*>(smem + L::W_OFF);
+    const int64_t j = j0 + tid;
+#pragma unroll 1
+    for (int cc = 0; cc < kTileM / 32; ++cc) {
+      uint32_t v[32];
+      const uint32_t addr = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(cc * 32);
+      asm volatile(
+          "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+          "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+          : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+            "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+            "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]),
+            "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]),
+            "=r"(v[30]), "=r"(v[31])
+          : "r"(addr));
+      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+      for (int qq = 0; qq < kQpc; ++qq) {
+        const int ql = cc * kQpc + qq;
+        const int64_t qi = q0 + ql;
+        if (ql < QT && qi < n_q) {  // the same in every lane
+          const int64_t c = (n_kv - n_q + qi) / B;
+          if (j <= c) {
+            float sc = 0.f;
+#pragma unroll
+            for (int h = 0; h < (HET > 0 ? HET : 1); ++h)
+              sc = fmaf(wsm[ql * HET + h], fmaxf(__uint_as_float(v[qq * HET + h]), 0.f), sc);
+            scores[((int64_t)seq * n_q + qi) * n_blk + j] = sc;
+          }
+        }
+      }
+    }
+  } else if (ok) {
     // this thread's TMEM lane = tile row tid: query q0 + tid / HE (within the sequence), head tid % HE
     const int head = tid % HE;
     const int64_t qi = q0 + tid / HE;
@@ -280,7 +326,11 @@ cudaError_t launch_tc(const Shape& s, const void* q_idx, const float* bk, float*
   if (!make_map_2d(&mb, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, bk, D, (uint64_t)s.batch * s.n_blk, D, kTileN,
                    CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorNotSupported;
-  auto kern = block_score_tc_kernel<D>;
+  // 4, 8 or 16 indexer heads: the token-major readout (a query's heads in one thread)
+  auto kern = s.HI == 4    ? block_score_tc_kernel<D, 4>
+              : s.HI == 8  ? block_score_tc_kernel<D, 8>
+              : s.HI == 16 ? block_score_tc_kernel<D, 16>
+                           : block_score_tc_kernel<D, 0>;
   cudaError_t e = ensure_smem((const void*)kern, L::SMEM);
   if (e != cudaSuccess) return e;
   const int q_tiles = (int)((s.n_q + QT - 1) / QT);
