@@ -17,6 +17,11 @@
 //     fp32 accumulator in 128 TMEM columns) and commits them to an mbarrier.
 //   * Each warp reads its 32 TMEM lanes (= query rows) back with tcgen05.ld
 //     and stores the causally visible scores.
+// With a multi-head indexer the 128 rows are 128 / H queries x H heads and the
+// readout applies w_j * max(0, .) and sums a query's rows: by shuffles for 1
+// or 2 heads; for 4, 8 or 16 heads the MMA operands swap (TMEM lane = block,
+// columns = rows), so a query's heads are one thread's registers and a warp
+// writes 32 consecutive blocks of a query's score row.
 // Every wait is bounded (1 s of %globaltimer); a timeout sets status bit 1
 // and the CTA skips to releasing its TMEM.
 #include "common.cuh"
