@@ -77,6 +77,13 @@ def workload(a, seed_offset=0):
     return w.with_(seed=w.seed + seed_offset)
 
 
+def workload_config(w) -> dict:
+    """The workload's fields as the JSON line's `config` (both arms)."""
+    return {"workload": w.name, "batch": w.batch, "n_q": w.n_q, "n_kv": w.n_kv, "d_idx": w.d_idx,
+            "block": w.block, "top_m": w.top_m, "top_k": w.top_k, "n_heads": w.n_heads,
+            "n_kv_heads": w.n_kv_heads, "d_head": w.d_head, "n_idx_heads": w.n_idx_heads, "needles": w.needles}
+
+
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -431,10 +438,7 @@ def run_ours(a, rank, world, local_rank):
         "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded SplitMix64; integer indexer q/k in [-4,4], unit-variance "
                                   "Irwin-Hall Q/K/V, planted needle blocks)",
-        "config": {"workload": w.name, "batch": w.batch, "n_q": w.n_q, "n_kv": w.n_kv, "d_idx": w.d_idx,
-                   "block": w.block, "top_m": w.top_m, "top_k": w.top_k, "n_heads": w.n_heads,
-                   "n_kv_heads": w.n_kv_heads, "d_head": w.d_head,
-                   "needles": w.needles, "parallelism": f"dp{world} (independent copies)",
+        "config": {**workload_config(w), "parallelism": f"dp{world} (independent copies)",
                    "l2": f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write)"},
         "roofline": {"bound": "hbm", "kernel": "sparse_attn", "achieved": achieved, "peak": hbm_gbs, "unit": "GB/s",
                      "frac": achieved / hbm_gbs, "peak_kind": peak_kind,
@@ -683,7 +687,7 @@ def main():
             line = {"impl": "reference", "metric": METRIC, "value": cpu["value"], "unit": UNIT, "n_gpus": world,
                     "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * w.batch * w.n_q / cpu["value"],
                     "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-                    "data": "synthetic", "config": {"workload": w.name},
+                    "data": "synthetic", "config": {**workload_config(w), "parallelism": "host cores (oracle)"},
                     "cpu_baseline": {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")},
                     "e2e": {"value": cpu["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
             print(json.dumps(line), flush=True)

@@ -57,3 +57,10 @@ def test_byte_formulas(bench):
                                          + nq * 8 * 128 * 2 * 2 + nq * 8 * 4)
     wm = w.with_(n_idx_heads=4)
     assert bench.compulsory_bytes(wm) - bench.compulsory_bytes(w) == nq * 3 * 64 * 2 + nq * 4 * 4
+
+
+def test_workload_config_names_the_workload(bench):
+    w = Workload("cfg", 2, 300, 1000, 64, 64, 4, 150, 8, 2, 128, n_idx_heads=4, needles=3)
+    c = bench.workload_config(w)
+    assert c == {"workload": "cfg", "batch": 2, "n_q": 300, "n_kv": 1000, "d_idx": 64, "block": 64, "top_m": 4,
+                 "top_k": 150, "n_heads": 8, "n_kv_heads": 2, "d_head": 128, "n_idx_heads": 4, "needles": 3}
