@@ -111,7 +111,22 @@ def params_of(w) -> HisaParams:
 
 
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    """Device address of a CUDA tensor (None passes through).  A CPU tensor is refused here, before
+    a host address could reach a kernel."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"expected a CUDA tensor, got one on {t.device}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _hptr(t):
+    """Host address of a CPU tensor (None passes through), for the host-buffer entry point."""
+    if t is None:
+        return None
+    if t.is_cuda:
+        raise ValueError("expected a host (CPU) tensor, got a CUDA one")
+    return ctypes.c_void_p(t.data_ptr())
 
 
 def _stream(stream):
@@ -233,9 +248,9 @@ def hisa_forward_host(p, q_idx, k_idx, q, k, v, o, lse=None, dev_status=None, wo
         workspace = _workspace(hisa_forward_host_workspace_size(p), torch.device("cuda", torch.cuda.current_device()))
     cs = ctypes.c_void_p(copy_stream.cuda_stream) if copy_stream is not None else None
     _check("hisa_forward_host",
-           _lib.hisa_forward_host(ctypes.byref(p), _ptr(q_idx), _ptr(idx_weights), _ptr(k_idx), _ptr(q), _ptr(k),
-                                  _ptr(v), _ptr(o), _ptr(lse), _ptr(dev_status), _ptr(workspace), workspace.numel(),
-                                  _stream(stream), cs))
+           _lib.hisa_forward_host(ctypes.byref(p), _hptr(q_idx), _hptr(idx_weights), _hptr(k_idx), _hptr(q),
+                                  _hptr(k), _hptr(v), _hptr(o), _hptr(lse), _ptr(dev_status), _ptr(workspace),
+                                  workspace.numel(), _stream(stream), cs))
 
 
 def hisa_flat_topk_workspace_size(p):

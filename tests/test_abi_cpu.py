@@ -188,3 +188,19 @@ def test_forward_host_validation():
     assert call(nbytes=need - 1) == hs.HISA_ERR_WORKSPACE
     assert call(ws=None) == hs.HISA_ERR_WORKSPACE
     assert call(ws=ctypes.c_void_p(4104)) == hs.HISA_ERR_WORKSPACE
+
+
+def test_binding_refuses_tensors_on_the_wrong_side():
+    """The Python binding checks where each tensor lives before calling the library: the device
+    calls refuse CPU tensors (a host address must not reach a kernel) and hisa_forward_host
+    refuses CUDA tensors for its host arguments."""
+    torch = pytest.importorskip("torch")
+    p = _p()
+    cpu = torch.zeros(16, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        hs.hisa_block_pool(p, cpu, torch.zeros(16, dtype=torch.float32))
+    with pytest.raises(ValueError):
+        hs.sparse_attn_fwd(p, cpu, cpu, cpu, torch.zeros(4, dtype=torch.int32), cpu)
+    with pytest.raises(ValueError):
+        hs._hptr(type("FakeCuda", (), {"is_cuda": True})())
+    assert hs._hptr(cpu).value == cpu.data_ptr()
