@@ -41,10 +41,14 @@ class HisaParams(ctypes.Structure):
 
 
 class HisaError(RuntimeError):
-    def __init__(self, call: str, status: int):
-        detail = _lib.hisa_status_string(status).decode()
-        if status == HISA_ERR_CUDA:
-            detail += f" (cudaError {_lib.hisa_last_cuda_error()})"
+    """A call of the library returned a status other than HISA_OK, or the binding refused an argument
+    before the call (then ``status`` is HISA_ERR_INVALID_ARG, the status the library gives bad arguments)."""
+
+    def __init__(self, call: str, status: int, detail: str | None = None):
+        if detail is None:
+            detail = _lib.hisa_status_string(status).decode()
+            if status == HISA_ERR_CUDA:
+                detail += f" (cudaError {_lib.hisa_last_cuda_error()})"
         super().__init__(f"{call}: {detail}")
         self.status = status
 
@@ -116,7 +120,7 @@ def _ptr(t):
     if t is None:
         return None
     if not t.is_cuda:
-        raise ValueError(f"expected a CUDA tensor, got one on {t.device}")
+        raise HisaError("binding", HISA_ERR_INVALID_ARG, f"expected a CUDA tensor, got one on {t.device}")
     return ctypes.c_void_p(t.data_ptr())
 
 
@@ -125,7 +129,7 @@ def _hptr(t):
     if t is None:
         return None
     if t.is_cuda:
-        raise ValueError("expected a host (CPU) tensor, got a CUDA one")
+        raise HisaError("binding", HISA_ERR_INVALID_ARG, "expected a host (CPU) tensor, got a CUDA one")
     return ctypes.c_void_p(t.data_ptr())
 
 

@@ -197,10 +197,12 @@ def test_binding_refuses_tensors_on_the_wrong_side():
     torch = pytest.importorskip("torch")
     p = _p()
     cpu = torch.zeros(16, dtype=torch.bfloat16)
-    with pytest.raises(ValueError):
-        hs.hisa_block_pool(p, cpu, torch.zeros(16, dtype=torch.float32))
-    with pytest.raises(ValueError):
-        hs.sparse_attn_fwd(p, cpu, cpu, cpu, torch.zeros(4, dtype=torch.int32), cpu)
-    with pytest.raises(ValueError):
-        hs._hptr(type("FakeCuda", (), {"is_cuda": True})())
+    calls = (lambda: hs.hisa_block_pool(p, cpu, torch.zeros(16, dtype=torch.float32)),
+             lambda: hs.sparse_attn_fwd(p, cpu, cpu, cpu, torch.zeros(4, dtype=torch.int32), cpu),
+             lambda: hs._hptr(type("FakeCuda", (), {"is_cuda": True})()))
+    for call in calls:
+        with pytest.raises(hs.HisaError) as err:
+            call()
+        assert err.value.status == hs.HISA_ERR_INVALID_ARG
+        assert isinstance(err.value, RuntimeError)
     assert hs._hptr(cpu).value == cpu.data_ptr()

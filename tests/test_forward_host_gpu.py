@@ -97,8 +97,9 @@ def test_host_forward_rejects_device_buffers(hs):
     dev = dev_inputs(inp)
     p = hs.params_of(w)
     o = torch.empty((1, 256, 2, 64), dtype=torch.bfloat16).pin_memory()
-    with pytest.raises(RuntimeError):
+    with pytest.raises(hs.HisaError) as err:
         hs.hisa_forward_host(p, h["q_idx"], dev["k_idx"], h["q"], h["k"], h["v"], o)
+    assert err.value.status == hs.HISA_ERR_INVALID_ARG
     torch.cuda.synchronize()
 
 
