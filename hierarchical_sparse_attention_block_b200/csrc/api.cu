@@ -243,7 +243,7 @@ hisa_status_t hisa_sparse_attn_workspace_size(const hisa_params_t* params, size_
   hisa_status_t rc = hisa::make_shape(params, false, true, &s);
   if (rc != HISA_OK) return rc;
   if (!bytes) return HISA_ERR_INVALID_ARG;
-  *bytes = hisa::attn_partial_bytes(s, hisa::attn_pick_splits(s));
+  *bytes = hisa::attn_workspace_bytes(s);
   return HISA_OK;
 }
 
@@ -258,10 +258,9 @@ hisa_status_t sparse_attn_fwd(const hisa_params_t* params, const void* q, const 
       !hisa::aligned16(o))
     return HISA_ERR_INVALID_ARG;
   if (lse && !hisa::aligned16(lse)) return HISA_ERR_INVALID_ARG;
-  int splits = hisa::attn_pick_splits(s);
-  if (splits > 1 && (!workspace || !hisa::aligned16(workspace) || workspace_bytes < hisa::attn_partial_bytes(s, splits)))
-    splits = 1;
-  return hisa::cuda_fail(hisa::launch_sparse_attn(s, q, k, v, token_idx, o, lse, dev_status, splits, workspace, stream));
+  if (workspace && !hisa::aligned16(workspace)) return HISA_ERR_WORKSPACE;
+  return hisa::cuda_fail(hisa::launch_sparse_attn(s, q, k, v, token_idx, o, lse, dev_status, workspace,
+                                                  workspace ? workspace_bytes : 0, stream));
 }
 
 // Workspace of hisa_forward: block keys | block stage | block_idx | token_idx | attention partials | token keys.
@@ -281,7 +280,7 @@ FwdLayout fwd_layout(const Shape& s) {
   L.token_idx = off;
   off += hisa::align_up((size_t)s.n_query * s.k * sizeof(int32_t));
   L.attn = off;
-  off += hisa::align_up(hisa::attn_partial_bytes(s, hisa::attn_pick_splits(s)));
+  off += hisa::align_up(hisa::attn_workspace_bytes(s));
   L.keys = off;
   off += hisa::align_up(hisa::keys_preferred(s, s.m));
   L.total = off;
@@ -313,8 +312,8 @@ hisa_status_t forward_impl(const Shape& s, const FwdLayout& L, const void* q_idx
   rc = hisa::run_token_stage(s, q_idx, k_idx, blk, s.m, tok, nullptr, dev_status, ws + L.keys,
                              workspace_bytes - L.keys, stream);
   if (rc != HISA_OK) return rc;
-  const int splits = hisa::attn_pick_splits(s);
-  return hisa::cuda_fail(hisa::launch_sparse_attn(s, q, k, v, tok, o, lse, dev_status, splits, ws + L.attn, stream));
+  return hisa::cuda_fail(hisa::launch_sparse_attn(s, q, k, v, tok, o, lse, dev_status, ws + L.attn,
+                                                  hisa::attn_workspace_bytes(s), stream));
 }
 
 hisa_status_t check_forward_args(const void* q_idx, const void* k_idx, const void* q, const void* k, const void* v,
@@ -419,7 +418,7 @@ HostFwdLayout host_fwd_layout(const Shape& s) {
   size_t part = 0;
   for (const HostUnit& u : host_units(s)) {
     const Shape c = unit_shape(s, u);
-    part = std::max(part, hisa::attn_partial_bytes(c, hisa::attn_pick_splits(c)));
+    part = std::max(part, hisa::attn_workspace_bytes(c));
   }
   size_t off = L.f.total;
   auto take = [&](size_t bytes) {
@@ -565,9 +564,9 @@ hisa_status_t hisa_forward_host(const hisa_params_t* params, const void* q_idx, 
       if (overlap && !ok(cudaStreamWaitEvent(stream, in[j], 0))) return hisa::cuda_fail(e);
       const size_t q0 = (size_t)u.s0 * s.n_q + u.i0;  // first query row of the unit
       const size_t kv_off = (size_t)u.s0 * s.n_kv * kvrow;
-      const int splits = hisa::attn_pick_splits(c);
       if (!ok(hisa::launch_sparse_attn(c, d_q + q0 * qrow, d_k + kv_off, d_v + kv_off, tok + q0 * s.k, d_o + q0 * qrow,
-                                       d_lse + q0 * s.H, dev_status, splits, ws + L.part, stream)))
+                                       d_lse + q0 * s.H, dev_status, ws + L.part, hisa::attn_workspace_bytes(c),
+                                       stream)))
         return hisa::cuda_fail(e);
       if (overlap && ok(events.make(&done[j]))) ok(cudaEventRecord(done[j], stream));
       if (e != cudaSuccess) return hisa::cuda_fail(e);

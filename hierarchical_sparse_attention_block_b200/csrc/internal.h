@@ -57,11 +57,21 @@ cudaError_t launch_token_score_tc(const Shape& s, const void* q_idx, const void*
 cudaError_t launch_token_select(const Shape& s, const uint32_t* keys, const int32_t* block_idx, int slots,
                                 int32_t* token_idx, float* token_scores, int64_t q0, int64_t nq, cudaStream_t st);
 
-// Step 6.  splits > 1 needs partial buffers of attn_partial_bytes(s, splits).
+// Step 6.  The kernel is picked from the shape and the workspace: the query-tile kernel when it
+// applies and `ws` holds its masks, else the gather kernels, with the token lists split across CTAs
+// (few queries) when `ws` holds the partial states.  attn_workspace_bytes: what lets every path run.
 int attn_pick_splits(const Shape& s);
 size_t attn_partial_bytes(const Shape& s, int splits);
+size_t attn_workspace_bytes(const Shape& s);
 cudaError_t launch_sparse_attn(const Shape& s, const void* q, const void* k, const void* v, const int32_t* token_idx,
-                               void* o, float* lse, int32_t* status, int splits, void* partial, cudaStream_t st);
+                               void* o, float* lse, int32_t* status, void* ws, size_t ws_bytes, cudaStream_t st);
+// Step 6 for many queries per sequence: tiles of 128 queries x 128 keys on the tensor cores with
+// the selections as bit masks (masks: sparse_attn_qtile_bytes of device memory).
+bool sparse_attn_qtile_eligible(const Shape& s);
+size_t sparse_attn_qtile_bytes(const Shape& s);
+cudaError_t launch_sparse_attn_qtile(const Shape& s, const void* q, const void* k, const void* v,
+                                     const int32_t* token_idx, void* o, float* lse, int32_t* status, void* masks,
+                                     cudaStream_t st);
 // Merge of the per-split (max, sum, output) states into O and the LSE.
 cudaError_t launch_attn_merge(const Shape& s, const float* partial, void* o, float* lse, int splits, cudaStream_t st);
 // Step 6 on the tensor cores (tcgen05, TMA gather), head dimension 128; cudaErrorNotSupported

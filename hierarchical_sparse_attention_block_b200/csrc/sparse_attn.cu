@@ -537,9 +537,22 @@ cudaError_t launch_attn_merge(const Shape& s, const float* partial, void* o, flo
   return cudaGetLastError();
 }
 
+size_t attn_workspace_bytes(const Shape& s) {
+  const size_t part = attn_partial_bytes(s, attn_pick_splits(s));
+  const size_t masks = sparse_attn_qtile_eligible(s) ? sparse_attn_qtile_bytes(s) : 0;
+  return part > masks ? part : masks;
+}
+
 cudaError_t launch_sparse_attn(const Shape& s, const void* q, const void* k, const void* v, const int32_t* token_idx,
-                               void* o, float* lse, int32_t* status, int splits, void* partial, cudaStream_t st) {
-  float* part = static_cast<float*>(partial);
+                               void* o, float* lse, int32_t* status, void* ws, size_t ws_bytes, cudaStream_t st) {
+  // Many queries per sequence: tiles of queries against tiles of keys.
+  if (ws && sparse_attn_qtile_eligible(s) && ws_bytes >= sparse_attn_qtile_bytes(s)) {
+    const cudaError_t e = launch_sparse_attn_qtile(s, q, k, v, token_idx, o, lse, status, ws, st);
+    if (e != cudaErrorNotSupported) return e;
+  }
+  int splits = attn_pick_splits(s);
+  if (splits > 1 && (!ws || ws_bytes < attn_partial_bytes(s, splits))) splits = 1;
+  float* part = static_cast<float*>(ws);
   // Heads sharing K/V (GQA/MQA): the tensor-core kernel takes a KV group's heads together.
   if (sparse_attn_tc_eligible(s)) {
     const cudaError_t e = launch_sparse_attn_tc(s, q, k, v, token_idx, o, lse, status, splits, part, st);

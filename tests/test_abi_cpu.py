@@ -136,8 +136,16 @@ def test_workspace_sizes_follow_the_shapes():
     assert mn == 64 * 128 * 4 and pref == 32 * mn
     # the attention list is split across CTAs when there are few queries
     assert hs.hisa_sparse_attn_workspace_size(p) > 0
+    # many queries per sequence: the query-tile kernel's masks, 128 x 128 bits per (query tile,
+    # key tile), 512 x 512 tiles at 64K
     big = hs.params(1, 65536, 65536, 128, 128, 64, 2048, 16, 16, 128)
-    assert hs.hisa_sparse_attn_workspace_size(big) == 0
+    assert hs.hisa_sparse_attn_workspace_size(big) == 512 * 512 * 2048
+    # d = 64 has no query-tile kernel and no split lists at this size
+    big64 = hs.params(1, 65536, 65536, 128, 128, 64, 2048, 16, 16, 64)
+    assert hs.hisa_sparse_attn_workspace_size(big64) == 0
+    # a context much longer than the kept tokens: dense tiles would cost more than gathers
+    far = hs.params(1, 4096, 1 << 20, 128, 128, 64, 2048, 16, 16, 128)
+    assert hs.hisa_sparse_attn_workspace_size(far) == 0
 
 
 def test_gather_probe_validation():
