@@ -20,23 +20,26 @@
 // entry t of a row's list that lies in [0, p] and exceeds every in-range entry
 // before it; -1 entries are padding; other entries are skipped and flagged.
 //
-// Roles of the attention CTA (192 threads):
-//   * warp 4, one thread: TMA loads of the query tile (once) and of each key
-//     tile's K, V and 2 KB mask block into a ring of two stages;
+// Roles of the attention CTA (224 threads):
+//   * warps 0-3, one thread per query row (TMEM lane = row): first the row's
+//     q into tensor memory (the A operand of the score MMA); then per key
+//     tile read the row's 128 scores, mask them, raise the running max lazily
+//     (O in TMEM is rescaled only when a weight would exceed 2^8), write the
+//     weights over the scores, and at the end write O / l and the LSE;
+//   * warp 4, one thread: TMA loads of the K tiles into a ring of three slots,
+//     a slot refilled as soon as its score MMA has read it;
+//   * warp 6, one thread: TMA loads of the V tiles and 2 KB mask blocks into a
+//     ring of three slots, refilled once the output MMA has read them;
 //   * warp 5, one thread: S_j = Q K_jᵀ into one of two TMEM buffers
-//     (tcgen05.mma kind::f16, M = 128 queries, N = 128 keys), then
-//     O += P_{j-1} V_{j-1} (M = 128 queries, N = 128 dimensions; V read
-//     MN-major from its rows) with the weights P as the A operand in tensor
-//     memory, in the buffer their scores came from: the weights carry ~16
-//     significant bits as a bf16 pair hi + lo (hi the upper half of the fp32
-//     weight, lo the rounded rest), so the output MMA runs over K = 2 x 128
-//     (hi columns, then lo columns, both against the same V rows).  MMAs of
-//     one thread run in issue order, so S_{j+2} is written into the buffer
-//     only after P_j has been read from it;
-//   * warps 0-3, one thread per query row (TMEM lane = row): read the row's
-//     128 scores, mask them, raise the running max lazily (O in TMEM is
-//     rescaled only when a weight would exceed 2^8), write the weights over
-//     the scores, and at the end write O / l and the LSE.
+//     (tcgen05.mma kind::f16, M = 128 queries, N = 128 keys, q from tensor
+//     memory), then O += P_{j-1} V_{j-1} (M = 128 queries, N = 128
+//     dimensions; V read MN-major from its rows) with the weights P as the A
+//     operand in tensor memory, in the buffer their scores came from: the
+//     weights carry ~16 significant bits as a bf16 pair hi + lo (hi the upper
+//     half of the fp32 weight, lo the rounded rest), so the output MMA runs
+//     over K = 2 x 128 (hi columns, then lo columns, both against the same V
+//     rows).  MMAs of one thread run in issue order, so S_{j+2} is written
+//     into the buffer only after P_j has been read from it.
 // Every wait is bounded (1 s): a timeout sets status bit 1 and the CTA stops.
 #include <math.h>
 
@@ -65,24 +68,27 @@ using namespace tc;
 
 constexpr int kRows = 128;  // queries per tile = keys per key tile
 constexpr int kD = 128;     // head dimension
-constexpr int kNS = 2;      // K/V stages
-constexpr int kThreads = 192;
-constexpr int kWarpTMA = 4, kWarpMMA = 5;
-constexpr uint32_t kTmemCols = 512;  // scores / weights: buffer 0 at 0-127, 1 at 128-255; output O 256-383
-constexpr uint32_t kColO = 256;
+constexpr int kNS = 3;      // slots of the K ring and of the V ring
+constexpr int kThreads = 224;
+constexpr int kWarpK = 4, kWarpMMA = 5, kWarpV = 6;
+// Tensor memory: scores / weights buffer 0 at columns 0-127, buffer 1 at 128-255, output O at
+// 256-383, the query tile (bf16 pairs) at 384-447.
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColO = 256, kColQ = 384;
 
 constexpr int kHalf = kRows * 128;      // 64 columns of 128 rows of bf16 (one 128-byte swizzle span): 16 KB
 constexpr int kTile = 2 * kHalf;        // a 128 x 128 bf16 tile as two column halves
 constexpr int kMaskBytes = kRows * 16;  // 128 rows x 128 bits
-constexpr int kStage = 2 * kTile;       // K tile, then V tile
-constexpr int Q_OFF = 0;
-constexpr int KV_OFF = kTile;
-constexpr int MASK_OFF = KV_OFF + kNS * kStage;
+constexpr int K_OFF = 0;                        // K slot i at K_OFF + i * kTile
+constexpr int V_OFF = K_OFF + kNS * kTile;      // V slot i at V_OFF + i * kTile
+constexpr int MASK_OFF = V_OFF + kNS * kTile;   // mask of V slot i at MASK_OFF + i * kMaskBytes
 constexpr int BAR_OFF = MASK_OFF + kNS * kMaskBytes;
 enum : int {
-  B_FULL = 0,
-  B_EMPTY = kNS,
-  B_QFULL = 2 * kNS,
+  B_KFULL = 0,
+  B_KEMPTY = kNS,
+  B_VFULL = 2 * kNS,
+  B_VEMPTY = 3 * kNS,
+  B_QREADY = 4 * kNS,
   B_SFULL,  // [2]
   B_PREADY = B_SFULL + 2,
   B_PFREE,
@@ -92,7 +98,7 @@ enum : int {
 constexpr int MISC_OFF = BAR_OFF + kNBar * 8;
 constexpr int kSmem = MISC_OFF + 16 + 1024;  // + slack for the 1024-byte alignment of the swizzled tiles
 static_assert(kSmem <= 227 * 1024, "shared memory budget");
-static_assert(KV_OFF % 1024 == 0 && kStage % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
+static_assert(V_OFF % 1024 == 0 && kTile % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
 
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
@@ -162,8 +168,8 @@ __global__ void __launch_bounds__(kRows) attn_mask_kernel(const int32_t* __restr
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    sparse_attn_qtile_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
-                             const __grid_constant__ CUtensorMap map_v, const uint4* __restrict__ masks,
+    sparse_attn_qtile_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+                             const uint16_t* __restrict__ q, const uint4* __restrict__ masks,
                              uint16_t* __restrict__ o, float* __restrict__ lse, int32_t* __restrict__ status,
                              int64_t n_q, int64_t n_kv, int H, int Hkv, int batch, int nqt, int nkt, float qscale) {
   extern __shared__ uint8_t smem_raw[];
@@ -199,10 +205,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (tid == 0) {
     for (int i = 0; i < kNS; ++i) {
-      mbar_init(bar(B_FULL + i), 1);
-      mbar_init(bar(B_EMPTY + i), 1);
+      mbar_init(bar(B_KFULL + i), 1);
+      mbar_init(bar(B_KEMPTY + i), 1);
+      mbar_init(bar(B_VFULL + i), 1);
+      mbar_init(bar(B_VEMPTY + i), 1);
     }
-    mbar_init(bar(B_QFULL), 1);
+    mbar_init(bar(B_QREADY), kRows);
     for (int i = 0; i < 2; ++i) mbar_init(bar(B_SFULL + i), 1);
     mbar_init(bar(B_PREADY), kRows);
     mbar_init(bar(B_PFREE), 1);
@@ -215,70 +223,68 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == kWarpTMA) {
-    // ---------------- TMA producer ----------------
+  if (warp == kWarpK || warp == kWarpV) {
+    // ---------------- TMA producers: K tiles (warp 4), V tiles + masks (warp 6) ----------------
     if (lane == 0) {
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_k)) : "memory");
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_v)) : "memory");
-      mbar_expect_tx(bar(B_QFULL), kTile);
-      tma_load_3d(sb + Q_OFF, &map_q, 0, h, (int)row0, bar(B_QFULL));
-      tma_load_3d(sb + Q_OFF + kHalf, &map_q, 64, h, (int)row0, bar(B_QFULL));
+      const bool is_k = warp == kWarpK;
+      const CUtensorMap* map = is_k ? &map_k : &map_v;
+      const int full = is_k ? B_KFULL : B_VFULL, empty = is_k ? B_KEMPTY : B_VEMPTY;
+      const uint32_t base = sb + (uint32_t)(is_k ? K_OFF : V_OFF);
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
       int issued = 0;
       for (int j = 0; j < nv; ++j) {
         const int s = j % kNS;
-        if (j >= kNS && !mbar_wait_or_abort(bar(B_EMPTY + s), ((j / kNS) - 1) & 1, abort_flag)) {
+        if (j >= kNS && !mbar_wait_or_abort(bar(empty + s), ((j / kNS) - 1) & 1, abort_flag)) {
           fail();
           break;
         }
-        const uint32_t st = sb + (uint32_t)(KV_OFF + s * kStage);
+        const uint32_t dst = base + (uint32_t)(s * kTile);
         const int z = (int)((int64_t)seq * n_kv + (int64_t)j * kRows);
-        mbar_expect_tx(bar(B_FULL + s), kStage + kMaskBytes);
-        tma_load_3d(st, &map_k, 0, g, z, bar(B_FULL + s));
-        tma_load_3d(st + kHalf, &map_k, 64, g, z, bar(B_FULL + s));
-        tma_load_3d(st + kTile, &map_v, 0, g, z, bar(B_FULL + s));
-        tma_load_3d(st + kTile + kHalf, &map_v, 64, g, z, bar(B_FULL + s));
-        bulk_load(sb + (uint32_t)(MASK_OFF + s * kMaskBytes), mbase + (int64_t)j * kRows, kMaskBytes,
-                  bar(B_FULL + s));
+        mbar_expect_tx(bar(full + s), is_k ? kTile : kTile + kMaskBytes);
+        tma_load_3d(dst, map, 0, g, z, bar(full + s));
+        tma_load_3d(dst + kHalf, map, 64, g, z, bar(full + s));
+        if (!is_k)
+          bulk_load(sb + (uint32_t)(MASK_OFF + s * kMaskBytes), mbase + (int64_t)j * kRows, kMaskBytes,
+                    bar(full + s));
         issued = j + 1;
       }
       // The copies in flight land before the CTA may exit.
-      mbar_wait(bar(B_QFULL), 0);
-      for (int j = issued > kNS ? issued - kNS : 0; j < issued; ++j) mbar_wait(bar(B_FULL + j % kNS), (j / kNS) & 1);
+      for (int j = issued > kNS ? issued - kNS : 0; j < issued; ++j) mbar_wait(bar(full + j % kNS), (j / kNS) & 1);
     }
   } else if (warp == kWarpMMA) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);  // Q and K both K-major
+      constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);  // q (tensor memory), K K-major
       constexpr uint32_t kIdO = idesc_bf16(128, 128, false, true);   // P (tensor memory), V MN-major
-      bool ok = mbar_wait_or_abort(bar(B_QFULL), 0, abort_flag);
+      bool ok = mbar_wait_or_abort(bar(B_QREADY), 0, abort_flag);
       for (int j = 0; ok && j <= nv; ++j) {
         if (j < nv) {
-          const int s = j % kNS, b = j & 1;
-          // Buffer b held P_{j-2}, whose output MMA was issued before this one.
-          ok = mbar_wait_or_abort(bar(B_FULL + s), (j / kNS) & 1, abort_flag);
+          // Buffer j & 1 held P_{j-2}, whose output MMA was issued before this one.
+          const int s = j % kNS;
+          ok = mbar_wait_or_abort(bar(B_KFULL + s), (j / kNS) & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t kt = sb + (uint32_t)(KV_OFF + s * kStage);
+          const uint32_t kt = sb + (uint32_t)(K_OFF + s * kTile);
 #pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2)
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              umma_bf16(tmem + (uint32_t)(b * 128), desc_kmajor_sw128(sb + Q_OFF + h2 * kHalf + kk * 32),
-                        desc_kmajor_sw128(kt + h2 * kHalf + kk * 32), kIdS, (h2 | kk) ? 1u : 0u);
-          umma_commit(bar(B_SFULL + b));
+          for (int kk = 0; kk < kD / 16; ++kk)
+            umma_bf16_ta(tmem + (uint32_t)((j & 1) * 128), tmem + kColQ + (uint32_t)(8 * kk),
+                         desc_kmajor_sw128(kt + (kk >> 2) * kHalf + (kk & 3) * 32), kIdS, kk > 0 ? 1u : 0u);
+          umma_commit(bar(B_SFULL + (j & 1)));
+          umma_commit(bar(B_KEMPTY + s));
         }
         if (j >= 1) {
           const int jj = j - 1, s = jj % kNS;
-          ok = mbar_wait_or_abort(bar(B_PREADY), jj & 1, abort_flag);
+          ok = mbar_wait_or_abort(bar(B_VFULL + s), (jj / kNS) & 1, abort_flag) &&
+               mbar_wait_or_abort(bar(B_PREADY), jj & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t vt = sb + (uint32_t)(KV_OFF + s * kStage + kTile);
+          const uint32_t vt = sb + (uint32_t)(V_OFF + s * kTile);
           const uint32_t pt = tmem + (uint32_t)((jj & 1) * 128);
 #pragma unroll
           for (int t = 0; t < 2 * (kRows / 16); ++t)  // keys 16 t' .. 16 t' + 15, t' = t mod 8: hi, then lo
             umma_bf16_ta(tmem + kColO, pt + (uint32_t)(8 * t), desc_mnmajor_sw128(vt + (t & 7) * 2048, kHalf), kIdO,
                          (jj > 0 || t > 0) ? 1u : 0u);
-          umma_commit(bar(B_EMPTY + s));
+          umma_commit(bar(B_VEMPTY + s));
           umma_commit(bar(B_PFREE));
         }
       }
@@ -286,17 +292,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       umma_commit(bar(B_DRAIN));
       mbar_wait(bar(B_DRAIN), 0);
     }
-  } else {
+  } else if (warp < 4) {
     // ---------------- softmax and output: warps 0-3, thread = query row ----------------
     const int r = tid;
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    {
+      // q of this row (zero past the last query) as bf16 pairs in columns kColQ .. kColQ + 63
+      uint32_t qv[2][32];
+      const uint4* qrow = reinterpret_cast<const uint4*>(q + ((row0 + r) * H + h) * (int64_t)kD);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const uint4 x = r < nr ? __ldg(qrow + c) : make_uint4(0u, 0u, 0u, 0u);
+        qv[c >> 3][(c & 7) * 4 + 0] = x.x;
+        qv[c >> 3][(c & 7) * 4 + 1] = x.y;
+        qv[c >> 3][(c & 7) * 4 + 2] = x.z;
+        qv[c >> 3][(c & 7) * 4 + 3] = x.w;
+      }
+      tmem_st32_issue(tl + kColQ, qv[0]);
+      tmem_st32_issue(tl + kColQ + 32, qv[1]);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(B_QREADY));
+    }
     float m_run = -INFINITY;  // running max of the row's selected raw scores
     float l = 0.f;            // sum of the row's weights, relative to m_run
     const float lim = 8.f / qscale;
     bool err = false;
     for (int j = 0; j < nv; ++j) {
       const int s = j % kNS, b = j & 1;
-      const bool ok = mbar_wait_or_abort(bar(B_FULL + s), (j / kNS) & 1, abort_flag) &&
+      const bool ok = mbar_wait_or_abort(bar(B_VFULL + s), (j / kNS) & 1, abort_flag) &&
                       mbar_wait_or_abort(bar(B_SFULL + b), (j >> 1) & 1, abort_flag);
       if (!__all_sync(0xFFFFFFFFu, ok)) {
         err = true;
@@ -428,9 +452,8 @@ cudaError_t launch_sparse_attn_qtile(const Shape& s, const void* q, const void* 
                                      const int32_t* token_idx, void* o, float* lse, int32_t* status, void* masks,
                                      cudaStream_t st) {
   if (!sparse_attn_qtile_eligible(s)) return cudaErrorNotSupported;
-  CUtensorMap mq, mk, mv;
-  if (!map_bf16_rows_of_head(&mq, q, kD, (uint64_t)s.H, (uint64_t)s.n_query, kRows) ||
-      !map_bf16_rows_of_head(&mk, k, kD, (uint64_t)s.Hkv, (uint64_t)s.batch * s.n_kv, kRows) ||
+  CUtensorMap mk, mv;
+  if (!map_bf16_rows_of_head(&mk, k, kD, (uint64_t)s.Hkv, (uint64_t)s.batch * s.n_kv, kRows) ||
       !map_bf16_rows_of_head(&mv, v, kD, (uint64_t)s.Hkv, (uint64_t)s.batch * s.n_kv, kRows))
     return cudaErrorNotSupported;
   const int nqt = (int)n_tiles(s.n_q), nkt = (int)n_tiles(s.n_kv);
@@ -443,7 +466,8 @@ cudaError_t launch_sparse_attn_qtile(const Shape& s, const void* q, const void* 
   if (e != cudaSuccess) return e;
   const int64_t grid = (int64_t)s.H * nqt * s.batch;
   const float qscale = s.scale * 1.4426950408889634f;
-  sparse_attn_qtile_kernel<<<(unsigned)grid, kThreads, kSmem, st>>>(mq, mk, mv, m, static_cast<uint16_t*>(o), lse,
+  sparse_attn_qtile_kernel<<<(unsigned)grid, kThreads, kSmem, st>>>(mk, mv, static_cast<const uint16_t*>(q), m,
+                                                                    static_cast<uint16_t*>(o), lse,
                                                                     status, s.n_q, s.n_kv, s.H, s.Hkv, s.batch, nqt,
                                                                     nkt, qscale);
   return cudaGetLastError();
