@@ -25,7 +25,7 @@ EXPORTS = (
     "hisa_forward", "hisa_flat_topk_workspace_size", "hisa_flat_topk", "hisa_status_string",
     "hisa_last_cuda_error", "hisa_version", "hisa_token_topk_noalloc", "hisa_forward_cached", "hisa_gather_probe",
     "hisa_block_candidates_workspace_size", "hisa_block_candidates", "hisa_topk_merge", "hisa_remap_ids",
-    "hisa_lse_merge", "hisa_forward_host_workspace_size", "hisa_forward_host",
+    "hisa_lse_merge", "hisa_forward_host_workspace_size", "hisa_forward_host", "hisa_sparse_attn_kernel",
 )
 
 
@@ -82,6 +82,7 @@ def _load():
         "hisa_topk_merge": [vp, vp, ctypes.c_int32, i64, ctypes.c_int32, ctypes.c_int32, vp, vp, vp],
         "hisa_remap_ids": [vp, i64, ctypes.c_int32, i64, i64, i64, vp, vp],
         "hisa_lse_merge": [vp, vp, ctypes.c_int32, i64, ctypes.c_int32, vp, vp, vp],
+        "hisa_sparse_attn_kernel": [pp, ctypes.c_size_t, ctypes.POINTER(ctypes.c_int32)],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -209,6 +210,17 @@ def sparse_attn_fwd(p, q, k, v, token_idx, o, lse=None, dev_status=None, workspa
     _check("sparse_attn_fwd", _lib.sparse_attn_fwd(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(token_idx),
                                                    _ptr(o), _ptr(lse), _ptr(dev_status), _ptr(workspace),
                                                    0 if workspace is None else workspace.numel(), _stream(stream)))
+
+
+ATTN_GATHER, ATTN_QTILE = 0, 1
+
+
+def hisa_sparse_attn_kernel(p, workspace_bytes: int) -> int:
+    """Which step-6 kernel sparse_attn_fwd runs with this workspace: ATTN_QTILE or ATTN_GATHER."""
+    k = ctypes.c_int32(-1)
+    _check("hisa_sparse_attn_kernel", _lib.hisa_sparse_attn_kernel(ctypes.byref(p), int(workspace_bytes),
+                                                                    ctypes.byref(k)))
+    return k.value
 
 
 def hisa_forward_workspace_size(p) -> int:

@@ -263,6 +263,15 @@ hisa_status_t sparse_attn_fwd(const hisa_params_t* params, const void* q, const 
                                                   workspace ? workspace_bytes : 0, stream));
 }
 
+hisa_status_t hisa_sparse_attn_kernel(const hisa_params_t* params, size_t workspace_bytes, int32_t* kind) {
+  Shape s;
+  hisa_status_t rc = hisa::make_shape(params, false, true, &s);
+  if (rc != HISA_OK) return rc;
+  if (!kind) return HISA_ERR_INVALID_ARG;
+  *kind = hisa::sparse_attn_qtile_eligible(s) && workspace_bytes >= hisa::sparse_attn_qtile_bytes(s) ? 1 : 0;
+  return HISA_OK;
+}
+
 // Workspace of hisa_forward: block keys | block stage | block_idx | token_idx | attention partials | token keys.
 namespace {
 struct FwdLayout {

@@ -66,11 +66,12 @@ size_t attn_workspace_bytes(const Shape& s);
 cudaError_t launch_sparse_attn(const Shape& s, const void* q, const void* k, const void* v, const int32_t* token_idx,
                                void* o, float* lse, int32_t* status, void* ws, size_t ws_bytes, cudaStream_t st);
 // Step 6 for many queries per sequence: tiles of 128 queries x 128 keys on the tensor cores with
-// the selections as bit masks (masks: sparse_attn_qtile_bytes of device memory).
+// the selections as bit masks (ws: sparse_attn_qtile_bytes of device memory for the masks and an
+// fp16 copy of V).
 bool sparse_attn_qtile_eligible(const Shape& s);
 size_t sparse_attn_qtile_bytes(const Shape& s);
 cudaError_t launch_sparse_attn_qtile(const Shape& s, const void* q, const void* k, const void* v,
-                                     const int32_t* token_idx, void* o, float* lse, int32_t* status, void* masks,
+                                     const int32_t* token_idx, void* o, float* lse, int32_t* status, void* ws,
                                      cudaStream_t st);
 // Merge of the per-split (max, sum, output) states into O and the LSE.
 cudaError_t launch_attn_merge(const Shape& s, const float* partial, void* o, float* lse, int splits, cudaStream_t st);

@@ -20,26 +20,38 @@
 // entry t of a row's list that lies in [0, p] and exceeds every in-range entry
 // before it; -1 entries are padding; other entries are skipped and flagged.
 //
-// Roles of the attention CTA (224 threads):
-//   * warps 0-3, one thread per query row (TMEM lane = row): first the row's
-//     q into tensor memory (the A operand of the score MMA); then per key
-//     tile read the row's 128 scores, mask them, raise the running max lazily
-//     (O in TMEM is rescaled only when a weight would exceed 2^8), write the
-//     weights over the scores, and at the end write O / l and the LSE;
-//   * warp 4, one thread: TMA loads of the K tiles into a ring of three slots,
-//     a slot refilled as soon as its score MMA has read it;
-//   * warp 6, one thread: TMA loads of the V tiles and 2 KB mask blocks into a
-//     ring of three slots, refilled once the output MMA has read them;
-//   * warp 5, one thread: S_j = Q K_jᵀ into one of two TMEM buffers
-//     (tcgen05.mma kind::f16, M = 128 queries, N = 128 keys, q from tensor
-//     memory), then O += P_{j-1} V_{j-1} (M = 128 queries, N = 128
-//     dimensions; V read MN-major from its rows) with the weights P as the A
-//     operand in tensor memory, in the buffer their scores came from: the
-//     weights carry ~16 significant bits as a bf16 pair hi + lo (hi the upper
-//     half of the fp32 weight, lo the rounded rest), so the output MMA runs
-//     over K = 2 x 128 (hi columns, then lo columns, both against the same V
-//     rows).  MMAs of one thread run in issue order, so S_{j+2} is written
-//     into the buffer only after P_j has been read from it.
+// Roles of the attention CTA (352 threads):
+//   * warps 0-7, two threads per query row (TMEM lane = row; warp w reads the
+//     lanes of quarter w % 4 and the key columns of half w / 4): per key tile
+//     read the row's 64 scores of the half, mask them, exchange the
+//     two halves' maxima through shared memory (one named barrier per tile,
+//     which also carries the error flags, so every thread passes the same
+//     barriers), raise the running max lazily (O in TMEM is rescaled only when
+//     a weight would exceed 2^8), write the weights over the scores, and at the
+//     end write O / l and the LSE;
+//   * warp 8, one thread: TMA loads of the query tile (once) and of the K
+//     tiles into a ring of three slots, a slot refilled as soon as its score
+//     MMA has read it;
+//   * warp 10, one thread: TMA loads of the V tiles and 2 KB mask blocks into a
+//     ring of two slots, refilled once the output MMA has read them;
+//   * warp 9, one thread: S_j = Q K_jᵀ into one of three TMEM buffers
+//     (tcgen05.mma kind::f16, bf16, M = 128 queries, N = 128 keys), and
+//     O += P_j V_j (fp16, M = 128 queries, N = 128 dimensions; V read MN-major
+//     from its rows) with the weights P as the A operand in tensor memory, in
+//     the buffer their scores came from.  The scores run three tiles ahead:
+//     S_{j+3} is issued right after O += P_j V_j, into the buffer P_j was just
+//     read from (MMAs of one thread run in issue order), so the softmax never
+//     waits for its next scores behind an output MMA.
+//
+// Precision of the output MMA: the weights (at most 2^8 with the lazy max)
+// are rounded to fp16, 11 significant bits, so a row's output moves by at most
+// 2^-11 * max |v| (rows normalised by the fp32 sum of the unrounded weights).
+// V enters as fp16 too (both operands of one MMA have one type): a pre-pass
+// (attn_v_max_kernel, attn_v_half_kernel) converts it exactly, scaled per KV
+// head by a power of two 2^-e that brings the head's largest |v| below 2^15;
+// the output is multiplied back by 2^e.  bf16 has 8 significant bits, so the
+// conversion is exact apart from values that fall below fp16's normal range,
+// which lose less than 2^-25 of the head's largest |v|.
 // Every wait is bounded (1 s): a timeout sets status bit 1 and the CTA stops.
 #include <math.h>
 
@@ -68,29 +80,34 @@ using namespace tc;
 
 constexpr int kRows = 128;  // queries per tile = keys per key tile
 constexpr int kD = 128;     // head dimension
-constexpr int kNS = 3;      // slots of the K ring and of the V ring
-constexpr int kThreads = 224;
-constexpr int kWarpK = 4, kWarpMMA = 5, kWarpV = 6;
-// Tensor memory: scores / weights buffer 0 at columns 0-127, buffer 1 at 128-255, output O at
-// 256-383, the query tile (bf16 pairs) at 384-447.
+constexpr int kNK = 3;      // K ring slots
+constexpr int kNV = 2;      // V ring slots (each with its key tile's masks)
+constexpr int kNB = 3;      // score / weight buffers in tensor memory
+constexpr int kSoftmax = 256;  // softmax threads: warps 0-7
+constexpr int kThreads = kSoftmax + 96;
+constexpr int kWarpK = 8, kWarpMMA = 9, kWarpV = 10;
+// Tensor memory: scores / weights buffer i at columns 128 i (i < 3), output O at 384-511.
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 256, kColQ = 384;
+constexpr uint32_t kColO = 384;
 
 constexpr int kHalf = kRows * 128;      // 64 columns of 128 rows of bf16 (one 128-byte swizzle span): 16 KB
 constexpr int kTile = 2 * kHalf;        // a 128 x 128 bf16 tile as two column halves
 constexpr int kMaskBytes = kRows * 16;  // 128 rows x 128 bits
-constexpr int K_OFF = 0;                        // K slot i at K_OFF + i * kTile
-constexpr int V_OFF = K_OFF + kNS * kTile;      // V slot i at V_OFF + i * kTile
-constexpr int MASK_OFF = V_OFF + kNS * kTile;   // mask of V slot i at MASK_OFF + i * kMaskBytes
-constexpr int BAR_OFF = MASK_OFF + kNS * kMaskBytes;
+constexpr int Q_OFF = 0;
+constexpr int K_OFF = Q_OFF + kTile;            // K slot i at K_OFF + i * kTile
+constexpr int V_OFF = K_OFF + kNK * kTile;      // V slot i at V_OFF + i * kTile
+constexpr int MASK_OFF = V_OFF + kNV * kTile;   // mask of V slot i at MASK_OFF + i * kMaskBytes
+constexpr int RED_OFF = MASK_OFF + kNV * kMaskBytes;  // [2][2][128] maxima, [2][8] errors, [2][128] sums, [8] errors
+constexpr int RED_FLOATS = 2 * 2 * kRows + 2 * 8 + 2 * kRows + 8;
+constexpr int BAR_OFF = (RED_OFF + RED_FLOATS * 4 + 7) & ~7;
 enum : int {
   B_KFULL = 0,
-  B_KEMPTY = kNS,
-  B_VFULL = 2 * kNS,
-  B_VEMPTY = 3 * kNS,
-  B_QREADY = 4 * kNS,
-  B_SFULL,  // [2]
-  B_PREADY = B_SFULL + 2,
+  B_KEMPTY = kNK,
+  B_VFULL = 2 * kNK,
+  B_VEMPTY = 2 * kNK + kNV,
+  B_QFULL = 2 * kNK + 2 * kNV,
+  B_SFULL,  // [kNB]
+  B_PREADY = B_SFULL + kNB,
   B_PFREE,
   B_DRAIN,
   kNBar
@@ -98,7 +115,7 @@ enum : int {
 constexpr int MISC_OFF = BAR_OFF + kNBar * 8;
 constexpr int kSmem = MISC_OFF + 16 + 1024;  // + slack for the 1024-byte alignment of the swizzled tiles
 static_assert(kSmem <= 227 * 1024, "shared memory budget");
-static_assert(V_OFF % 1024 == 0 && kTile % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
+static_assert(K_OFF % 1024 == 0 && V_OFF % 1024 == 0 && kTile % 1024 == 0, "swizzle atoms stay 1024-byte aligned");
 
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
@@ -106,14 +123,31 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// Packed pairs of fp32 (sm_100 f32x2 instructions): a * b + c, a + b.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(r)
+      : "l"(*reinterpret_cast<uint64_t*>(&a)), "l"(*reinterpret_cast<uint64_t*>(&b)),
+        "l"(*reinterpret_cast<uint64_t*>(&c)));
+  return *reinterpret_cast<float2*>(&r);
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  uint64_t r;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(r) : "l"(*reinterpret_cast<uint64_t*>(&a)), "l"(*reinterpret_cast<uint64_t*>(&b)));
+  return *reinterpret_cast<float2*>(&r);
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+__device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kSoftmax) : "memory"); }
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&b);
-}
-
-// Upper halves of two fp32 values as a bf16 pair (x0 in the low half): truncation, exact in bf16.
-__device__ __forceinline__ uint32_t pack_hi(float x0, float x1) {
-  return (__float_as_uint(x0) >> 16) | (__float_as_uint(x1) & 0xFFFF0000u);
 }
 
 // Masks of one query tile: [key tile][row] x 128 bits, key tiles 0 .. (last position of the tile) / 128.
@@ -167,10 +201,60 @@ __global__ void __launch_bounds__(kRows) attn_mask_kernel(const int32_t* __restr
   if (bad && status) atomicOr(status, kStatusBadIndex);
 }
 
+// Largest |v| of every KV head of V [rows][Hkv][128] bf16, as the bits of |v| (which order like
+// unsigned integers); blockIdx.y = KV head, 16 threads per 256-byte row slice.  hmax starts at 0.
+__global__ void __launch_bounds__(256) attn_v_max_kernel(const uint16_t* __restrict__ v, int64_t rows, int Hkv,
+                                                         uint32_t* __restrict__ hmax) {
+  __shared__ uint32_t wmax[8];
+  const int hd = blockIdx.y, c = threadIdx.x & 15;
+  uint32_t m = 0;
+  for (int64_t r = (int64_t)blockIdx.x * 16 + (threadIdx.x >> 4); r < rows; r += (int64_t)gridDim.x * 16) {
+    const uint4 x = ld_stream_v4(v + (r * Hkv + hd) * kD + c * 8);
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) m = max(m, max(w[i] & 0x7FFFu, (w[i] >> 16) & 0x7FFFu));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int i = 1; i < 8; ++i) m = max(m, wmax[i]);
+    atomicMax(hmax + hd, m);
+  }
+}
+
+// Exponent e >= 0 with (largest |v| of the head) * 2^-e < 2^15, from the bf16 bits of that |v|.
+__device__ __forceinline__ int v_half_shift(uint32_t vmax_bits) { return max(0, (int)((vmax_bits >> 7) & 0xFFu) - 141); }
+
+// V [rows][Hkv][128] bf16 -> fp16 scaled by 2^-e per head (exact but for values below fp16's normal
+// range); vscale[head] = 2^e.
+__global__ void __launch_bounds__(256) attn_v_half_kernel(const uint16_t* __restrict__ v, uint16_t* __restrict__ vh,
+                                                          int64_t rows, int Hkv, const uint32_t* __restrict__ hmax,
+                                                          float* __restrict__ vscale) {
+  const int hd = blockIdx.y, c = threadIdx.x & 15;
+  const int e = v_half_shift(hmax[hd]);
+  const float sc = __uint_as_float((uint32_t)(127 - e) << 23);
+  if (blockIdx.x == 0 && threadIdx.x == 0) vscale[hd] = __uint_as_float((uint32_t)(127 + e) << 23);
+  for (int64_t r = (int64_t)blockIdx.x * 16 + (threadIdx.x >> 4); r < rows; r += (int64_t)gridDim.x * 16) {
+    const int64_t at = (r * Hkv + hd) * kD + c * 8;
+    const uint4 x = ld_stream_v4(v + at);
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    uint32_t h[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __half2 p = __floats2half2_rn(__uint_as_float(w[i] << 16) * sc, __uint_as_float(w[i] & 0xFFFF0000u) * sc);
+      h[i] = *reinterpret_cast<const uint32_t*>(&p);
+    }
+    *reinterpret_cast<uint4*>(vh + at) = make_uint4(h[0], h[1], h[2], h[3]);
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
-    sparse_attn_qtile_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
-                             const uint16_t* __restrict__ q, const uint4* __restrict__ masks,
-                             uint16_t* __restrict__ o, float* __restrict__ lse, int32_t* __restrict__ status,
+    sparse_attn_qtile_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
+                             const __grid_constant__ CUtensorMap map_v, const uint4* __restrict__ masks,
+                             const float* __restrict__ vscale, uint16_t* __restrict__ o, float* __restrict__ lse,
+                             int32_t* __restrict__ status,
                              int64_t n_q, int64_t n_kv, int H, int Hkv, int batch, int nqt, int nkt, float qscale) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -204,15 +288,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   if (tid == 0) {
-    for (int i = 0; i < kNS; ++i) {
+    for (int i = 0; i < kNK; ++i) {
       mbar_init(bar(B_KFULL + i), 1);
       mbar_init(bar(B_KEMPTY + i), 1);
+    }
+    for (int i = 0; i < kNV; ++i) {
       mbar_init(bar(B_VFULL + i), 1);
       mbar_init(bar(B_VEMPTY + i), 1);
     }
-    mbar_init(bar(B_QREADY), kRows);
-    for (int i = 0; i < 2; ++i) mbar_init(bar(B_SFULL + i), 1);
-    mbar_init(bar(B_PREADY), kRows);
+    mbar_init(bar(B_QFULL), 1);
+    for (int i = 0; i < kNB; ++i) mbar_init(bar(B_SFULL + i), 1);
+    mbar_init(bar(B_PREADY), kSoftmax);
     mbar_init(bar(B_PFREE), 1);
     mbar_init(bar(B_DRAIN), 1);
     *abort_flag = 0;
@@ -224,17 +310,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == kWarpK || warp == kWarpV) {
-    // ---------------- TMA producers: K tiles (warp 4), V tiles + masks (warp 6) ----------------
+    // ---------------- TMA producers: Q and K tiles (warp 8), V tiles + masks (warp 10) ----------------
     if (lane == 0) {
       const bool is_k = warp == kWarpK;
       const CUtensorMap* map = is_k ? &map_k : &map_v;
       const int full = is_k ? B_KFULL : B_VFULL, empty = is_k ? B_KEMPTY : B_VEMPTY;
+      const int ns = is_k ? kNK : kNV;
       const uint32_t base = sb + (uint32_t)(is_k ? K_OFF : V_OFF);
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+      if (is_k) {
+        mbar_expect_tx(bar(B_QFULL), kTile);
+        tma_load_3d(sb + Q_OFF, &map_q, 0, h, (int)row0, bar(B_QFULL));
+        tma_load_3d(sb + Q_OFF + kHalf, &map_q, 64, h, (int)row0, bar(B_QFULL));
+      }
       int issued = 0;
       for (int j = 0; j < nv; ++j) {
-        const int s = j % kNS;
-        if (j >= kNS && !mbar_wait_or_abort(bar(empty + s), ((j / kNS) - 1) & 1, abort_flag)) {
+        const int s = j % ns;
+        if (j >= ns && !mbar_wait_or_abort(bar(empty + s), ((j / ns) - 1) & 1, abort_flag)) {
           fail();
           break;
         }
@@ -249,162 +341,177 @@ __global__ void __launch_bounds__(kThreads, 1)
         issued = j + 1;
       }
       // The copies in flight land before the CTA may exit.
-      for (int j = issued > kNS ? issued - kNS : 0; j < issued; ++j) mbar_wait(bar(full + j % kNS), (j / kNS) & 1);
+      if (is_k) mbar_wait(bar(B_QFULL), 0);
+      for (int j = issued > ns ? issued - ns : 0; j < issued; ++j) mbar_wait(bar(full + j % ns), (j / ns) & 1);
     }
   } else if (warp == kWarpMMA) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);  // q (tensor memory), K K-major
-      constexpr uint32_t kIdO = idesc_bf16(128, 128, false, true);   // P (tensor memory), V MN-major
-      bool ok = mbar_wait_or_abort(bar(B_QREADY), 0, abort_flag);
-      for (int j = 0; ok && j <= nv; ++j) {
-        if (j < nv) {
-          // Buffer j & 1 held P_{j-2}, whose output MMA was issued before this one.
-          const int s = j % kNS;
-          ok = mbar_wait_or_abort(bar(B_KFULL + s), (j / kNS) & 1, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t kt = sb + (uint32_t)(K_OFF + s * kTile);
+      constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);  // Q and K both K-major
+      constexpr uint32_t kIdO = idesc_f16(128, 128, false, true);    // P (tensor memory), V MN-major: fp16
+      // S_j = Q K_jᵀ into buffer j % kNB.
+      auto scores = [&](int j) -> bool {
+        const int s = j % kNK;
+        if (!mbar_wait_or_abort(bar(B_KFULL + s), (j / kNK) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t kt = sb + (uint32_t)(K_OFF + s * kTile);
 #pragma unroll
-          for (int kk = 0; kk < kD / 16; ++kk)
-            umma_bf16_ta(tmem + (uint32_t)((j & 1) * 128), tmem + kColQ + (uint32_t)(8 * kk),
-                         desc_kmajor_sw128(kt + (kk >> 2) * kHalf + (kk & 3) * 32), kIdS, kk > 0 ? 1u : 0u);
-          umma_commit(bar(B_SFULL + (j & 1)));
-          umma_commit(bar(B_KEMPTY + s));
-        }
-        if (j >= 1) {
-          const int jj = j - 1, s = jj % kNS;
-          ok = mbar_wait_or_abort(bar(B_VFULL + s), (jj / kNS) & 1, abort_flag) &&
-               mbar_wait_or_abort(bar(B_PREADY), jj & 1, abort_flag);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t vt = sb + (uint32_t)(V_OFF + s * kTile);
-          const uint32_t pt = tmem + (uint32_t)((jj & 1) * 128);
+        for (int h2 = 0; h2 < 2; ++h2)
 #pragma unroll
-          for (int t = 0; t < 2 * (kRows / 16); ++t)  // keys 16 t' .. 16 t' + 15, t' = t mod 8: hi, then lo
-            umma_bf16_ta(tmem + kColO, pt + (uint32_t)(8 * t), desc_mnmajor_sw128(vt + (t & 7) * 2048, kHalf), kIdO,
-                         (jj > 0 || t > 0) ? 1u : 0u);
-          umma_commit(bar(B_VEMPTY + s));
-          umma_commit(bar(B_PFREE));
-        }
+          for (int kk = 0; kk < 4; ++kk)
+            umma_bf16(tmem + (uint32_t)((j % kNB) * 128), desc_kmajor_sw128(sb + Q_OFF + h2 * kHalf + kk * 32),
+                      desc_kmajor_sw128(kt + h2 * kHalf + kk * 32), kIdS, (h2 | kk) ? 1u : 0u);
+        umma_commit(bar(B_SFULL + j % kNB));
+        umma_commit(bar(B_KEMPTY + s));
+        return true;
+      };
+      bool ok = mbar_wait_or_abort(bar(B_QFULL), 0, abort_flag);
+      for (int j = 0; ok && j < kNB && j < nv; ++j) ok = scores(j);
+      for (int j = 0; ok && j < nv; ++j) {
+        const int s = j % kNV;
+        ok = mbar_wait_or_abort(bar(B_VFULL + s), (j / kNV) & 1, abort_flag) &&
+             mbar_wait_or_abort(bar(B_PREADY), j & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t vt = sb + (uint32_t)(V_OFF + s * kTile);
+        const uint32_t pt = tmem + (uint32_t)((j % kNB) * 128);
+#pragma unroll
+        for (int t = 0; t < kRows / 16; ++t)  // keys 16 t .. 16 t + 15
+          umma_bf16_ta(tmem + kColO, pt + (uint32_t)(8 * t), desc_mnmajor_sw128(vt + t * 2048, kHalf), kIdO,
+                       (j > 0 || t > 0) ? 1u : 0u);
+        umma_commit(bar(B_VEMPTY + s));
+        umma_commit(bar(B_PFREE));
+        if (j + kNB < nv) ok = scores(j + kNB);
       }
       if (!ok) fail();
       umma_commit(bar(B_DRAIN));
       mbar_wait(bar(B_DRAIN), 0);
     }
-  } else if (warp < 4) {
-    // ---------------- softmax and output: warps 0-3, thread = query row ----------------
-    const int r = tid;
-    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
-    {
-      // q of this row (zero past the last query) as bf16 pairs in columns kColQ .. kColQ + 63
-      uint32_t qv[2][32];
-      const uint4* qrow = reinterpret_cast<const uint4*>(q + ((row0 + r) * H + h) * (int64_t)kD);
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const uint4 x = r < nr ? __ldg(qrow + c) : make_uint4(0u, 0u, 0u, 0u);
-        qv[c >> 3][(c & 7) * 4 + 0] = x.x;
-        qv[c >> 3][(c & 7) * 4 + 1] = x.y;
-        qv[c >> 3][(c & 7) * 4 + 2] = x.z;
-        qv[c >> 3][(c & 7) * 4 + 3] = x.w;
-      }
-      tmem_st32_issue(tl + kColQ, qv[0]);
-      tmem_st32_issue(tl + kColQ + 32, qv[1]);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(B_QREADY));
-    }
-    float m_run = -INFINITY;  // running max of the row's selected raw scores
-    float l = 0.f;            // sum of the row's weights, relative to m_run
+  } else if (warp < kSoftmax / 32) {
+    // ---------------- softmax and output: warps 0-7, two threads per query row ----------------
+    const int wq = warp & 3, hf = warp >> 2;  // lane quarter, key / dimension half
+    const int r = wq * 32 + lane;
+    const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
+    volatile float* red_max = reinterpret_cast<volatile float*>(smem + RED_OFF);  // [2][2][kRows]
+    volatile float* red_err = red_max + 2 * 2 * kRows;                             // [2][8]
+    volatile float* red_sum = red_err + 2 * 8;                                     // [2][kRows]
+    volatile float* red_err2 = red_sum + 2 * kRows;                                // [8]
+    float m_run = -INFINITY;   // running max of the row's selected raw scores (the same in both halves)
+    float2 l2 = {0.f, 0.f};    // this half's sum of weights, relative to m_run
     const float lim = 8.f / qscale;
+    const float2 qs2 = {qscale, qscale};
     bool err = false;
     for (int j = 0; j < nv; ++j) {
-      const int s = j % kNS, b = j & 1;
-      const bool ok = mbar_wait_or_abort(bar(B_VFULL + s), (j / kNS) & 1, abort_flag) &&
-                      mbar_wait_or_abort(bar(B_SFULL + b), (j >> 1) & 1, abort_flag);
-      if (!__all_sync(0xFFFFFFFFu, ok)) {
+      const int s = j % kNV, b = j % kNB, pb = j & 1;  // V / mask slot, TMEM buffer, exchange buffer
+      bool ok = !err && mbar_wait_or_abort(bar(B_VFULL + s), (j / kNV) & 1, abort_flag) &&
+                mbar_wait_or_abort(bar(B_SFULL + b), (j / kNB) & 1, abort_flag);
+      ok = __all_sync(0xFFFFFFFFu, ok);
+      float sv[64];
+      float pmax = -INFINITY;
+      if (ok) {
+        tc_fence_after();
+        {
+          uint32_t raw[2][32];
+          tmem_ld32_issue(tl + (uint32_t)(b * 128 + 64 * hf), raw[0]);
+          tmem_ld32_issue(tl + (uint32_t)(b * 128 + 64 * hf + 32), raw[1]);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 64; ++c) sv[c] = __uint_as_float(raw[c >> 5][c & 31]);
+        }
+        const uint2 mk = *reinterpret_cast<const uint2*>(smem + MASK_OFF + s * kMaskBytes + r * 16 + 8 * hf);
+        const uint32_t mw[2] = {mk.x, mk.y};
+#pragma unroll
+        for (int c = 0; c < 64; ++c) sv[c] = ((mw[c >> 5] >> (c & 31)) & 1u) ? sv[c] : -INFINITY;
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int c = 0; c < 64; c += 8)
+#pragma unroll
+          for (int a4 = 0; a4 < 4; ++a4) m4[a4] = fmax3(m4[a4], sv[c + 2 * a4], sv[c + 2 * a4 + 1]);
+        pmax = fmax3(fmaxf(m4[0], m4[1]), m4[2], m4[3]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) sv[c] = -INFINITY;
+      }
+      // Both halves' maxima and every warp's error flag, then one decision for all softmax threads.
+      red_max[(pb * 2 + hf) * kRows + r] = pmax;
+      if (lane == 0) red_err[pb * 8 + warp] = ok ? 0.f : 1.f;
+      softmax_sync();
+      float e = 0.f;
+#pragma unroll
+      for (int w8 = 0; w8 < 8; ++w8) e += red_err[pb * 8 + w8];
+      if (e != 0.f) {
         err = true;
         break;
       }
-      tc_fence_after();
-      float sv[kRows];
-      {
-        uint32_t raw[4][32];
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) tmem_ld32_issue(tl + (uint32_t)(b * 128 + 32 * c4), raw[c4]);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < kRows; ++c) sv[c] = __uint_as_float(raw[c >> 5][c & 31]);
-      }
-      const uint4 mk = *reinterpret_cast<const uint4*>(smem + MASK_OFF + s * kMaskBytes + r * 16);
-      const uint32_t mw[4] = {mk.x, mk.y, mk.z, mk.w};
-      float tmax = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < kRows; ++c) {
-        sv[c] = ((mw[c >> 5] >> (c & 31)) & 1u) ? sv[c] : -INFINITY;
-        tmax = fmaxf(tmax, sv[c]);
-      }
+      const float tmax = fmaxf(pmax, red_max[(pb * 2 + (hf ^ 1)) * kRows + r]);
       float alpha = 1.f;
       bool resc = false;
       if (tmax > m_run + lim) {  // also the first selected entry of the row (m_run = -inf)
         if (m_run != -INFINITY) {
           alpha = exp2f((m_run - tmax) * qscale);
-          l *= alpha;
+          l2.x *= alpha;
+          l2.y *= alpha;
           resc = true;
         }
         m_run = tmax;
       }
-      if (__any_sync(0xFFFFFFFFu, resc)) {  // O holds earlier tiles: rescale it once they are in
-        const bool ok2 = mbar_wait_or_abort(bar(B_PFREE), (j - 1) & 1, abort_flag);
-        if (!__all_sync(0xFFFFFFFFu, ok2)) {
-          err = true;
-          break;
-        }
-        tc_fence_after();
+      if (__any_sync(0xFFFFFFFFu, resc)) {  // O holds earlier tiles: rescale this half once they are in
+        const bool ok2 = __all_sync(0xFFFFFFFFu, mbar_wait_or_abort(bar(B_PFREE), (j - 1) & 1, abort_flag));
+        if (ok2) {
+          tc_fence_after();
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          uint32_t ov[32];
-          tmem_ld32_issue(tl + kColO + 32 * c4, ov);
-          tmem_wait_ld();
+          for (int c2 = 0; c2 < 2; ++c2) {
+            uint32_t ov[32];
+            tmem_ld32_issue(tl + kColO + 64 * hf + 32 * c2, ov);
+            tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-          tmem_st32_issue(tl + kColO + 32 * c4, ov);
+            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+            tmem_st32_issue(tl + kColO + 64 * hf + 32 * c2, ov);
+          }
+          tmem_wait_st();
+        } else {
+          err = true;  // reported at the next exchange
         }
+      }
+      if (!err) {
+        const float nmq = m_run == -INFINITY ? 0.f : -m_run * qscale;
+        const float2 nmq2 = {nmq, nmq};
+        // Weights over the scores of buffer b: keys 64 hf + 2 i, + 1 as the fp16 pair in column 32 hf + i.
+        uint32_t pw[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float2 x = ffma2(make_float2(sv[2 * i], sv[2 * i + 1]), qs2, nmq2);
+          const float2 p = make_float2(fast_exp2(x.x), fast_exp2(x.y));  // 0 where masked
+          l2 = fadd2(l2, p);
+          const __half2 ph = __floats2half2_rn(p.x, p.y);
+          pw[i] = *reinterpret_cast<const uint32_t*>(&ph);
+        }
+        tmem_st32_issue(tl + (uint32_t)(b * 128 + 32 * hf), pw);
         tmem_wait_st();
       }
-      const float nmq = m_run == -INFINITY ? 0.f : -m_run * qscale;
-      // Weights over the scores of buffer b: hi pairs in columns 0-63, lo pairs in 64-127.
-#pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        uint32_t hi[16], lo[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = fast_exp2(fmaf(sv[32 * c4 + 2 * i], qscale, nmq));  // 0 where masked
-          const float p1 = fast_exp2(fmaf(sv[32 * c4 + 2 * i + 1], qscale, nmq));
-          l += p0 + p1;
-          hi[i] = pack_hi(p0, p1);
-          lo[i] = pack_bf16(p0 - __uint_as_float(__float_as_uint(p0) & 0xFFFF0000u),
-                            p1 - __uint_as_float(__float_as_uint(p1) & 0xFFFF0000u));
-        }
-        tmem_st16_issue(tl + (uint32_t)(b * 128 + 16 * c4), hi);
-        tmem_st16_issue(tl + (uint32_t)(b * 128 + 64 + 16 * c4), lo);
-      }
-      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(B_PREADY));
     }
-    if (!err) {
-      const bool ok = mbar_wait_or_abort(bar(B_PFREE), (nv - 1) & 1, abort_flag);
-      err = !__all_sync(0xFFFFFFFFu, ok);
+    // Both halves' sums, the last output MMA, and the error flags: one more exchange.
+    {
+      const bool ok = __all_sync(0xFFFFFFFFu, !err && mbar_wait_or_abort(bar(B_PFREE), (nv - 1) & 1, abort_flag));
+      red_sum[hf * kRows + r] = l2.x + l2.y;
+      if (lane == 0) red_err2[warp] = ok ? 0.f : 1.f;
+      softmax_sync();
+      float e = 0.f;
+#pragma unroll
+      for (int w8 = 0; w8 < 8; ++w8) e += red_err2[w8];
+      err = e != 0.f;
     }
     if (!err) {
       tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      uint16_t* orow = o + ((row0 + r) * H + h) * (int64_t)kD;
+      const float l = red_sum[r] + red_sum[kRows + r];
+      const float inv = l > 0.f ? vscale[g] / l : 0.f;  // V entered scaled by 1 / vscale
+      uint16_t* orow = o + ((row0 + r) * H + h) * (int64_t)kD + 64 * hf;
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
+      for (int c2 = 0; c2 < 2; ++c2) {
         uint32_t ov[32];
-        tmem_ld32_issue(tl + kColO + 32 * c4, ov);
+        tmem_ld32_issue(tl + kColO + 64 * hf + 32 * c2, ov);
         tmem_wait_ld();
         if (r < nr) {
 #pragma unroll
@@ -414,11 +521,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             w.y = pack_bf16(__uint_as_float(ov[8 * q4 + 2]) * inv, __uint_as_float(ov[8 * q4 + 3]) * inv);
             w.z = pack_bf16(__uint_as_float(ov[8 * q4 + 4]) * inv, __uint_as_float(ov[8 * q4 + 5]) * inv);
             w.w = pack_bf16(__uint_as_float(ov[8 * q4 + 6]) * inv, __uint_as_float(ov[8 * q4 + 7]) * inv);
-            *reinterpret_cast<uint4*>(orow + 32 * c4 + 8 * q4) = w;
+            *reinterpret_cast<uint4*>(orow + 32 * c2 + 8 * q4) = w;
           }
         }
       }
-      if (r < nr && lse)
+      if (r < nr && hf == 0 && lse)
         lse[(row0 + r) * H + h] = l > 0.f ? (m_run * qscale + log2f(l)) * 0.69314718055994531f : -INFINITY;
     }
     if (err && lane == 0) fail();
@@ -439,37 +546,67 @@ int64_t n_tiles(int64_t n) { return (n + kRows - 1) / kRows; }
 bool sparse_attn_qtile_eligible(const Shape& s) {
   if (!HISA_ATTN_QT || s.d != kD || s.n_q < HISA_ATTN_QT_MIN_NQ) return false;
   if ((int64_t)s.batch * s.n_kv >= ((int64_t)1 << 31) || s.n_query >= ((int64_t)1 << 31)) return false;
-  if ((int64_t)s.H * n_tiles(s.n_q) * s.batch >= ((int64_t)1 << 31)) return false;
+  if ((int64_t)s.H * n_tiles(s.n_q) * s.batch >= ((int64_t)1 << 31) || s.Hkv > 65535) return false;
   const double avg_keys = (double)(s.n_kv - s.n_q) + 0.5 * (double)s.n_q;
   return avg_keys <= (double)HISA_ATTN_QT_RATIO * (double)s.k;
 }
 
-size_t sparse_attn_qtile_bytes(const Shape& s) {
-  return (size_t)s.batch * (size_t)n_tiles(s.n_q) * (size_t)n_tiles(s.n_kv) * kMaskBytes;
+namespace {
+// Workspace of the query-tile path: masks | V in fp16 | per-head max |v| bits | per-head scale.
+struct QtileLayout {
+  size_t masks, vh, hmax, vscale, total;
+};
+QtileLayout qtile_layout(const Shape& s) {
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  QtileLayout L;
+  L.masks = 0;
+  L.vh = up((size_t)s.batch * (size_t)n_tiles(s.n_q) * (size_t)n_tiles(s.n_kv) * kMaskBytes);
+  L.hmax = L.vh + up((size_t)s.batch * s.n_kv * s.Hkv * kD * 2);
+  L.vscale = L.hmax + up((size_t)s.Hkv * 4);
+  L.total = L.vscale + up((size_t)s.Hkv * 4);
+  return L;
 }
+}  // namespace
+
+size_t sparse_attn_qtile_bytes(const Shape& s) { return qtile_layout(s).total; }
 
 cudaError_t launch_sparse_attn_qtile(const Shape& s, const void* q, const void* k, const void* v,
-                                     const int32_t* token_idx, void* o, float* lse, int32_t* status, void* masks,
+                                     const int32_t* token_idx, void* o, float* lse, int32_t* status, void* ws,
                                      cudaStream_t st) {
   if (!sparse_attn_qtile_eligible(s)) return cudaErrorNotSupported;
-  CUtensorMap mk, mv;
-  if (!map_bf16_rows_of_head(&mk, k, kD, (uint64_t)s.Hkv, (uint64_t)s.batch * s.n_kv, kRows) ||
-      !map_bf16_rows_of_head(&mv, v, kD, (uint64_t)s.Hkv, (uint64_t)s.batch * s.n_kv, kRows))
+  const QtileLayout L = qtile_layout(s);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  uint4* m = reinterpret_cast<uint4*>(w + L.masks);
+  uint16_t* vh = reinterpret_cast<uint16_t*>(w + L.vh);
+  uint32_t* hmax = reinterpret_cast<uint32_t*>(w + L.hmax);
+  float* vscale = reinterpret_cast<float*>(w + L.vscale);
+  const int64_t rows = (int64_t)s.batch * s.n_kv;
+  CUtensorMap mq, mk, mv;
+  if (!map_rows_of_head(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, kD, (uint64_t)s.H, (uint64_t)s.n_query, kRows) ||
+      !map_rows_of_head(&mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k, kD, (uint64_t)s.Hkv, (uint64_t)rows, kRows) ||
+      !map_rows_of_head(&mv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, vh, kD, (uint64_t)s.Hkv, (uint64_t)rows, kRows))
     return cudaErrorNotSupported;
   const int nqt = (int)n_tiles(s.n_q), nkt = (int)n_tiles(s.n_kv);
-  uint4* m = static_cast<uint4*>(masks);
   attn_mask_kernel<<<dim3((unsigned)nqt, (unsigned)s.batch), kRows, 0, st>>>(token_idx, m, status, s.n_q, s.n_kv, s.k,
                                                                              nqt, nkt);
   cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(hmax, 0, (size_t)s.Hkv * 4, st);
+  if (e != cudaSuccess) return e;
+  const int64_t want = (148 * 8 + s.Hkv - 1) / s.Hkv;  // about eight blocks per SM over all heads
+  const int64_t need = (rows + 15) / 16;
+  const dim3 vgrid((unsigned)(want < need ? want : need), (unsigned)s.Hkv);
+  attn_v_max_kernel<<<vgrid, 256, 0, st>>>(static_cast<const uint16_t*>(v), rows, s.Hkv, hmax);
+  attn_v_half_kernel<<<vgrid, 256, 0, st>>>(static_cast<const uint16_t*>(v), vh, rows, s.Hkv, hmax, vscale);
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = ensure_smem((const void*)sparse_attn_qtile_kernel, kSmem);
   if (e != cudaSuccess) return e;
   const int64_t grid = (int64_t)s.H * nqt * s.batch;
   const float qscale = s.scale * 1.4426950408889634f;
-  sparse_attn_qtile_kernel<<<(unsigned)grid, kThreads, kSmem, st>>>(mk, mv, static_cast<const uint16_t*>(q), m,
-                                                                    static_cast<uint16_t*>(o), lse,
-                                                                    status, s.n_q, s.n_kv, s.H, s.Hkv, s.batch, nqt,
-                                                                    nkt, qscale);
+  sparse_attn_qtile_kernel<<<(unsigned)grid, kThreads, kSmem, st>>>(mq, mk, mv, m, vscale, static_cast<uint16_t*>(o),
+                                                                    lse, status, s.n_q, s.n_kv, s.H, s.Hkv, s.batch,
+                                                                    nqt, nkt, qscale);
   return cudaGetLastError();
 }
 

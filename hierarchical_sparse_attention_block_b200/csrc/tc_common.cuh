@@ -101,6 +101,12 @@ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn) {
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// The same for fp16 x fp16 -> fp32.
+constexpr uint32_t idesc_f16(int M, int N, bool a_mn, bool b_mn) {
+  return (1u << 4) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
 // D[tmem] (+)= A x B, issued by one thread.
 __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                           uint32_t accumulate) {
@@ -266,17 +272,17 @@ inline bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, int esize, const
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// bf16 [rows][heads][cols] (row stride heads * cols elements) with 128-byte swizzle; a box is
+// 16-bit [rows][heads][cols] (row stride heads * cols elements) with 128-byte swizzle; a box is
 // 64 columns of one head for box_r consecutive rows.
-inline bool map_bf16_rows_of_head(CUtensorMap* m, const void* base, uint64_t cols, uint64_t heads, uint64_t rows,
-                                  uint32_t box_r) {
+inline bool map_rows_of_head(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t cols, uint64_t heads,
+                             uint64_t rows, uint32_t box_r) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {cols, heads, rows};
   cuuint64_t strides[2] = {cols * 2, heads * cols * 2};
   cuuint32_t box[3] = {64, 1, box_r};
   cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+  return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }

@@ -14,12 +14,19 @@
 // fit; larger requests are rejected with HISA_ERR_UNSUPPORTED.
 //
 // Set-up: the first call on each device looks up the array's device address
-// (cudaGetSymbolAddress, with that device current) and keeps it; make that
-// first call before any stream capture.  Every call shares the one array and
+// (cudaGetSymbolAddress, with that device current) and keeps it together with
+// the id of the device's current context; make that first call before any
+// stream capture.  A later call checks the context id (two driver queries, no
+// synchronization) and looks the address up again only if the context was
+// replaced (cudaDeviceReset, or the primary context released and retained
+// anew), so the kept address never outlives the context it belongs to.  Every call shares the one array and
 // it keeps the last call's contents: nothing in it needs to start at zero,
 // because the scoring kernel of a call writes every key that the selection
 // kernel of the same call reads.  Calls whose work overlaps on the GPU (other
 // streams, other host threads) race on the array; serialize them.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "hisa.h"
@@ -35,20 +42,46 @@ static __device__ __align__(256) uint8_t g_token_scratch[kNoAllocScratchBytes];
 
 std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxDevices];
+unsigned long long g_scratch_ctx[kMaxDevices];  // id of the context the address belongs to
 
-// Device address of the scratch array on the current device (set up once per device).
+// Id of the calling thread's current context (unique for the life of the process), 0 if unknown.
+unsigned long long current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(f);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of the scratch array on the current device: looked up once per device and
+// context (the runtime makes the device's context current first).
 cudaError_t scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
+  const unsigned long long ctx = g_scratch_ptr[dev] ? current_context_id() : 0;
+  if (!g_scratch_ptr[dev] || ctx == 0 || ctx != g_scratch_ctx[dev]) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_token_scratch);
+    e = cudaGetSymbolAddress(&p, g_token_scratch);  // also makes the device's primary context current
     if (e != cudaSuccess) return e;
     if (!p) return cudaErrorInvalidSymbol;
     g_scratch_ptr[dev] = p;
+    g_scratch_ctx[dev] = current_context_id();
   }
   *out = g_scratch_ptr[dev];
   return cudaSuccess;

@@ -151,12 +151,27 @@ hisa_status_t hisa_token_topk(const hisa_params_t* params, const void* q_idx, co
  * over the entries t of token_idx[s][i] (-1 skipped).  bf16 inputs, fp32
  * accumulation, bf16 output.  An empty list gives o = 0, lse = -inf.
  * lse and dev_status are nullable.  Workspace may be NULL (then every
- * query/head is one work item); with hisa_sparse_attn_workspace_size bytes the
- * token list is split across CTAs when there are few queries (decode). */
+ * query/head is one work item of a gather kernel); with
+ * hisa_sparse_attn_workspace_size bytes the token list is split across CTAs
+ * when there are few queries (decode), and with many queries per sequence and
+ * d = 128 the query-tile kernel runs (tiles of 128 queries x 128 keys on the
+ * tensor cores, each query's tokens as a bit mask over the key tile; its
+ * workspace holds the masks and an fp16 copy of V scaled per KV head by a
+ * power of two, and its weights are rounded to fp16: every output stays
+ * within 2^-11 * max|v| of the exact weighted sum).  hisa_sparse_attn_kernel
+ * tells which kernel a workspace size selects. */
 hisa_status_t hisa_sparse_attn_workspace_size(const hisa_params_t* params, size_t* bytes);
 hisa_status_t sparse_attn_fwd(const hisa_params_t* params, const void* q, const void* k, const void* v,
                               const int32_t* token_idx, void* o, float* lse, int32_t* dev_status, void* workspace,
                               size_t workspace_bytes, cudaStream_t stream);
+
+/* Which step-6 kernel sparse_attn_fwd runs for these parameters and a workspace of
+ * workspace_bytes (0: none): *kind = 1 for the query-tile kernel (many queries per sequence, head
+ * dimension 128: tiles of 128 queries against tiles of 128 keys on the tensor cores, the kept
+ * tokens as bit masks; it needs the full hisa_sparse_attn_workspace_size), 0 for the gather
+ * kernels (each query's kept K/V rows gathered on their own).  No counterpart on the pages: it
+ * tells a caller or a benchmark which kernel, and so which roofline, applies. */
+hisa_status_t hisa_sparse_attn_kernel(const hisa_params_t* params, size_t workspace_bytes, int32_t* kind);
 
 /* Steps 1-6 in one call.  block_idx_out and token_idx_out (nullable) receive
  * the intermediate selections.  Workspace: hisa_forward_workspace_size. */
@@ -229,7 +244,9 @@ hisa_status_t hisa_flat_topk(const hisa_params_t* params, const void* q_idx, con
  * more than 16 MiB of candidate keys (top_m * block * 4 bytes) returns
  * HISA_ERR_UNSUPPORTED.  Nothing is allocated by the call.  The first call on
  * each device looks up the array's device address; make that first call
- * before any stream capture.  All calls share the array: calls that overlap
+ * before any stream capture.  The address is looked up again after the
+ * device's context is replaced (cudaDeviceReset), which a later call detects
+ * by the context's id.  All calls share the array: calls that overlap
  * on the GPU (other streams or host threads) race, so serialize them. */
 hisa_status_t hisa_token_topk_noalloc(const hisa_params_t* params, const void* q_idx, const float* idx_weights,
                                       const void* k_idx, const int32_t* block_idx, int32_t* token_idx,

@@ -137,9 +137,9 @@ def test_workspace_sizes_follow_the_shapes():
     # the attention list is split across CTAs when there are few queries
     assert hs.hisa_sparse_attn_workspace_size(p) > 0
     # many queries per sequence: the query-tile kernel's masks, 128 x 128 bits per (query tile,
-    # key tile), 512 x 512 tiles at 64K
+    # key tile), 512 x 512 tiles at 64K, then an fp16 copy of V and two words per KV head
     big = hs.params(1, 65536, 65536, 128, 128, 64, 2048, 16, 16, 128)
-    assert hs.hisa_sparse_attn_workspace_size(big) == 512 * 512 * 2048
+    assert hs.hisa_sparse_attn_workspace_size(big) == 512 * 512 * 2048 + 65536 * 16 * 128 * 2 + 2 * 256
     # d = 64 has no query-tile kernel and no split lists at this size
     big64 = hs.params(1, 65536, 65536, 128, 128, 64, 2048, 16, 16, 64)
     assert hs.hisa_sparse_attn_workspace_size(big64) == 0
@@ -214,3 +214,19 @@ def test_binding_refuses_tensors_on_the_wrong_side():
         assert err.value.status == hs.HISA_ERR_INVALID_ARG
         assert isinstance(err.value, RuntimeError)
     assert hs._hptr(cpu).value == cpu.data_ptr()
+
+
+def test_sparse_attn_kernel_choice_follows_shape_and_workspace():
+    """hisa_sparse_attn_kernel (host logic only): the query-tile kernel needs d = 128, many queries per
+    sequence and the full workspace; otherwise the gather kernels run."""
+    p = hs.params(1, 65536, 65536, 128, 128, 64, 2048, 16, 16, 128)
+    need = hs.hisa_sparse_attn_workspace_size(p)
+    assert hs.hisa_sparse_attn_kernel(p, need) == hs.ATTN_QTILE
+    assert hs.hisa_sparse_attn_kernel(p, need - 1) == hs.ATTN_GATHER
+    assert hs.hisa_sparse_attn_kernel(p, 0) == hs.ATTN_GATHER
+    decode = hs.params(32, 1, 131072, 128, 128, 64, 2048, 16, 16, 128)
+    assert hs.hisa_sparse_attn_kernel(decode, 1 << 40) == hs.ATTN_GATHER
+    d64 = hs.params(1, 1024, 1024, 64, 64, 4, 128, 1, 1, 64)
+    assert hs.hisa_sparse_attn_kernel(d64, 1 << 40) == hs.ATTN_GATHER
+    with pytest.raises(hs.HisaError):
+        hs.hisa_sparse_attn_kernel(hs.params(1, 8, 8, 64, 64, 4, 8, 3, 2, 128), 0)  # 3 heads on 2 KV heads

@@ -64,3 +64,19 @@ def test_workload_config_names_the_workload(bench):
     c = bench.workload_config(w)
     assert c == {"workload": "cfg", "batch": 2, "n_q": 300, "n_kv": 1000, "d_idx": 64, "block": 64, "top_m": 4,
                  "top_k": 150, "n_heads": 8, "n_kv_heads": 2, "d_head": 128, "n_idx_heads": 4, "needles": 3}
+
+
+@pytest.mark.parametrize("shape", [(1, 300, 300), (3, 200, 777), (1, 65536, 65536), (2, 129, 1000)])
+def test_qtile_flops_count_every_visible_key_tile(bench, shape):
+    """The query-tile kernel's flops: 4 * 128^3 per (query tile, visible key tile, head), the visible
+    key tiles of a query tile being those up to its last query's position; checked against a count
+    over the queries themselves."""
+    b, n_q, n_kv = shape
+    w = Workload("tiles", b, n_q, n_kv, 64, 64, 4, 64, 3, 3, 128)
+    fl, tiles = bench.qtile_flops(w)
+    pos = n_kv - n_q + np.arange(n_q)
+    last_tile = {}
+    for i, p in enumerate(pos):
+        last_tile[i // 128] = max(last_tile.get(i // 128, -1), p // 128)
+    want = sum(t + 1 for t in last_tile.values()) * b * 3
+    assert tiles == want and fl == want * 4 * 128 ** 3
