@@ -20,29 +20,29 @@
 // entry t of a row's list that lies in [0, p] and exceeds every in-range entry
 // before it; -1 entries are padding; other entries are skipped and flagged.
 //
-// Roles of the attention CTA (352 threads):
-//   * warps 0-7, two threads per query row (TMEM lane = row; warp w reads the
-//     lanes of quarter w % 4 and the key columns of half w / 4): per key tile
-//     read the row's 64 scores of the half, mask them, exchange the
-//     two halves' maxima through shared memory (one named barrier per tile,
-//     which also carries the error flags, so every thread passes the same
-//     barriers), raise the running max lazily (O in TMEM is rescaled only when
-//     a weight would exceed 2^8), write the weights over the scores, and at the
-//     end write O / l and the LSE;
-//   * warp 8, one thread: TMA loads of the query tile (once) and of the K
-//     tiles into a ring of three slots, a slot refilled as soon as its score
-//     MMA has read it;
-//   * warp 10, one thread: TMA loads of the V tiles and 2 KB mask blocks into a
-//     ring of two slots, refilled once the output MMA has read them;
-//   * warp 9, one thread: S_j = Q K_jᵀ into one of three TMEM buffers
-//     (tcgen05.mma kind::f16, bf16, M = 128 queries, N = 128 keys), and
-//     O += P_j V_j (fp16, M = 128 queries, N = 128 dimensions; V read MN-major
-//     from its rows) with the weights P as the A operand in tensor memory, in
-//     the buffer their scores came from.  The scores run three tiles ahead:
-//     S_{j+3} is issued right after O += P_j V_j, into the buffer P_j was just
-//     read from (MMAs of one thread run in issue order), so the softmax never
-//     waits for its next scores behind an output MMA.
-//
+// A CTA takes TWO consecutive query tiles A and B of one head (256 queries), so
+// every K/V tile it stages serves 256 queries, and their softmax work
+// alternates with each other's MMAs (ping-pong).  Roles (352 threads):
+//   * warps 0-3 (tile A) and 4-7 (tile B), one thread per query row (TMEM
+//     lane = row, warp w reads the lanes of quarter w % 4): per key tile read
+//     the row's 128 scores, mask them, raise the running max lazily (O in TMEM
+//     is rescaled only when a weight would exceed 2^8), write the weights over
+//     the scores, and at the end write O / l and the LSE;
+//   * warp 8, one thread: TMA loads of both query tiles (once) and of the K
+//     tiles into a ring of two slots, a slot refilled once both score MMAs of
+//     its key tile have read it;
+//   * warp 10, one thread: TMA loads of the V tiles and of both query tiles'
+//     2 KB mask blocks into a ring of two slots, refilled once both output
+//     MMAs of the key tile have read them;
+//   * warp 9, one thread: per key tile j, O_A += P_A(j) V_j, S_A(j+1) =
+//     Q_A K_{j+1}ᵀ, O_B += P_B(j) V_j, S_B(j+1) = Q_B K_{j+1}ᵀ (tcgen05.mma
+//     kind::f16, M = 128 queries, N = 128; scores bf16, outputs fp16 with the
+//     weights P as the A operand in tensor memory, written over the scores
+//     they came from: MMAs of one thread run in issue order, so S_A(j+1)
+//     overwrites P_A(j) only after O_A += P_A(j) V_j has read it).  While the
+//     warps of tile A work on S_A(j), the tensor cores run tile B's MMAs, and
+//     the other way round.  Tensor memory: S_A | S_B | O_A | O_B, 128 columns
+//     each.
 // Precision of the output MMA: the weights (at most 2^8 with the lazy max)
 // are rounded to fp16, 11 significant bits, so a row's output moves by at most
 // 2^-11 * max |v| (rows normalised by the fp32 sum of the unrounded weights).
@@ -80,36 +80,32 @@ using namespace tc;
 
 constexpr int kRows = 128;  // queries per tile = keys per key tile
 constexpr int kD = 128;     // head dimension
-constexpr int kNK = 3;      // K ring slots
-constexpr int kNV = 2;      // V ring slots (each with its key tile's masks)
-constexpr int kNB = 3;      // score / weight buffers in tensor memory
-constexpr int kSoftmax = 256;  // softmax threads: warps 0-7
-constexpr int kThreads = kSoftmax + 96;
+constexpr int kNS = 2;      // slots of the K ring and of the V ring
+constexpr int kThreads = 352;
 constexpr int kWarpK = 8, kWarpMMA = 9, kWarpV = 10;
-// Tensor memory: scores / weights buffer i at columns 128 i (i < 3), output O at 384-511.
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColO = 384;
+// Tensor memory columns of query tile t: scores / weights at col_s(t), output at col_o(t).
+__host__ __device__ constexpr uint32_t col_s(int t) { return 128u * (uint32_t)t; }
+__host__ __device__ constexpr uint32_t col_o(int t) { return 256u + 128u * (uint32_t)t; }
 
-constexpr int kHalf = kRows * 128;      // 64 columns of 128 rows of bf16 (one 128-byte swizzle span): 16 KB
-constexpr int kTile = 2 * kHalf;        // a 128 x 128 bf16 tile as two column halves
+constexpr int kHalf = kRows * 128;      // 64 columns of 128 rows of 16-bit values (one 128-byte swizzle span): 16 KB
+constexpr int kTile = 2 * kHalf;        // a 128 x 128 tile as two column halves
 constexpr int kMaskBytes = kRows * 16;  // 128 rows x 128 bits
-constexpr int Q_OFF = 0;
-constexpr int K_OFF = Q_OFF + kTile;            // K slot i at K_OFF + i * kTile
-constexpr int V_OFF = K_OFF + kNK * kTile;      // V slot i at V_OFF + i * kTile
-constexpr int MASK_OFF = V_OFF + kNV * kTile;   // mask of V slot i at MASK_OFF + i * kMaskBytes
-constexpr int RED_OFF = MASK_OFF + kNV * kMaskBytes;  // [2][2][128] maxima, [2][8] errors, [2][128] sums, [8] errors
-constexpr int RED_FLOATS = 2 * 2 * kRows + 2 * 8 + 2 * kRows + 8;
-constexpr int BAR_OFF = (RED_OFF + RED_FLOATS * 4 + 7) & ~7;
+constexpr int Q_OFF = 0;                        // query tile t at Q_OFF + t * kTile
+constexpr int K_OFF = Q_OFF + 2 * kTile;        // K slot i at K_OFF + i * kTile
+constexpr int V_OFF = K_OFF + kNS * kTile;      // V slot i at V_OFF + i * kTile
+constexpr int MASK_OFF = V_OFF + kNS * kTile;   // masks of V slot i, query tile t at MASK_OFF + (2 i + t) * kMaskBytes
+constexpr int BAR_OFF = MASK_OFF + 2 * kNS * kMaskBytes;
 enum : int {
   B_KFULL = 0,
-  B_KEMPTY = kNK,
-  B_VFULL = 2 * kNK,
-  B_VEMPTY = 2 * kNK + kNV,
-  B_QFULL = 2 * kNK + 2 * kNV,
-  B_SFULL,  // [kNB]
-  B_PREADY = B_SFULL + kNB,
-  B_PFREE,
-  B_DRAIN,
+  B_KEMPTY = kNS,
+  B_VFULL = 2 * kNS,
+  B_VEMPTY = 3 * kNS,
+  B_QFULL = 4 * kNS,
+  B_SFULL,                // [2]: per query tile
+  B_PREADY = B_SFULL + 2, // [2]
+  B_PFREE = B_PREADY + 2, // [2]
+  B_DRAIN = B_PFREE + 2,
   kNBar
 };
 constexpr int MISC_OFF = BAR_OFF + kNBar * 8;
@@ -142,8 +138,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
-
-__device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kSoftmax) : "memory"); }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
@@ -250,12 +244,13 @@ __global__ void __launch_bounds__(256) attn_v_half_kernel(const uint16_t* __rest
   }
 }
 
+// Eleven warps put three on some SM sub-partitions, which caps a thread at 168 registers.
 __global__ void __launch_bounds__(kThreads, 1)
     sparse_attn_qtile_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
                              const __grid_constant__ CUtensorMap map_v, const uint4* __restrict__ masks,
                              const float* __restrict__ vscale, uint16_t* __restrict__ o, float* __restrict__ lse,
-                             int32_t* __restrict__ status,
-                             int64_t n_q, int64_t n_kv, int H, int Hkv, int batch, int nqt, int nkt, float qscale) {
+                             int32_t* __restrict__ status, int64_t n_q, int64_t n_kv, int H, int Hkv, int batch,
+                             int nqt, int nkt, float qscale) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -269,18 +264,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
 
   // Work unit: heads outermost (the CTAs running together read one head's K and V, which the L2
-  // keeps), then query tiles from the longest, then sequences.
-  const int64_t per_head = (int64_t)nqt * batch;
+  // keeps), then pairs of query tiles from the longest, then sequences.
+  const int npair = (nqt + 1) / 2;
+  const int64_t per_head = (int64_t)npair * batch;
   const int h = (int)(blockIdx.x / per_head);
   const int64_t rem = blockIdx.x - (int64_t)h * per_head;
-  const int qt = nqt - 1 - (int)(rem / batch);
+  const int pair = npair - 1 - (int)(rem / batch);
   const int seq = (int)(rem - (rem / batch) * batch);
   const int g = h / (H / Hkv);
-  const int64_t row0 = (int64_t)seq * n_q + (int64_t)qt * kRows;  // first query row of the tile
-  const int nr = (int)min((int64_t)kRows, n_q - (int64_t)qt * kRows);
-  const int64_t pos0 = n_kv - n_q + (int64_t)qt * kRows;            // position of row 0
-  const int nv = (int)((pos0 + nr - 1) / kRows) + 1;                // visible key tiles
-  const uint4* mbase = masks + ((int64_t)seq * nqt + qt) * nkt * kRows;
+  const int ntile = 2 * pair + 1 < nqt ? 2 : 1;  // query tiles of this CTA
+  // Query tile t (0 or 1) of the CTA: first row, rows, visible key tiles (0 for a missing tile B).
+  auto row0_of = [&](int t) { return (int64_t)seq * n_q + (int64_t)(2 * pair + t) * kRows; };
+  auto nr_of = [&](int t) { return (int)min((int64_t)kRows, n_q - (int64_t)(2 * pair + t) * kRows); };
+  auto nv_of = [&](int t) {
+    return t < ntile ? (int)((n_kv - n_q + (int64_t)(2 * pair + t) * kRows + nr_of(t) - 1) / kRows) + 1 : 0;
+  };
+  const int nv0 = nv_of(0), nv1 = nv_of(1);
+  const int nvx = max(nv0, nv1);  // key tiles of the CTA
 
   if (warp == kWarpMMA) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
@@ -288,18 +288,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   if (tid == 0) {
-    for (int i = 0; i < kNK; ++i) {
+    for (int i = 0; i < kNS; ++i) {
       mbar_init(bar(B_KFULL + i), 1);
       mbar_init(bar(B_KEMPTY + i), 1);
-    }
-    for (int i = 0; i < kNV; ++i) {
       mbar_init(bar(B_VFULL + i), 1);
       mbar_init(bar(B_VEMPTY + i), 1);
     }
     mbar_init(bar(B_QFULL), 1);
-    for (int i = 0; i < kNB; ++i) mbar_init(bar(B_SFULL + i), 1);
-    mbar_init(bar(B_PREADY), kSoftmax);
-    mbar_init(bar(B_PFREE), 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(B_SFULL + t), 1);
+      mbar_init(bar(B_PREADY + t), kRows);
+      mbar_init(bar(B_PFREE + t), 1);
+    }
     mbar_init(bar(B_DRAIN), 1);
     *abort_flag = 0;
     mbar_init_fence();
@@ -315,135 +315,147 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool is_k = warp == kWarpK;
       const CUtensorMap* map = is_k ? &map_k : &map_v;
       const int full = is_k ? B_KFULL : B_VFULL, empty = is_k ? B_KEMPTY : B_VEMPTY;
-      const int ns = is_k ? kNK : kNV;
       const uint32_t base = sb + (uint32_t)(is_k ? K_OFF : V_OFF);
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
       if (is_k) {
-        mbar_expect_tx(bar(B_QFULL), kTile);
-        tma_load_3d(sb + Q_OFF, &map_q, 0, h, (int)row0, bar(B_QFULL));
-        tma_load_3d(sb + Q_OFF + kHalf, &map_q, 64, h, (int)row0, bar(B_QFULL));
+        mbar_expect_tx(bar(B_QFULL), ntile * kTile);
+        for (int t = 0; t < ntile; ++t) {
+          tma_load_3d(sb + Q_OFF + t * kTile, &map_q, 0, h, (int)row0_of(t), bar(B_QFULL));
+          tma_load_3d(sb + Q_OFF + t * kTile + kHalf, &map_q, 64, h, (int)row0_of(t), bar(B_QFULL));
+        }
       }
       int issued = 0;
-      for (int j = 0; j < nv; ++j) {
-        const int s = j % ns;
-        if (j >= ns && !mbar_wait_or_abort(bar(empty + s), ((j / ns) - 1) & 1, abort_flag)) {
+      for (int j = 0; j < nvx; ++j) {
+        const int s = j % kNS;
+        if (j >= kNS && !mbar_wait_or_abort(bar(empty + s), ((j / kNS) - 1) & 1, abort_flag)) {
           fail();
           break;
         }
         const uint32_t dst = base + (uint32_t)(s * kTile);
         const int z = (int)((int64_t)seq * n_kv + (int64_t)j * kRows);
-        mbar_expect_tx(bar(full + s), is_k ? kTile : kTile + kMaskBytes);
+        const int nmask = is_k ? 0 : (j < nv0 ? 1 : 0) + (j < nv1 ? 1 : 0);
+        mbar_expect_tx(bar(full + s), kTile + nmask * kMaskBytes);
         tma_load_3d(dst, map, 0, g, z, bar(full + s));
         tma_load_3d(dst + kHalf, map, 64, g, z, bar(full + s));
-        if (!is_k)
-          bulk_load(sb + (uint32_t)(MASK_OFF + s * kMaskBytes), mbase + (int64_t)j * kRows, kMaskBytes,
-                    bar(full + s));
+        if (!is_k) {
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            if (j < (t ? nv1 : nv0)) {
+              const int qt = 2 * pair + t;
+              const uint4* mb = masks + (((int64_t)seq * nqt + qt) * nkt + j) * kRows;
+              bulk_load(sb + (uint32_t)(MASK_OFF + (2 * s + t) * kMaskBytes), mb, kMaskBytes, bar(full + s));
+            }
+          }
+        }
         issued = j + 1;
       }
       // The copies in flight land before the CTA may exit.
       if (is_k) mbar_wait(bar(B_QFULL), 0);
-      for (int j = issued > ns ? issued - ns : 0; j < issued; ++j) mbar_wait(bar(full + j % ns), (j / ns) & 1);
+      for (int j = issued > kNS ? issued - kNS : 0; j < issued; ++j) mbar_wait(bar(full + j % kNS), (j / kNS) & 1);
     }
   } else if (warp == kWarpMMA) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_bf16(128, 128, false, false);  // Q and K both K-major
       constexpr uint32_t kIdO = idesc_f16(128, 128, false, true);    // P (tensor memory), V MN-major: fp16
-      // S_j = Q K_jᵀ into buffer j % kNB.
-      auto scores = [&](int j) -> bool {
-        const int s = j % kNK;
-        if (!mbar_wait_or_abort(bar(B_KFULL + s), (j / kNK) & 1, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t kt = sb + (uint32_t)(K_OFF + s * kTile);
+      // S_t(j) = Q_t K_jᵀ (K_j in its slot already)
+      auto scores = [&](int t, int j) {
+        const uint32_t kt = sb + (uint32_t)(K_OFF + (j % kNS) * kTile);
+        const uint32_t qb = sb + (uint32_t)(Q_OFF + t * kTile);
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            umma_bf16(tmem + (uint32_t)((j % kNB) * 128), desc_kmajor_sw128(sb + Q_OFF + h2 * kHalf + kk * 32),
+            umma_bf16(tmem + col_s(t), desc_kmajor_sw128(qb + h2 * kHalf + kk * 32),
                       desc_kmajor_sw128(kt + h2 * kHalf + kk * 32), kIdS, (h2 | kk) ? 1u : 0u);
-        umma_commit(bar(B_SFULL + j % kNB));
-        umma_commit(bar(B_KEMPTY + s));
-        return true;
+        umma_commit(bar(B_SFULL + t));
       };
-      bool ok = mbar_wait_or_abort(bar(B_QFULL), 0, abort_flag);
-      for (int j = 0; ok && j < kNB && j < nv; ++j) ok = scores(j);
-      for (int j = 0; ok && j < nv; ++j) {
-        const int s = j % kNV;
-        ok = mbar_wait_or_abort(bar(B_VFULL + s), (j / kNV) & 1, abort_flag) &&
-             mbar_wait_or_abort(bar(B_PREADY), j & 1, abort_flag);
-        if (!ok) break;
+      bool ok = mbar_wait_or_abort(bar(B_QFULL), 0, abort_flag) && mbar_wait_or_abort(bar(B_KFULL), 0, abort_flag);
+      if (ok) {
         tc_fence_after();
-        const uint32_t vt = sb + (uint32_t)(V_OFF + s * kTile);
-        const uint32_t pt = tmem + (uint32_t)((j % kNB) * 128);
+        if (nv0 > 0) scores(0, 0);
+        if (nv1 > 0) scores(1, 0);
+        umma_commit(bar(B_KEMPTY));
+      }
+      for (int j = 0; ok && j < nvx; ++j) {
+        const int s = j % kNS;
+        ok = mbar_wait_or_abort(bar(B_VFULL + s), (j / kNS) & 1, abort_flag);
+        const bool next = j + 1 < nvx;
+        bool knext = false;  // K_{j+1} waited for
 #pragma unroll
-        for (int t = 0; t < kRows / 16; ++t)  // keys 16 t .. 16 t + 15
-          umma_bf16_ta(tmem + kColO, pt + (uint32_t)(8 * t), desc_mnmajor_sw128(vt + t * 2048, kHalf), kIdO,
-                       (j > 0 || t > 0) ? 1u : 0u);
-        umma_commit(bar(B_VEMPTY + s));
-        umma_commit(bar(B_PFREE));
-        if (j + kNB < nv) ok = scores(j + kNB);
+        for (int t = 0; t < 2; ++t) {
+          const int nvt = t ? nv1 : nv0;
+          if (!ok || j >= nvt) continue;
+          ok = mbar_wait_or_abort(bar(B_PREADY + t), j & 1, abort_flag);
+          if (!ok) continue;
+          tc_fence_after();
+          const uint32_t vt = sb + (uint32_t)(V_OFF + s * kTile);
+#pragma unroll
+          for (int kk = 0; kk < kRows / 16; ++kk)  // keys 16 kk .. 16 kk + 15
+            umma_bf16_ta(tmem + col_o(t), tmem + col_s(t) + (uint32_t)(8 * kk),
+                         desc_mnmajor_sw128(vt + kk * 2048, kHalf), kIdO, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(bar(B_PFREE + t));
+          if (j + 1 < nvt) {
+            if (!knext) {
+              ok = mbar_wait_or_abort(bar(B_KFULL + (j + 1) % kNS), ((j + 1) / kNS) & 1, abort_flag);
+              if (!ok) continue;
+              tc_fence_after();
+              knext = true;
+            }
+            scores(t, j + 1);
+          }
+        }
+        if (!ok) break;
+        umma_commit(bar(B_VEMPTY + s));                    // V_j and its masks read by both output MMAs
+        if (next) umma_commit(bar(B_KEMPTY + (j + 1) % kNS));  // K_{j+1} read by both score MMAs
       }
       if (!ok) fail();
       umma_commit(bar(B_DRAIN));
       mbar_wait(bar(B_DRAIN), 0);
     }
-  } else if (warp < kSoftmax / 32) {
-    // ---------------- softmax and output: warps 0-7, two threads per query row ----------------
-    const int wq = warp & 3, hf = warp >> 2;  // lane quarter, key / dimension half
-    const int r = wq * 32 + lane;
-    const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
-    volatile float* red_max = reinterpret_cast<volatile float*>(smem + RED_OFF);  // [2][2][kRows]
-    volatile float* red_err = red_max + 2 * 2 * kRows;                             // [2][8]
-    volatile float* red_sum = red_err + 2 * 8;                                     // [2][kRows]
-    volatile float* red_err2 = red_sum + 2 * kRows;                                // [8]
-    float m_run = -INFINITY;   // running max of the row's selected raw scores (the same in both halves)
-    float2 l2 = {0.f, 0.f};    // this half's sum of weights, relative to m_run
+  } else {
+    // ---------------- softmax and output: warps 0-3 tile A, 4-7 tile B, thread = query row ----------------
+    const int t = warp >> 2;
+    const int r = (warp & 3) * 32 + lane;
+    const uint32_t lanes = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t ts = tmem + lanes + col_s(t), to = tmem + lanes + col_o(t);
+    const int nvt = t ? nv1 : nv0;
+    const int64_t row0 = row0_of(t);
+    const int nrt = nr_of(t);
+    float m_run = -INFINITY;  // running max of the row's selected raw scores
+    float2 l2 = {0.f, 0.f};   // sum of the row's weights, relative to m_run
     const float lim = 8.f / qscale;
     const float2 qs2 = {qscale, qscale};
     bool err = false;
-    for (int j = 0; j < nv; ++j) {
-      const int s = j % kNV, b = j % kNB, pb = j & 1;  // V / mask slot, TMEM buffer, exchange buffer
-      bool ok = !err && mbar_wait_or_abort(bar(B_VFULL + s), (j / kNV) & 1, abort_flag) &&
-                mbar_wait_or_abort(bar(B_SFULL + b), (j / kNB) & 1, abort_flag);
-      ok = __all_sync(0xFFFFFFFFu, ok);
-      float sv[64];
-      float pmax = -INFINITY;
-      if (ok) {
-        tc_fence_after();
-        {
-          uint32_t raw[2][32];
-          tmem_ld32_issue(tl + (uint32_t)(b * 128 + 64 * hf), raw[0]);
-          tmem_ld32_issue(tl + (uint32_t)(b * 128 + 64 * hf + 32), raw[1]);
-          tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 64; ++c) sv[c] = __uint_as_float(raw[c >> 5][c & 31]);
-        }
-        const uint2 mk = *reinterpret_cast<const uint2*>(smem + MASK_OFF + s * kMaskBytes + r * 16 + 8 * hf);
-        const uint32_t mw[2] = {mk.x, mk.y};
-#pragma unroll
-        for (int c = 0; c < 64; ++c) sv[c] = ((mw[c >> 5] >> (c & 31)) & 1u) ? sv[c] : -INFINITY;
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-        for (int c = 0; c < 64; c += 8)
-#pragma unroll
-          for (int a4 = 0; a4 < 4; ++a4) m4[a4] = fmax3(m4[a4], sv[c + 2 * a4], sv[c + 2 * a4 + 1]);
-        pmax = fmax3(fmaxf(m4[0], m4[1]), m4[2], m4[3]);
-      } else {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) sv[c] = -INFINITY;
-      }
-      // Both halves' maxima and every warp's error flag, then one decision for all softmax threads.
-      red_max[(pb * 2 + hf) * kRows + r] = pmax;
-      if (lane == 0) red_err[pb * 8 + warp] = ok ? 0.f : 1.f;
-      softmax_sync();
-      float e = 0.f;
-#pragma unroll
-      for (int w8 = 0; w8 < 8; ++w8) e += red_err[pb * 8 + w8];
-      if (e != 0.f) {
+    for (int j = 0; j < nvt; ++j) {
+      const int s = j % kNS;
+      const bool ok = mbar_wait_or_abort(bar(B_VFULL + s), (j / kNS) & 1, abort_flag) &&
+                      mbar_wait_or_abort(bar(B_SFULL + t), j & 1, abort_flag);
+      if (!__all_sync(0xFFFFFFFFu, ok)) {
         err = true;
         break;
       }
-      const float tmax = fmaxf(pmax, red_max[(pb * 2 + (hf ^ 1)) * kRows + r]);
+      tc_fence_after();
+      // Pass 1, 32 columns at a time: mask the scores (-inf where the row did not keep the key),
+      // write them back over the scores, and take their max.
+      const uint4 mk = *reinterpret_cast<const uint4*>(smem + MASK_OFF + (2 * s + t) * kMaskBytes + r * 16);
+      const uint32_t mw[4] = {mk.x, mk.y, mk.z, mk.w};
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+        uint32_t raw[32];
+        tmem_ld32_issue(ts + (uint32_t)(32 * c4), raw);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 32; ++c) raw[c] = ((mw[c4] >> c) & 1u) ? raw[c] : 0xFF800000u;  // -inf
+#pragma unroll
+        for (int c = 0; c < 32; c += 8)
+#pragma unroll
+          for (int a4 = 0; a4 < 4; ++a4)
+            m4[a4] = fmax3(m4[a4], __uint_as_float(raw[c + 2 * a4]), __uint_as_float(raw[c + 2 * a4 + 1]));
+        tmem_st32_issue(ts + (uint32_t)(32 * c4), raw);
+      }
+      const float tmax = fmax3(fmaxf(m4[0], m4[1]), m4[2], m4[3]);
       float alpha = 1.f;
       bool resc = false;
       if (tmax > m_run + lim) {  // also the first selected entry of the row (m_run = -inf)
@@ -455,65 +467,59 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         m_run = tmax;
       }
-      if (__any_sync(0xFFFFFFFFu, resc)) {  // O holds earlier tiles: rescale this half once they are in
-        const bool ok2 = __all_sync(0xFFFFFFFFu, mbar_wait_or_abort(bar(B_PFREE), (j - 1) & 1, abort_flag));
-        if (ok2) {
-          tc_fence_after();
+      if (__any_sync(0xFFFFFFFFu, resc)) {  // O holds earlier tiles: rescale it once they are in
+        const bool ok2 = __all_sync(0xFFFFFFFFu, mbar_wait_or_abort(bar(B_PFREE + t), (j - 1) & 1, abort_flag));
+        if (!ok2) {
+          err = true;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll 1
+        for (int c8 = 0; c8 < 16; ++c8) {  // 8 columns at a time: the row's scores stay in registers
+          uint32_t ov[8];
+          tmem_ld<8>(to + 8 * c8, ov);
 #pragma unroll
-          for (int c2 = 0; c2 < 2; ++c2) {
-            uint32_t ov[32];
-            tmem_ld32_issue(tl + kColO + 64 * hf + 32 * c2, ov);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-            tmem_st32_issue(tl + kColO + 64 * hf + 32 * c2, ov);
-          }
-          tmem_wait_st();
-        } else {
-          err = true;  // reported at the next exchange
+          for (int i = 0; i < 8; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+          tmem_st<8>(to + 8 * c8, ov);
         }
       }
-      if (!err) {
-        const float nmq = m_run == -INFINITY ? 0.f : -m_run * qscale;
-        const float2 nmq2 = {nmq, nmq};
-        // Weights over the scores of buffer b: keys 64 hf + 2 i, + 1 as the fp16 pair in column 32 hf + i.
-        uint32_t pw[32];
+      const float nmq = m_run == -INFINITY ? 0.f : -m_run * qscale;
+      const float2 nmq2 = {nmq, nmq};
+      tmem_wait_st();  // the masked scores are back in tensor memory
+      // Pass 2: weights over the scores, keys 2 i, 2 i + 1 as the fp16 pair in column i (columns
+      // 16 c4 .. 16 c4 + 15 are written only after columns 32 c4 .. 32 c4 + 31 have been read).
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float2 x = ffma2(make_float2(sv[2 * i], sv[2 * i + 1]), qs2, nmq2);
+      for (int c4 = 0; c4 < 4; ++c4) {
+        uint32_t raw[32];
+        tmem_ld32_issue(ts + (uint32_t)(32 * c4), raw);
+        tmem_wait_ld();
+        uint32_t pw[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float2 x = ffma2(make_float2(__uint_as_float(raw[2 * i]), __uint_as_float(raw[2 * i + 1])), qs2, nmq2);
           const float2 p = make_float2(fast_exp2(x.x), fast_exp2(x.y));  // 0 where masked
           l2 = fadd2(l2, p);
           const __half2 ph = __floats2half2_rn(p.x, p.y);
           pw[i] = *reinterpret_cast<const uint32_t*>(&ph);
         }
-        tmem_st32_issue(tl + (uint32_t)(b * 128 + 32 * hf), pw);
-        tmem_wait_st();
+        tmem_st16_issue(ts + (uint32_t)(16 * c4), pw);
       }
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(B_PREADY));
+      mbar_arrive(bar(B_PREADY + t));
     }
-    // Both halves' sums, the last output MMA, and the error flags: one more exchange.
-    {
-      const bool ok = __all_sync(0xFFFFFFFFu, !err && mbar_wait_or_abort(bar(B_PFREE), (nv - 1) & 1, abort_flag));
-      red_sum[hf * kRows + r] = l2.x + l2.y;
-      if (lane == 0) red_err2[warp] = ok ? 0.f : 1.f;
-      softmax_sync();
-      float e = 0.f;
-#pragma unroll
-      for (int w8 = 0; w8 < 8; ++w8) e += red_err2[w8];
-      err = e != 0.f;
-    }
-    if (!err) {
+    if (!err && nvt > 0) err = !__all_sync(0xFFFFFFFFu, mbar_wait_or_abort(bar(B_PFREE + t), (nvt - 1) & 1, abort_flag));
+    if (!err && nvt > 0) {
       tc_fence_after();
-      const float l = red_sum[r] + red_sum[kRows + r];
+      const float l = l2.x + l2.y;
       const float inv = l > 0.f ? vscale[g] / l : 0.f;  // V entered scaled by 1 / vscale
-      uint16_t* orow = o + ((row0 + r) * H + h) * (int64_t)kD + 64 * hf;
+      uint16_t* orow = o + ((row0 + r) * H + h) * (int64_t)kD;
 #pragma unroll
-      for (int c2 = 0; c2 < 2; ++c2) {
+      for (int c4 = 0; c4 < 4; ++c4) {
         uint32_t ov[32];
-        tmem_ld32_issue(tl + kColO + 64 * hf + 32 * c2, ov);
+        tmem_ld32_issue(to + 32 * c4, ov);
         tmem_wait_ld();
-        if (r < nr) {
+        if (r < nrt) {
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
             uint4 w;
@@ -521,11 +527,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             w.y = pack_bf16(__uint_as_float(ov[8 * q4 + 2]) * inv, __uint_as_float(ov[8 * q4 + 3]) * inv);
             w.z = pack_bf16(__uint_as_float(ov[8 * q4 + 4]) * inv, __uint_as_float(ov[8 * q4 + 5]) * inv);
             w.w = pack_bf16(__uint_as_float(ov[8 * q4 + 6]) * inv, __uint_as_float(ov[8 * q4 + 7]) * inv);
-            *reinterpret_cast<uint4*>(orow + 32 * c2 + 8 * q4) = w;
+            *reinterpret_cast<uint4*>(orow + 32 * c4 + 8 * q4) = w;
           }
         }
       }
-      if (r < nr && hf == 0 && lse)
+      if (r < nrt && lse)
         lse[(row0 + r) * H + h] = l > 0.f ? (m_run * qscale + log2f(l)) * 0.69314718055994531f : -INFINITY;
     }
     if (err && lane == 0) fail();
@@ -546,7 +552,7 @@ int64_t n_tiles(int64_t n) { return (n + kRows - 1) / kRows; }
 bool sparse_attn_qtile_eligible(const Shape& s) {
   if (!HISA_ATTN_QT || s.d != kD || s.n_q < HISA_ATTN_QT_MIN_NQ) return false;
   if ((int64_t)s.batch * s.n_kv >= ((int64_t)1 << 31) || s.n_query >= ((int64_t)1 << 31)) return false;
-  if ((int64_t)s.H * n_tiles(s.n_q) * s.batch >= ((int64_t)1 << 31) || s.Hkv > 65535) return false;
+  if ((int64_t)s.H * ((n_tiles(s.n_q) + 1) / 2) * s.batch >= ((int64_t)1 << 31) || s.Hkv > 65535) return false;
   const double avg_keys = (double)(s.n_kv - s.n_q) + 0.5 * (double)s.n_q;
   return avg_keys <= (double)HISA_ATTN_QT_RATIO * (double)s.k;
 }
@@ -602,7 +608,7 @@ cudaError_t launch_sparse_attn_qtile(const Shape& s, const void* q, const void* 
   if (e != cudaSuccess) return e;
   e = ensure_smem((const void*)sparse_attn_qtile_kernel, kSmem);
   if (e != cudaSuccess) return e;
-  const int64_t grid = (int64_t)s.H * nqt * s.batch;
+  const int64_t grid = (int64_t)s.H * ((nqt + 1) / 2) * s.batch;
   const float qscale = s.scale * 1.4426950408889634f;
   sparse_attn_qtile_kernel<<<(unsigned)grid, kThreads, kSmem, st>>>(mq, mk, mv, m, vscale, static_cast<uint16_t*>(o),
                                                                     lse, status, s.n_q, s.n_kv, s.H, s.Hkv, s.batch,
