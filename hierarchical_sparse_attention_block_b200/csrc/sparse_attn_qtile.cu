@@ -436,10 +436,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      // Pass 1, 32 columns at a time: mask the scores (-inf where the row did not keep the key),
-      // write them back over the scores, and take their max.
       const uint4 mk = *reinterpret_cast<const uint4*>(smem + MASK_OFF + (2 * s + t) * kMaskBytes + r * 16);
       const uint32_t mw[4] = {mk.x, mk.y, mk.z, mk.w};
+      // One pass, 32 columns at a time: mask the scores (-inf where the row did not keep the key),
+      // take their max, and form the weights against the running max so far (kept in registers as
+      // fp16 pairs; keys 2 i, 2 i + 1 -> pair i).  They stand unless this tile raises the max past
+      // the lazy bound, in which case they are formed again below from the scores, which stay in
+      // tensor memory until the weights are written over them.
+      const float nmq0 = m_run == -INFINITY ? 0.f : -m_run * qscale;
+      const float2 nmq0_2 = {nmq0, nmq0};
+      uint32_t pw[64];
+      float2 ls = {0.f, 0.f};
       float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4) {
@@ -453,56 +460,84 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int a4 = 0; a4 < 4; ++a4)
             m4[a4] = fmax3(m4[a4], __uint_as_float(raw[c + 2 * a4]), __uint_as_float(raw[c + 2 * a4 + 1]));
-        tmem_st32_issue(ts + (uint32_t)(32 * c4), raw);
-      }
-      const float tmax = fmax3(fmaxf(m4[0], m4[1]), m4[2], m4[3]);
-      float alpha = 1.f;
-      bool resc = false;
-      if (tmax > m_run + lim) {  // also the first selected entry of the row (m_run = -inf)
-        if (m_run != -INFINITY) {
-          alpha = exp2f((m_run - tmax) * qscale);
-          l2.x *= alpha;
-          l2.y *= alpha;
-          resc = true;
-        }
-        m_run = tmax;
-      }
-      if (__any_sync(0xFFFFFFFFu, resc)) {  // O holds earlier tiles: rescale it once they are in
-        const bool ok2 = __all_sync(0xFFFFFFFFu, mbar_wait_or_abort(bar(B_PFREE + t), (j - 1) & 1, abort_flag));
-        if (!ok2) {
-          err = true;
-          break;
-        }
-        tc_fence_after();
-#pragma unroll 1
-        for (int c8 = 0; c8 < 16; ++c8) {  // 8 columns at a time: the row's scores stay in registers
-          uint32_t ov[8];
-          tmem_ld<8>(to + 8 * c8, ov);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-          tmem_st<8>(to + 8 * c8, ov);
-        }
-      }
-      const float nmq = m_run == -INFINITY ? 0.f : -m_run * qscale;
-      const float2 nmq2 = {nmq, nmq};
-      tmem_wait_st();  // the masked scores are back in tensor memory
-      // Pass 2: weights over the scores, keys 2 i, 2 i + 1 as the fp16 pair in column i (columns
-      // 16 c4 .. 16 c4 + 15 are written only after columns 32 c4 .. 32 c4 + 31 have been read).
-#pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        uint32_t raw[32];
-        tmem_ld32_issue(ts + (uint32_t)(32 * c4), raw);
-        tmem_wait_ld();
-        uint32_t pw[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float2 x = ffma2(make_float2(__uint_as_float(raw[2 * i]), __uint_as_float(raw[2 * i + 1])), qs2, nmq2);
+          const float2 x = ffma2(make_float2(__uint_as_float(raw[2 * i]), __uint_as_float(raw[2 * i + 1])), qs2, nmq0_2);
           const float2 p = make_float2(fast_exp2(x.x), fast_exp2(x.y));  // 0 where masked
-          l2 = fadd2(l2, p);
+          ls = fadd2(ls, p);
           const __half2 ph = __floats2half2_rn(p.x, p.y);
-          pw[i] = *reinterpret_cast<const uint32_t*>(&ph);
+          pw[16 * c4 + i] = *reinterpret_cast<const uint32_t*>(&ph);
         }
-        tmem_st16_issue(ts + (uint32_t)(16 * c4), pw);
+      }
+      const float tmax = fmax3(fmaxf(m4[0], m4[1]), m4[2], m4[3]);
+      const bool raise = tmax > m_run + lim;  // also the first selected entry of the row (m_run = -inf)
+      if (__any_sync(0xFFFFFFFFu, raise)) {
+        float alpha = 1.f;
+        bool resc = false;
+        if (raise) {
+          if (m_run != -INFINITY) {
+            alpha = exp2f((m_run - tmax) * qscale);
+            l2.x *= alpha;
+            l2.y *= alpha;
+            resc = true;
+          }
+          m_run = tmax;
+        }
+        if (__any_sync(0xFFFFFFFFu, resc)) {  // O holds earlier tiles: rescale it once they are in
+          const bool ok2 = __all_sync(0xFFFFFFFFu, mbar_wait_or_abort(bar(B_PFREE + t), (j - 1) & 1, abort_flag));
+          if (!ok2) {
+            err = true;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll 1
+          for (int c8 = 0; c8 < 16; ++c8) {  // 8 columns at a time: the weights stay in registers
+            uint32_t ov[8];
+            tmem_ld<8>(to + 8 * c8, ov);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+            tmem_st<8>(to + 8 * c8, ov);
+          }
+        }
+        // the weights again, against the raised max (rows whose max did not move get the same values)
+        const float nmq = m_run == -INFINITY ? 0.f : -m_run * qscale;
+        const float2 nmq2 = {nmq, nmq};
+        ls = make_float2(0.f, 0.f);
+#pragma unroll 1
+        for (int c4 = 0; c4 < 4; ++c4) {
+          uint32_t raw[32];
+          tmem_ld32_issue(ts + (uint32_t)(32 * c4), raw);
+          tmem_wait_ld();
+          const uint32_t w = c4 == 0 ? mw[0] : c4 == 1 ? mw[1] : c4 == 2 ? mw[2] : mw[3];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float s0 = ((w >> (2 * i)) & 1u) ? __uint_as_float(raw[2 * i]) : -INFINITY;
+            const float s1 = ((w >> (2 * i + 1)) & 1u) ? __uint_as_float(raw[2 * i + 1]) : -INFINITY;
+            const float2 x = ffma2(make_float2(s0, s1), qs2, nmq2);
+            const float2 p = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+            ls = fadd2(ls, p);
+            const __half2 ph = __floats2half2_rn(p.x, p.y);
+            raw[i] = *reinterpret_cast<const uint32_t*>(&ph);
+          }
+          // pw[16 c4 + i] = raw[i]: dynamic indexing of pw would spill it, so the pairs go to tensor
+          // memory here and the store below is skipped for this tile
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pk[i] = raw[i];
+          tmem_st16_issue(ts + (uint32_t)(16 * c4), pk);
+        }
+        l2 = fadd2(l2, ls);
+        tmem_wait_st();
+      } else {
+        l2 = fadd2(l2, ls);
+        // weights over the scores: pairs 0-63 into columns 0-63 (all scores have been read)
+#pragma unroll
+        for (int c2 = 0; c2 < 2; ++c2) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) pk[i] = pw[32 * c2 + i];
+          tmem_st32_issue(ts + (uint32_t)(32 * c2), pk);
+        }
       }
       tmem_wait_st();
       tc_fence_before();
