@@ -5,7 +5,7 @@ One step = one pass of the whole path (block pooling, block scoring + top-m,
 token scoring + top-k, sparse attention) over one batch of synthetic input
 already resident in HBM.  The default workload is the 64K-token prefill
 (1 sequence, B=128, m=64, k=2048, 16 heads of 128); the metric is queries per
-second, with the attention kernel's fraction of the HBM roofline.
+second, with the dominant (attention) kernel's fraction of its roofline.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
@@ -17,9 +17,12 @@ rank's time.
 Besides the device-resident step the line carries: `e2e` (the same metric
 through the public API with the inputs in pinned host memory and O/LSE read
 back: hisa_forward_host for prefill, hisa_forward_cached for decode),
-`roofline` (the attention kernel against the measured copy bandwidth, plus the
-measured L2 or HBM gather ceiling of its access pattern, and the DRAM traffic
-of the committed ncu record when its source hash matches), `cpu_baseline`
+`roofline` (the attention kernel against the bound of the kernel that ran:
+the query-tile kernel's executed flops against the measured sustained bf16
+rate; a gather kernel's gathered bytes against the measured L2 gather ceiling
+(prefill) or the measured copy bandwidth (decode); the gathered bytes over
+HBM as `effective_gbs`, and the DRAM traffic of the committed ncu record when
+its source hash matches), `cpu_baseline`
 (the oracle on the host cores, all cores and one), `clocks`, the flat-indexer
 speedup and the needle recall of the probe query.
 """
