@@ -130,8 +130,8 @@ hisa_status_t run_block_stage(const Shape& s, const void* q_idx, const float* bl
 
 }  // namespace
 
-cudaError_t ensure_smem(const void* func, int bytes) {
-  if (bytes <= 48 * 1024) return cudaSuccess;
+cudaError_t ensure_smem(const void* func, int bytes, int static_bytes) {
+  if (bytes + static_bytes <= 48 * 1024) return cudaSuccess;  // within the default limit
   static std::mutex mu;
   static const void* done_f[64][64];
   static int done_b[64][64];

@@ -203,7 +203,8 @@ cudaError_t launch_block_topm(const Shape& s, const float* scores, int32_t* bloc
   const bool wide = s.n_query < 2 * 148;
   auto kern = wide ? block_topm_kernel<kTopmThreadsWide> : block_topm_kernel<kTopmThreads>;
   const int nt = wide ? kTopmThreadsWide : kTopmThreads;
-  cudaError_t e = ensure_smem((const void*)kern, smem);
+  const int stat = (int)(wide ? sizeof(SelectShared<kTopmThreadsWide>) : sizeof(SelectShared<kTopmThreads>));
+  cudaError_t e = ensure_smem((const void*)kern, smem, stat);
   if (e != cudaSuccess) return e;
   kern<<<(unsigned)s.n_query, nt, smem, st>>>(scores, block_idx, block_scores, s.n_q, s.n_kv, s.B, s.n_blk, s.m,
                                               in_smem);

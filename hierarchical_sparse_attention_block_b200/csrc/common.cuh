@@ -15,7 +15,7 @@ constexpr int kStatusBadIndex = 1;
 // values.  -0 is folded onto +0 first so equal scores get equal keys.  No
 // finite score maps to 0, which therefore marks "no candidate here".
 __device__ __forceinline__ uint32_t score_key(float f) {
-  if (f == 0.0f) f = 0.0f;
+  f = __fadd_rn(f, 0.0f);  // -0 + 0 = +0: both zeros get one key
   const uint32_t u = __float_as_uint(f);
   return u ^ ((u & 0x80000000u) ? 0xFFFFFFFFu : 0x80000000u);
 }

@@ -100,7 +100,8 @@ cudaError_t launch_gather_probe(const void* rows, int64_t n_rows, int row_bytes,
 // cudaError_t value behind the last HISA_ERR_CUDA on this host thread.
 extern thread_local int32_t g_last_cuda_error;
 
-// Dynamic shared memory opt-in, once per (kernel, device).
-cudaError_t ensure_smem(const void* func, int bytes);
+// Raises a kernel's dynamic shared-memory limit to `bytes` (once per device and kernel) when
+// `bytes` plus the kernel's static shared memory exceed the default 48 KiB.
+cudaError_t ensure_smem(const void* func, int bytes, int static_bytes = 0);
 
 }  // namespace hisa

@@ -211,34 +211,58 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ---------------- readout warps ----------------
-    // Slot map of query tid of the tile (threads tid < QT) for blocks jb0 .. jb0+nb-1.
+    // Slot map of query tid of the tile (threads tid < QT) for blocks jb0 .. jb0+nb-1, stored
+    // block-major (smap[jj * kTileQ + query]) so that a warp's 32 queries sit in consecutive halves.
     {
+      uint4* m4 = reinterpret_cast<uint4*>(smap);
+      for (int i = tid; i < L::MAP_BYTES / 16; i += kEpiWarps * 32) m4[i] = make_uint4(~0u, ~0u, ~0u, ~0u);
+      asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
       const int64_t qrow = tq0 + tid;  // global query id
       const bool row_ok = tid < QT && qrow >= t_lo && qrow < t_hi;
       const int64_t p = n_kv - n_q + (qrow - seq * n_q);
       const int64_t c = p / B;
       uint32_t* krow_keys = keys + (qrow - q0) * (int64_t)slots * B;
-      if (tid < QT)
-        for (int jj = 0; jj < kRun; ++jj) smap[tid * kRun + jj] = -1;
       if (row_ok) {
         if (block_idx) {
           const int32_t* lst = block_idx + qrow * slots;
+          // the list in batches of 32 entries, loaded together (16-byte loads when aligned)
+          const bool vec = ((reinterpret_cast<uintptr_t>(lst) & 15) == 0);
           int mx = -1;
-          for (int r = 0; r < slots; ++r) {
-            const int b = lst[r];
-            const bool in_range = b >= 0 && b <= c;
-            const bool ok = in_range && b > mx;
-            if (ok && b >= jb0 && b < jb0 + nb) smap[tid * kRun + (b - jb0)] = (int16_t)r;
-            if (run == 0 && !ok) {
-              if (b != -1 && status) atomicOr(status, kStatusBadIndex);
-              uint4* z = reinterpret_cast<uint4*>(krow_keys + (int64_t)r * B);
-              for (int i = 0; i < B / 4; ++i) z[i] = make_uint4(0, 0, 0, 0);
+#pragma unroll 1
+          for (int r0 = 0; r0 < slots; r0 += 32) {
+            int e[32];
+            if (vec && r0 + 32 <= slots) {
+              const int4* l4 = reinterpret_cast<const int4*>(lst + r0);
+#pragma unroll
+              for (int u = 0; u < 8; ++u) {
+                const int4 t = l4[u];
+                e[4 * u] = t.x;
+                e[4 * u + 1] = t.y;
+                e[4 * u + 2] = t.z;
+                e[4 * u + 3] = t.w;
+              }
+            } else {
+#pragma unroll
+              for (int u = 0; u < 32; ++u) e[u] = r0 + u < slots ? lst[r0 + u] : -1;
             }
-            if (in_range) mx = max(mx, b);
+#pragma unroll
+            for (int u = 0; u < 32; ++u) {
+              const int r = r0 + u;
+              const int b = e[u];
+              const bool in_range = b >= 0 && b <= c;
+              const bool ok = in_range && b > mx;
+              if (ok && b >= jb0 && b < jb0 + nb) smap[(b - jb0) * kTileQ + tid] = (int16_t)r;
+              if (run == 0 && !ok && r < slots) {
+                if (b != -1 && status) atomicOr(status, kStatusBadIndex);
+                uint4* z = reinterpret_cast<uint4*>(krow_keys + (int64_t)r * B);
+                for (int i = 0; i < B / 4; ++i) z[i] = make_uint4(0, 0, 0, 0);
+              }
+              if (in_range) mx = max(mx, b);
+            }
           }
         } else {
           for (int jj = 0; jj < nb; ++jj)
-            if (jb0 + jj <= c) smap[tid * kRun + jj] = (int16_t)(jb0 + jj);
+            if (jb0 + jj <= c) smap[jj * kTileQ + tid] = (int16_t)(jb0 + jj);
           if (run == 0) {  // blocks after the query's own block hold no candidate
             for (int64_t r = c + 1; r < slots; ++r) {
               uint4* z = reinterpret_cast<uint4*>(krow_keys + r * B);
@@ -286,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int qq = 0; qq < kQpc; ++qq) {
             const int ql = cc * kQpc + qq;
             const int64_t qr = tq0 + ql;
-            sl[qq] = (qr >= t_lo && qr < t_hi) ? smap[ql * kRun + b] : -1;  // the same in every lane
+            sl[qq] = (qr >= t_lo && qr < t_hi) ? smap[b * kTileQ + ql] : -1;  // the same in every lane
             any = any || sl[qq] >= 0;
           }
           if (!any) continue;  // warp-uniform
@@ -323,35 +347,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else {
         // rows whose query kept block jb0 + b
-        const int slot = row_ok ? smap[qi * kRun + b] : -1;
+        const int slot = row_ok ? smap[b * kTileQ + qi] : -1;
         if (__any_sync(0xFFFFFFFFu, slot >= 0)) {
           const int64_t j = jb0 + b;
           const int64_t tok0 = j * B;
           uint32_t* dst = krow_keys + (int64_t)(slot < 0 ? 0 : slot) * B;
-  #pragma unroll 1
-          for (int cc = 0; cc < B / 32; ++cc) {
-            uint32_t v[32];
-            const uint32_t addr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(g * B + cc * 32);
-            asm volatile(
-                "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-                "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-                : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-                  "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]),
-                  "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]),
-                  "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]),
-                  "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-                : "r"(addr));
-            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+          // lane 0 holds the warp's first query: a block wholly at or before it needs no causal test
+          const bool whole = tok0 + B - 1 <= __shfl_sync(0xFFFFFFFFu, p, 0);
+          auto chunk = [&](int cc, const uint32_t(&v)[32]) {
             if (HI == 0) {
               if (slot >= 0) {
-  #pragma unroll
+#pragma unroll
                 for (int t = 0; t < 32; t += 4) {
-                  const int64_t tk = tok0 + cc * 32 + t;
                   uint4 w;
-                  w.x = tk <= p ? score_key(__uint_as_float(v[t])) : 0u;
-                  w.y = tk + 1 <= p ? score_key(__uint_as_float(v[t + 1])) : 0u;
-                  w.z = tk + 2 <= p ? score_key(__uint_as_float(v[t + 2])) : 0u;
-                  w.w = tk + 3 <= p ? score_key(__uint_as_float(v[t + 3])) : 0u;
+                  w.x = score_key(__uint_as_float(v[t]));
+                  w.y = score_key(__uint_as_float(v[t + 1]));
+                  w.z = score_key(__uint_as_float(v[t + 2]));
+                  w.w = score_key(__uint_as_float(v[t + 3]));
+                  if (!whole) {
+                    const int64_t tk = tok0 + cc * 32 + t;
+                    w.x = tk <= p ? w.x : 0u;
+                    w.y = tk + 1 <= p ? w.y : 0u;
+                    w.z = tk + 2 <= p ? w.z : 0u;
+                    w.w = tk + 3 <= p ? w.w : 0u;
+                  }
                   *reinterpret_cast<uint4*>(dst + cc * 32 + t) = w;
                 }
               }
@@ -360,16 +379,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               // with a transposing reduction: after it, the lane of head h holds the sums of tokens
               // h * (32 / HE) .. (h + 1) * (32 / HE) - 1 of this chunk.
               float x[32];
-  #pragma unroll
+#pragma unroll
               for (int t = 0; t < 32; ++t) x[t] = wgt * fmaxf(__uint_as_float(v[t]), 0.f);
-  #pragma unroll
+#pragma unroll
               for (int m = 0; m < 4; ++m) {
                 if ((1 << m) < HE) {  // warp-uniform
                   constexpr int kHalfMax = 16;
                   const int half = 16 >> m;
                   const int o = HE >> (m + 1);
                   const bool up = (head & o) != 0;
-  #pragma unroll
+#pragma unroll
                   for (int t = 0; t < kHalfMax; ++t) {
                     if (t < half) {
                       const float send = up ? x[t] : x[t + half];
@@ -381,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
               if (slot >= 0) {
                 const int n = 32 / HE, t0 = head * n;
-  #pragma unroll
+#pragma unroll
                 for (int t = 0; t < 32; ++t) {
                   if (t < n) {
                     const int64_t tk = tok0 + cc * 32 + t0 + t;
@@ -390,6 +409,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
               }
             }
+          };
+          // 32 columns at a time, the load of the next chunk in flight while this one is converted
+          const uint32_t a0 = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(g * B);
+          uint32_t va[32], vb[32];
+          tmem_ld32_issue(a0, va);
+          tmem_wait_ld(va);
+#pragma unroll
+          for (int cc = 0; cc < B / 32; ++cc) {
+            uint32_t(&cur)[32] = (cc & 1) ? vb : va;
+            uint32_t(&nxt)[32] = (cc & 1) ? va : vb;
+            if (cc + 1 < B / 32) tmem_ld32_issue(a0 + (uint32_t)((cc + 1) * 32), nxt);
+            chunk(cc, cur);
+            if (cc + 1 < B / 32) tmem_wait_ld(nxt);
           }
         }
       }

@@ -12,9 +12,10 @@
 //
 // token_score_mh_kernel: the same for the multi-head weighted score.
 //
-// token_select_kernel: one CTA per query; the row of keys is staged in shared
-// memory (when it fits) and a CTA radix selection takes the best
-// min(k, candidates), emitted in ascending token order.
+// token_select_staged_kernel: one CTA per query; the row of keys is staged in
+// shared memory and a CTA radix selection in three wide digits takes the best
+// min(k, candidates), emitted in ascending token order (token_select_kernel:
+// the same for rows too long to stage, from global memory in 8-bit digits).
 #include <math.h>
 
 #include "common.cuh"
@@ -221,14 +222,16 @@ __global__ void __launch_bounds__(kScoreThreads)
   }
 }
 
-// KS: the query's keys are staged in shared memory (else read from global memory each pass).
-template <int NT, bool KS>
+// One CTA per query; the row of keys, read from global memory, is staged in
+// shared memory and the first selection digit counted on the way in (three
+// sweeps of the row in all: staging, the candidate sweep and the emit sweep).
+// V = 4: the row length is a multiple of four (16-byte staging).
+template <int NT, int V>
 __global__ void __launch_bounds__(NT)
-    token_select_kernel(const uint32_t* __restrict__ keys, const int32_t* __restrict__ block_idx, int slots,
-                        int32_t* __restrict__ token_idx, float* __restrict__ token_scores, int64_t n_q, int log2B,
-                        int k, int64_t q0) {
-  constexpr bool keys_in_smem = KS;
-  __shared__ SelectShared<NT> sm;
+    token_select_staged_kernel(const uint32_t* __restrict__ keys, const int32_t* __restrict__ block_idx, int slots,
+                               int32_t* __restrict__ token_idx, float* __restrict__ token_scores, int log2B, int k,
+                               int64_t q0) {
+  __shared__ StagedSelectShared<NT> sm;
   extern __shared__ __align__(16) uint32_t dsm[];
   const int B = 1 << log2B;
   const int64_t lq = blockIdx.x;
@@ -236,39 +239,63 @@ __global__ void __launch_bounds__(NT)
   const int n = slots * B;
   const uint32_t* row = keys + lq * (int64_t)n;
   uint32_t* skeys = dsm;
-  int32_t* sblk = reinterpret_cast<int32_t*>(dsm + (keys_in_smem ? n : 0));
+  int32_t* sblk = reinterpret_cast<int32_t*>(dsm + n);
 
   for (int r = threadIdx.x; r < slots; r += NT) sblk[r] = block_idx ? block_idx[qg * slots + r] : r;
-  int cnt = 0;  // nonzero keys this thread staged
-  if (keys_in_smem) {
-    if ((n & 3) == 0) {
-      const uint4* src = reinterpret_cast<const uint4*>(row);
-      uint4* dst = reinterpret_cast<uint4*>(skeys);
-      for (int i = threadIdx.x; i < n / 4; i += NT) {
-        const uint4 v = src[i];
-        dst[i] = v;
-        cnt += (v.x != 0u) + (v.y != 0u) + (v.z != 0u) + (v.w != 0u);
-      }
-    } else {
-      for (int i = threadIdx.x; i < n; i += NT) {
-        const uint32_t v = row[i];
-        skeys[i] = v;
-        cnt += v != 0u;
-      }
+  for (int i = threadIdx.x; i < kWideBins / 4; i += NT)
+    reinterpret_cast<uint4*>(sm.u.hist)[i] = make_uint4(0u, 0u, 0u, 0u);
+  __syncthreads();
+  if constexpr (V == 4) {
+    const uint4* src = reinterpret_cast<const uint4*>(row);
+    uint4* dst = reinterpret_cast<uint4*>(skeys);
+#pragma unroll 4
+    for (int i = threadIdx.x; i < n / 4; i += NT) {
+      const uint4 v = src[i];
+      dst[i] = v;
+      counts_first_digit(sm.u.hist, v.x);
+      counts_first_digit(sm.u.hist, v.y);
+      counts_first_digit(sm.u.hist, v.z);
+      counts_first_digit(sm.u.hist, v.w);
+    }
+  } else {
+    for (int i = threadIdx.x; i < n; i += NT) {
+      const uint32_t v = row[i];
+      skeys[i] = v;
+      counts_first_digit(sm.u.hist, v);
     }
   }
   __syncthreads();
-  auto key = [&](int i) -> uint32_t {
-    if constexpr (KS)
-      return skeys[i];
-    else
-      return row[i];
-  };
-  int nv;
-  if constexpr (KS)
-    nv = cta_sum<NT>(cnt, sm);  // counted while staging
-  else
-    nv = count_nonzero<NT>(key, n, sm);
+  int32_t* out = token_idx + qg * k;
+  float* osc = token_scores ? token_scores + qg * k : nullptr;
+  const int K = staged_select<NT>(skeys, n, k, sm, [&](int rank, int i, uint32_t key) {
+    out[rank] = sblk[i >> log2B] * B + (i & (B - 1));
+    if (osc) osc[rank] = key_score(key);
+  });
+  for (int r = K + threadIdx.x; r < k; r += NT) {
+    out[r] = -1;
+    if (osc) osc[r] = __int_as_float(0x7FC00000);
+  }
+}
+
+// Rows too long for shared memory: the selection reads the keys from global memory on every pass.
+template <int NT>
+__global__ void __launch_bounds__(NT)
+    token_select_kernel(const uint32_t* __restrict__ keys, const int32_t* __restrict__ block_idx, int slots,
+                        int32_t* __restrict__ token_idx, float* __restrict__ token_scores, int log2B, int k,
+                        int64_t q0) {
+  __shared__ SelectShared<NT> sm;
+  extern __shared__ __align__(16) uint32_t dsm[];
+  const int B = 1 << log2B;
+  const int64_t lq = blockIdx.x;
+  const int64_t qg = q0 + lq;
+  const int n = slots * B;
+  const uint32_t* row = keys + lq * (int64_t)n;
+  int32_t* sblk = reinterpret_cast<int32_t*>(dsm);
+
+  for (int r = threadIdx.x; r < slots; r += NT) sblk[r] = block_idx ? block_idx[qg * slots + r] : r;
+  __syncthreads();
+  auto key = [&](int i) -> uint32_t { return row[i]; };
+  const int nv = count_nonzero<NT>(key, n, sm);
   const int K = min(k, nv);
   int32_t* out = token_idx + qg * k;
   float* osc = token_scores ? token_scores + qg * k : nullptr;
@@ -345,20 +372,30 @@ cudaError_t launch_token_select(const Shape& s, const uint32_t* keys, const int3
                                 int32_t* token_idx, float* token_scores, int64_t q0, int64_t nq, cudaStream_t st) {
   if (nq <= 0) return cudaSuccess;
   const int64_t n = (int64_t)slots * s.B;
-  const int in_smem = n <= kSelectSmemKeys ? 1 : 0;
-  const int smem = (int)((in_smem ? n : 0) * 4 + (int64_t)slots * 4);
-  if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
   int log2B = 0;
   while ((1 << log2B) < s.B) ++log2B;
   // Few queries (decode): one wide CTA per query keeps the selection from being latency-bound.
   const bool wide = nq < 2 * 148;
-  auto kern = wide ? (in_smem ? token_select_kernel<kSelectThreadsWide, true>
-                              : token_select_kernel<kSelectThreadsWide, false>)
-                   : (in_smem ? token_select_kernel<kSelectThreads, true> : token_select_kernel<kSelectThreads, false>);
   const int nt = wide ? kSelectThreadsWide : kSelectThreads;
-  cudaError_t e = ensure_smem((const void*)kern, smem);
+  const size_t stat = wide ? sizeof(StagedSelectShared<kSelectThreadsWide>) : sizeof(StagedSelectShared<kSelectThreads>);
+  const int64_t staged = n * 4 + (int64_t)slots * 4;
+  if (n <= kSelectSmemKeys && staged + (int64_t)stat <= 227 * 1024) {
+    const bool v4 = (n & 3) == 0;
+    auto kern = wide ? (v4 ? token_select_staged_kernel<kSelectThreadsWide, 4>
+                           : token_select_staged_kernel<kSelectThreadsWide, 1>)
+                     : (v4 ? token_select_staged_kernel<kSelectThreads, 4> : token_select_staged_kernel<kSelectThreads, 1>);
+    cudaError_t e = ensure_smem((const void*)kern, (int)staged, (int)stat);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)nq, nt, (int)staged, st>>>(keys, block_idx, slots, token_idx, token_scores, log2B, s.k, q0);
+    return cudaGetLastError();
+  }
+  const int smem = slots * 4;
+  if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
+  auto kern = wide ? token_select_kernel<kSelectThreadsWide> : token_select_kernel<kSelectThreads>;
+  const int gstat = (int)(wide ? sizeof(SelectShared<kSelectThreadsWide>) : sizeof(SelectShared<kSelectThreads>));
+  cudaError_t e = ensure_smem((const void*)kern, smem, gstat);
   if (e != cudaSuccess) return e;
-  kern<<<(unsigned)nq, nt, smem, st>>>(keys, block_idx, slots, token_idx, token_scores, s.n_q, log2B, s.k, q0);
+  kern<<<(unsigned)nq, nt, smem, st>>>(keys, block_idx, slots, token_idx, token_scores, log2B, s.k, q0);
   return cudaGetLastError();
 }
 
