@@ -362,12 +362,12 @@ __device__ int staged_select(const uint32_t* skeys, int n, int k, StagedSelectSh
   warp_span<NT>(n, warp, w0, w1);
   uint32_t* seg = sm.u.cand + warp * SEG;
   int ng = 0, nc = 0;
-  for (int c0 = w0; c0 < w1; c0 += 32 * U) {
+  auto sweep = [&](int c0, bool full) {
     uint32_t kk[U];
 #pragma unroll
     for (int j = 0; j < U; ++j) {
       const int i = c0 + 32 * j + lane;
-      kk[j] = i < w1 ? skeys[i] : 0u;
+      kk[j] = (full || i < w1) ? skeys[i] : 0u;
     }
 #pragma unroll
     for (int j = 0; j < U; ++j) {
@@ -384,7 +384,10 @@ __device__ int staged_select(const uint32_t* skeys, int n, int k, StagedSelectSh
         nc += km == prefix;
       }
     }
-  }
+  };
+  int c0 = w0;
+  for (; c0 + 32 * U <= w1; c0 += 32 * U) sweep(c0, true);  // whole steps: no bound tests
+  if (c0 < w1) sweep(c0, false);
   ng = __reduce_add_sync(0xFFFFFFFFu, ng);
   if (!collect) nc = __reduce_add_sync(0xFFFFFFFFu, nc);
   if (lane == 0) {
@@ -452,21 +455,22 @@ __device__ int staged_select(const uint32_t* skeys, int n, int k, StagedSelectSh
     eqb += ew;
   }
   int rank = taken_before, eq_seen = eq_before;
-  for (int c0 = w0; c0 < w1; c0 += 32 * U) {
+  auto emit = [&](int c0, bool full) {
     uint32_t kk[U];
 #pragma unroll
     for (int j = 0; j < U; ++j) {
       const int i = c0 + 32 * j + lane;
-      kk[j] = i < w1 ? skeys[i] : 0u;
+      kk[j] = (full || i < w1) ? skeys[i] : 0u;
     }
 #pragma unroll
     for (int j = 0; j < U; ++j) {
       const int i = c0 + 32 * j + lane;
       const uint32_t km = kk[j] & mask;
+      const bool in = full || i < w1;
       bool sel = km > prefix;
-      const uint32_t be = __ballot_sync(0xFFFFFFFFu, km == prefix && i < w1);
+      const uint32_t be = __ballot_sync(0xFFFFFFFFu, km == prefix && in);
       if (be) {  // keys at the threshold in this group
-        const bool eq = km == prefix && i < w1;
+        const bool eq = km == prefix && in;
         sel = sel || (eq && eq_seen + __popc(be & below) < teq);
         eq_seen += __popc(be);
       }
@@ -474,7 +478,9 @@ __device__ int staged_select(const uint32_t* skeys, int n, int k, StagedSelectSh
       if (sel) put(rank + __popc(bs & below), i, kk[j]);
       rank += __popc(bs);
     }
-  }
+  };
+  for (c0 = w0; c0 + 32 * U <= w1; c0 += 32 * U) emit(c0, true);
+  if (c0 < w1) emit(c0, false);
   __syncthreads();
   return K;
 }

@@ -4,30 +4,34 @@
 //
 // A kept block is a contiguous B x d_idx tile of k_idx, and 128 consecutive
 // queries keep overlapping sets of blocks.  So instead of gathering rows per
-// query, a CTA takes a tile of 128 query rows of one sequence and a run of up
-// to kRun key blocks at or below the tile's causal limit, and scores every
-// block of the run against the whole tile with one group of tcgen05.mma
-// (kind::f16, M = 128 rows, N = B, fp32 in TMEM; exact on integer-valued
-// inputs).  The CTA is split by role, the roles handing work over through
-// mbarriers:
-//   * warp 8 (one thread): TMA of the query tile once, then of each key block
-//     (B rows, 128-byte swizzle: the K-major UMMA operand) into a ring of
-//     2-4 shared-memory stages;
-//   * warp 9 (one thread): the MMAs of block b into TMEM accumulator b & 1,
-//     once its stage has landed and that accumulator has been read out;
-//   * warps 0-7, two groups of four (group g reads accumulator g, so the
-//     blocks alternate between the groups): each warp reads its 32 rows back
+// query, a CTA takes a tile of 128 query rows of one sequence and every key
+// block that some query of the tile kept (the union of their lists, a bitmap
+// built once per tile), and scores each such block against the whole tile
+// with one group of tcgen05.mma (kind::f16, M = 128 rows, N = B, fp32 in
+// TMEM; exact on integer-valued inputs).  One CTA per tile, the tiles with the
+// most visible blocks launched first; the CTA is split by role, the roles
+// handing work over through mbarriers:
+//   * readout warps 0 .. 4A-1, A groups of four, with A = 4 TMEM
+//     accumulators of B columns (A = 2 when B = 256: 512 columns in all);
+//     the blocks rotate through the groups; each warp reads its 32 rows back
 //     (tcgen05.ld) -- only when one of its queries kept the block -- and
 //     writes that query's B order-preserving keys to its slot of the key
-//     buffer (0 for tokens after the query).
+//     buffer (0 for tokens after the query);
+//   * warp 4A (one thread): TMA of the query tile once, then of each block of
+//     the union (B rows, 128-byte swizzle: the K-major UMMA operand) into a
+//     ring of 2-4 shared-memory stages;
+//   * warp 4A + 1 (one thread): the MMAs of the u-th block into accumulator
+//     u % A, once its stage has landed and that accumulator has been read out.
+// Four groups keep four readout warps on each scheduler: the readout, not the
+// MMA, sets the pace, and more warps hide its TMEM and store latency.
 // With a multi-head indexer the 128 rows are 128 / H queries x H heads and
-// the readout applies w_j * max(0, .) and sums a query's rows.  The slot of
-// block j in each query's kept list comes from a per-CTA map built by
-// scanning the lists once (same acceptance rule as the CUDA-core scorer: in
-// range and above every earlier in-range entry).  The CTA holding the first
-// run also zero-fills unused slots and flags malformed entries.  With no list
-// (the flat indexer) slot = block id.  Waits are bounded (1 s): a role that
-// gives up sets status bit 1 and an abort flag the other roles poll.
+// the readout applies w_j * max(0, .) and sums a query's rows.  Each query's
+// list is accepted once per tile (same rule as the CUDA-core scorer: in range
+// and above every earlier in-range entry), kept in shared memory as ascending
+// (block, slot) pairs, and walked by a cursor as the blocks go by; rejected
+// entries are flagged and their slots zero-filled.  With no list (the flat
+// indexer) slot = block id.  Waits are bounded (1 s): a role that gives up
+// sets status bit 1 and an abort flag the other roles poll.
 #include "common.cuh"
 #include "internal.h"
 #include "tc_common.cuh"
@@ -35,13 +39,11 @@
 namespace hisa {
 namespace {
 
-constexpr int kEpiWarps = 8;  // two groups of four, one per TMEM accumulator
-constexpr int kWarpTma = 8, kWarpMma = 9;
-constexpr int kThreads = (kEpiWarps + 2) * 32;
 constexpr int kTileQ = 128;
-constexpr int kRun = 64;  // key blocks per CTA
+constexpr int kListSlots = 96;     // longest kept list a tile holds (longer lists: the CUDA-core scorer)
+constexpr int kMaxBlocks = 16384;  // blocks per sequence the tile's bitmap covers
 
-// Key stages in flight per CTA (fewer stages, less shared memory: more CTAs per SM).
+// Key stages in flight per CTA.
 #ifndef HISA_TS_MAX_STAGES
 #define HISA_TS_MAX_STAGES 4
 #endif
@@ -53,25 +55,39 @@ constexpr int kRun = 64;  // key blocks per CTA
 #define HISA_TS_TM_MIN_HEADS 4
 #endif
 
-template <int D, int B>
+template <int D, int B, int HET>
 struct TsLayout {
   static constexpr int HALVES = D / 64;
   static constexpr int Q_BYTES = HALVES * kTileQ * 128;
   static constexpr int K_BYTES = HALVES * B * 128;
-  static constexpr int MAP_BYTES = kTileQ * kRun * 2;  // int16 [kTileQ][kRun]
-  static constexpr int AVAIL = 227 * 1024 - 1024 - Q_BYTES - MAP_BYTES - kTileQ * 4 - 256;
+  // TMEM accumulators (B columns each, 512 columns in all) and the readout groups of four warps
+  // that read them, one group per accumulator; then the TMA warp and the MMA warp.
+  // (the token-major readout keeps two: its register use leaves no room for four groups)
+  static constexpr int NACC = HET > 0 ? 2 : (4 * B <= 512 ? 4 : 512 / B);
+  static constexpr int EPI_WARPS = 4 * NACC;
+  static constexpr int WARP_TMA = EPI_WARPS, WARP_MMA = EPI_WARPS + 1;
+  static constexpr int THREADS = (EPI_WARPS + 2) * 32;
+  // kept lists, entry = block << 16 | slot, stored [kListSlots + 1][kTileQ] (a sentinel ends each)
+  static constexpr int LIST_BYTES = (kListSlots + 1) * kTileQ * 4;
+  static constexpr int BITS_BYTES = kMaxBlocks / 8;
+  static constexpr int SLOTB_BYTES = 2 * NACC * kTileQ * 4;  // token-major: a group's slot table, 2 buffers
+  static constexpr int FIXED = 1024 + Q_BYTES + LIST_BYTES + BITS_BYTES + SLOTB_BYTES + kTileQ * 4 + 512;
+  static constexpr int AVAIL = 227 * 1024 - FIXED;
   static constexpr int STAGES = AVAIL / K_BYTES >= HISA_TS_MAX_STAGES ? HISA_TS_MAX_STAGES : AVAIL / K_BYTES;
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = Q_OFF + Q_BYTES;
-  static constexpr int MAP_OFF = K_OFF + STAGES * K_BYTES;
-  static constexpr int W_OFF = MAP_OFF + MAP_BYTES;  // fp32 [kTileQ] head weights of the tile rows
+  static constexpr int LIST_OFF = K_OFF + STAGES * K_BYTES;
+  static constexpr int BITS_OFF = LIST_OFF + LIST_BYTES;
+  static constexpr int SLOTB_OFF = BITS_OFF + BITS_BYTES;
+  static constexpr int W_OFF = SLOTB_OFF + SLOTB_BYTES;  // fp32 [kTileQ] head weights of the tile rows
   static constexpr int BAR_OFF = W_OFF + kTileQ * 4;
-  // mbarriers: q full | accumulator full x 2 | accumulator empty x 2 | K full x S | K empty x S
-  static constexpr int B_Q = 0, B_AFULL = 1, B_AEMPTY = 3, B_KFULL = 5, B_KEMPTY = 5 + STAGES;
-  static constexpr int NBAR = 5 + 2 * STAGES;
+  // mbarriers: q full | accumulator full x NACC | accumulator empty x NACC | K full x S | K empty x S
+  static constexpr int B_Q = 0, B_AFULL = 1, B_AEMPTY = 1 + NACC, B_KFULL = 1 + 2 * NACC,
+                       B_KEMPTY = B_KFULL + STAGES;
+  static constexpr int NBAR = B_KEMPTY + STAGES;
   static constexpr int MISC_OFF = BAR_OFF + 8 * NBAR;  // TMEM base, abort flag
   static constexpr int SMEM = MISC_OFF + 16 + 1024;
-  static constexpr uint32_t TMEM_COLS = 2 * B;  // two B-column accumulators
+  static constexpr uint32_t TMEM_COLS = NACC * B;
   static_assert(STAGES >= 2, "two key stages at least");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
   static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(B >> 3) << 17) |
@@ -80,18 +96,15 @@ struct TsLayout {
 
 using namespace tc;
 
-// HET = 0: TMEM lane = tile row (query, head), columns = the block's tokens.  HET = 8 or 16
-// (token-major, B = 128): the MMA operands swap, so TMEM lane = token and columns = tile rows; a
-// query's HET heads are then consecutive registers of one thread and a warp's 32 lanes write 32
-// consecutive keys of a query.
 template <int D, int B, int HET>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(TsLayout<D, B, HET>::THREADS, 1)
     token_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                           const int32_t* __restrict__ block_idx, int slots, uint32_t* __restrict__ keys,
-                          int32_t* __restrict__ status, int64_t n_q, int64_t n_kv, int q_tiles, int runs, int64_t q0,
-                          int64_t nq, const float* __restrict__ w_idx, int HI) {
-  using L = TsLayout<D, B>;
+                          int32_t* __restrict__ status, int64_t n_q, int64_t n_kv, int q_tiles, int64_t n_tiles,
+                          int64_t q0, int64_t nq, const float* __restrict__ w_idx, int HI) {
+  using L = TsLayout<D, B, HET>;
   constexpr int S = L::STAGES;
+  constexpr int NACC = L::NACC, kEpiWarps = L::EPI_WARPS, kWarpTma = L::WARP_TMA, kWarpMma = L::WARP_MMA;
   constexpr bool kTokenMajor = HET > 0;
   static_assert(!kTokenMajor || (B == kTileQ && 32 % HET == 0), "token-major readout: B = 128, HET divides 32");
   extern __shared__ uint8_t smem_raw[];
@@ -100,9 +113,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Rows of the tile are (query, indexer head) pairs: QT queries x HE heads.
   const int HE = HI > 0 ? HI : 1;
   const int QT = kTileQ / HE;
-  // Tiles are enumerated over the queries of the chunk [q0, q0 + nq).
-  const int run = blockIdx.x % runs;
-  const int64_t tile_lin = blockIdx.x / runs;
+  // One CTA per tile of the chunk [q0, q0 + nq), the last tiles (the most visible blocks) first.
+  const int64_t tile_lin = n_tiles - 1 - (int64_t)blockIdx.x;
   const int64_t seq_first = q0 / n_q;
   const int64_t tile0 = (q0 % n_q) / QT;      // first tile of the first sequence touched
   const int64_t tile_abs = tile0 + tile_lin;  // tile counted from the first sequence's start
@@ -112,15 +124,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t t_lo = max(tq0, q0);
   const int64_t t_hi = min(min(tq0 + QT, (seq + 1) * n_q), q0 + nq);  // exclusive
   if (t_lo >= t_hi) return;
-  const int64_t c_max = (n_kv - n_q + (t_hi - 1 - seq * n_q)) / B;
-  const int64_t jb0 = (int64_t)run * kRun;
-  if (jb0 > c_max) return;
-  const int nb = (int)min((int64_t)kRun, c_max + 1 - jb0);
+  const int c_max = (int)((n_kv - n_q + (t_hi - 1 - seq * n_q)) / B);  // last block visible to the tile
+  const int nwords = (c_max >> 5) + 1;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint8_t* sQ = smem + L::Q_OFF;
   uint8_t* sK = smem + L::K_OFF;
-  int16_t* smap = reinterpret_cast<int16_t*>(smem + L::MAP_OFF);
+  uint32_t* lists = reinterpret_cast<uint32_t*>(smem + L::LIST_OFF);
+  uint32_t* bits = reinterpret_cast<uint32_t*>(smem + L::BITS_OFF);
+  int32_t* slotb = reinterpret_cast<int32_t*>(smem + L::SLOTB_OFF);
   const uint32_t bar0 = smem_u32(smem + L::BAR_OFF);
   auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
@@ -137,7 +149,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (tid == 0) {
     mbar_init(bar(L::B_Q), 1);
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < NACC; ++a) {
       mbar_init(bar(L::B_AFULL + a), 1);
       mbar_init(bar(L::B_AEMPTY + a), 4);  // the four warps of group a
     }
@@ -153,39 +165,128 @@ __global__ void __launch_bounds__(kThreads, 1)
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = *tmem_slot;
 
+  if (warp == kWarpTma && lane == 0) {  // the query tile, while the lists are read
+    mbar_expect_tx(bar(L::B_Q), (uint32_t)L::Q_BYTES);
+    for (int hh = 0; hh < L::HALVES; ++hh)
+      tma_load_2d(smem_u32(sQ + hh * kTileQ * 128), &tmap_q, hh * 64, (int)(tq0 * HE), bar(L::B_Q));
+  }
+  if (warp < kEpiWarps) {
+    // ---------------- the kept lists and the tile's block bitmap ----------------
+    for (int i = tid; i < nwords; i += kEpiWarps * 32) bits[i] = 0u;
+    asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
+    if (tid < QT) {
+      const int64_t qrow = tq0 + tid;  // global query id
+      const bool row_ok = qrow >= t_lo && qrow < t_hi;
+      const int64_t p = n_kv - n_q + (qrow - seq * n_q);
+      const int64_t c = p / B;
+      uint32_t* krow_keys = keys + (qrow - q0) * (int64_t)slots * B;
+      int cnt = 0;
+      if (row_ok) {
+        if (block_idx) {
+          const int32_t* lst = block_idx + qrow * slots;
+          // the list in batches of 32 entries, loaded together (16-byte loads when aligned)
+          const bool vec = ((reinterpret_cast<uintptr_t>(lst) & 15) == 0);
+          int mx = -1;
+#pragma unroll 1
+          for (int r0 = 0; r0 < slots; r0 += 32) {
+            int e[32];
+            if (vec && r0 + 32 <= slots) {
+              const int4* l4 = reinterpret_cast<const int4*>(lst + r0);
+#pragma unroll
+              for (int uu = 0; uu < 8; ++uu) {
+                const int4 t = l4[uu];
+                e[4 * uu] = t.x;
+                e[4 * uu + 1] = t.y;
+                e[4 * uu + 2] = t.z;
+                e[4 * uu + 3] = t.w;
+              }
+            } else {
+#pragma unroll
+              for (int uu = 0; uu < 32; ++uu) e[uu] = r0 + uu < slots ? lst[r0 + uu] : -1;
+            }
+#pragma unroll
+            for (int uu = 0; uu < 32; ++uu) {
+              const int r = r0 + uu;
+              const int b = e[uu];
+              const bool in_range = b >= 0 && b <= c;
+              const bool ok = in_range && b > mx;
+              if (ok) {
+                lists[cnt * kTileQ + tid] = ((uint32_t)b << 16) | (uint32_t)r;
+                ++cnt;
+                atomicOr(&bits[b >> 5], 1u << (b & 31));
+              } else if (r < slots) {
+                if (b != -1 && status) atomicOr(status, kStatusBadIndex);
+                uint4* z = reinterpret_cast<uint4*>(krow_keys + (int64_t)r * B);
+                for (int i = 0; i < B / 4; ++i) z[i] = make_uint4(0, 0, 0, 0);
+              }
+              if (in_range) mx = max(mx, b);
+            }
+          }
+        } else {  // blocks after the query's own block hold no candidate
+          for (int64_t r = c + 1; r < slots; ++r) {
+            uint4* z = reinterpret_cast<uint4*>(krow_keys + r * B);
+            for (int i = 0; i < B / 4; ++i) z[i] = make_uint4(0, 0, 0, 0);
+          }
+        }
+      }
+      lists[cnt * kTileQ + tid] = 0xFFFF0000u;  // sentinel: above every block
+    }
+    if (!block_idx)  // the flat indexer: every block up to the tile's last
+      for (int i = tid; i < nwords; i += kEpiWarps * 32)
+        bits[i] = (32 * i + 31 <= c_max) ? 0xFFFFFFFFu : (0xFFFFFFFFu >> (31 - (c_max & 31)));
+    if constexpr (kTokenMajor) {
+      float* wsm = reinterpret_cast<float*>(smem + L::W_OFF);
+      if (tid < kTileQ) {
+        const int64_t qr = tq0 + tid / HET;
+        wsm[tid] = (HI > 0 && qr >= t_lo && qr < t_hi) ? w_idx[qr * HET + tid % HET] : 0.f;
+      }
+    }
+  }
+  __syncthreads();  // lists, bitmap and head weights complete
+
+  // the kept block after b (c_max + 1 when none): every role walks the same sequence
+  auto next_blk = [&](int b) -> int {
+    const int x = b + 1;
+    int w = x >> 5;
+    if (w >= nwords) return c_max + 1;
+    uint32_t m = bits[w] & (0xFFFFFFFFu << (x & 31));
+    while (m == 0u) {
+      if (++w >= nwords) return c_max + 1;
+      m = bits[w];
+    }
+    return (w << 5) + __ffs(m) - 1;
+  };
+
   if (warp == kWarpTma) {
-    // ---------------- producer: the query tile, then the key blocks into the stage ring ----------------
+    // ---------------- producer: the blocks of the union into the stage ring ----------------
     if (lane == 0) {
-      mbar_expect_tx(bar(L::B_Q), (uint32_t)L::Q_BYTES);
-      for (int hh = 0; hh < L::HALVES; ++hh)
-        tma_load_2d(smem_u32(sQ + hh * kTileQ * 128), &tmap_q, hh * 64, (int)(tq0 * HE), bar(L::B_Q));
-      int issued = 0;
-      for (int b = 0; b < nb; ++b) {
-        const int st = b % S;
-        if (!mbar_wait_or_abort(bar(L::B_KEMPTY + st), (uint32_t)(((b / S) & 1) ^ 1), abort_flag)) {
+      int issued = 0, u = 0;
+      for (int b = next_blk(-1); b <= c_max; b = next_blk(b), ++u) {
+        const int st = u % S;
+        if (!mbar_wait_or_abort(bar(L::B_KEMPTY + st), (uint32_t)(((u / S) & 1) ^ 1), abort_flag)) {
           fail();
           break;
         }
         mbar_expect_tx(bar(L::B_KFULL + st), (uint32_t)L::K_BYTES);
-        const int krow = (int)(seq * n_kv + (jb0 + b) * B);
+        const int krow = (int)(seq * n_kv + (int64_t)b * B);
         for (int hh = 0; hh < L::HALVES; ++hh)
           tma_load_2d(smem_u32(sK + st * L::K_BYTES + hh * B * 128), &tmap_k, hh * 64, krow, bar(L::B_KFULL + st));
-        issued = b + 1;
+        issued = u + 1;
       }
       // copies still in flight land before the CTA exits (all of them have, unless a role gave up)
       mbar_wait(bar(L::B_Q), 0);
-      for (int b = max(0, issued - S); b < issued; ++b) mbar_wait(bar(L::B_KFULL + b % S), (uint32_t)((b / S) & 1));
+      for (int v = max(0, issued - S); v < issued; ++v) mbar_wait(bar(L::B_KFULL + v % S), (uint32_t)((v / S) & 1));
     }
   } else if (warp == kWarpMma) {
-    // ---------------- MMA issuer: block b into accumulator b & 1 ----------------
+    // ---------------- MMA issuer: the u-th block into accumulator u % NACC ----------------
     if (lane == 0) {
       const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK);
       bool ok = mbar_wait_or_abort(bar(L::B_Q), 0, abort_flag);
-      int issued = 0;
-      for (int b = 0; b < nb && ok; ++b) {
-        const int st = b % S, a = b & 1;
-        ok = mbar_wait_or_abort(bar(L::B_KFULL + st), (uint32_t)((b / S) & 1), abort_flag) &&
-             mbar_wait_or_abort(bar(L::B_AEMPTY + a), (uint32_t)(((b >> 1) & 1) ^ 1), abort_flag);
+      int issued = 0, u = 0;
+      for (int b = next_blk(-1); b <= c_max && ok; b = next_blk(b), ++u) {
+        const int st = u % S, a = u % NACC;
+        ok = mbar_wait_or_abort(bar(L::B_KFULL + st), (uint32_t)((u / S) & 1), abort_flag) &&
+             mbar_wait_or_abort(bar(L::B_AEMPTY + a), (uint32_t)(((u / NACC) & 1) ^ 1), abort_flag);
         if (!ok) break;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         const uint32_t acc_col = tmem + (uint32_t)(a * B);
@@ -203,84 +304,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         umma_commit(bar(L::B_KEMPTY + st));  // the stage may be refilled once these MMAs have read it
         umma_commit(bar(L::B_AFULL + a));    // and the accumulator read out
-        issued = b + 1;
+        issued = u + 1;
       }
       if (!ok) fail();
       // every MMA issued has completed before the TMEM is released
-      if (issued > 0) mbar_wait(bar(L::B_AFULL + ((issued - 1) & 1)), (uint32_t)(((issued - 1) >> 1) & 1));
+      if (issued > 0) mbar_wait(bar(L::B_AFULL + (issued - 1) % NACC), (uint32_t)(((issued - 1) / NACC) & 1));
     }
   } else {
     // ---------------- readout warps ----------------
-    // Slot map of query tid of the tile (threads tid < QT) for blocks jb0 .. jb0+nb-1, stored
-    // block-major (smap[jj * kTileQ + query]) so that a warp's 32 queries sit in consecutive halves.
-    {
-      uint4* m4 = reinterpret_cast<uint4*>(smap);
-      for (int i = tid; i < L::MAP_BYTES / 16; i += kEpiWarps * 32) m4[i] = make_uint4(~0u, ~0u, ~0u, ~0u);
-      asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");
-      const int64_t qrow = tq0 + tid;  // global query id
-      const bool row_ok = tid < QT && qrow >= t_lo && qrow < t_hi;
-      const int64_t p = n_kv - n_q + (qrow - seq * n_q);
-      const int64_t c = p / B;
-      uint32_t* krow_keys = keys + (qrow - q0) * (int64_t)slots * B;
-      if (row_ok) {
-        if (block_idx) {
-          const int32_t* lst = block_idx + qrow * slots;
-          // the list in batches of 32 entries, loaded together (16-byte loads when aligned)
-          const bool vec = ((reinterpret_cast<uintptr_t>(lst) & 15) == 0);
-          int mx = -1;
-#pragma unroll 1
-          for (int r0 = 0; r0 < slots; r0 += 32) {
-            int e[32];
-            if (vec && r0 + 32 <= slots) {
-              const int4* l4 = reinterpret_cast<const int4*>(lst + r0);
-#pragma unroll
-              for (int u = 0; u < 8; ++u) {
-                const int4 t = l4[u];
-                e[4 * u] = t.x;
-                e[4 * u + 1] = t.y;
-                e[4 * u + 2] = t.z;
-                e[4 * u + 3] = t.w;
-              }
-            } else {
-#pragma unroll
-              for (int u = 0; u < 32; ++u) e[u] = r0 + u < slots ? lst[r0 + u] : -1;
-            }
-#pragma unroll
-            for (int u = 0; u < 32; ++u) {
-              const int r = r0 + u;
-              const int b = e[u];
-              const bool in_range = b >= 0 && b <= c;
-              const bool ok = in_range && b > mx;
-              if (ok && b >= jb0 && b < jb0 + nb) smap[(b - jb0) * kTileQ + tid] = (int16_t)r;
-              if (run == 0 && !ok && r < slots) {
-                if (b != -1 && status) atomicOr(status, kStatusBadIndex);
-                uint4* z = reinterpret_cast<uint4*>(krow_keys + (int64_t)r * B);
-                for (int i = 0; i < B / 4; ++i) z[i] = make_uint4(0, 0, 0, 0);
-              }
-              if (in_range) mx = max(mx, b);
-            }
-          }
-        } else {
-          for (int jj = 0; jj < nb; ++jj)
-            if (jb0 + jj <= c) smap[jj * kTileQ + tid] = (int16_t)(jb0 + jj);
-          if (run == 0) {  // blocks after the query's own block hold no candidate
-            for (int64_t r = c + 1; r < slots; ++r) {
-              uint4* z = reinterpret_cast<uint4*>(krow_keys + r * B);
-              for (int i = 0; i < B / 4; ++i) z[i] = make_uint4(0, 0, 0, 0);
-            }
-          }
-        }
-      }
-    }
-    if constexpr (kTokenMajor) {
-      float* wsm = reinterpret_cast<float*>(smem + L::W_OFF);
-      if (tid < kTileQ) {
-        const int64_t qr = tq0 + tid / HET;
-        wsm[tid] = (HI > 0 && qr >= t_lo && qr < t_hi) ? w_idx[qr * HET + tid % HET] : 0.f;
-      }
-    }
-    asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory");  // the slot maps are complete
-
     // This thread's TMEM lane = tile row r: query tq0 + r / HE, indexer head r % HE.
     const int g = warp >> 2, quarter = warp & 3;
     const int r = quarter * 32 + lane;
@@ -290,18 +321,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t p = n_kv - n_q + (qrow - seq * n_q);
     uint32_t* krow_keys = keys + (qrow - q0) * (int64_t)slots * B;
     const float wgt = (HI > 0 && row_ok) ? w_idx[qrow * HI + head] : 1.f;
-    for (int b = g; b < nb; b += 2) {
+    // The slot of block b in the kept list of query lq (the row's query; in the token-major
+    // readout, query r of the group's table), by a cursor that only moves forward.
+    const int lq = kTokenMajor ? r : qi;
+    const bool lq_ok = lq < QT && tq0 + lq >= t_lo && tq0 + lq < t_hi;
+    const int64_t lq_c = (n_kv - n_q + (tq0 + lq - seq * n_q)) / B;
+    int cur = 0;
+    uint32_t ent = (lq_ok && block_idx) ? lists[lq] : 0xFFFF0000u;
+    auto slot_of = [&](int b) -> int {
+      if (!lq_ok) return -1;
+      if (!block_idx) return b <= lq_c ? b : -1;
+      while ((int)(ent >> 16) < b) {
+        ++cur;
+        ent = lists[cur * kTileQ + lq];
+      }
+      return (int)(ent >> 16) == b ? (int)(ent & 0xFFFFu) : -1;
+    };
+    int u = 0;
+    for (int b = next_blk(-1); b <= c_max; b = next_blk(b), ++u) {
+      if (u % NACC != g) continue;
       // the warp leaves together (the shuffles and TMEM loads below are warp-wide)
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait_or_abort(bar(L::B_AFULL + g), (uint32_t)((b >> 1) & 1), abort_flag))) {
+      if (!__all_sync(0xFFFFFFFFu,
+                      mbar_wait_or_abort(bar(L::B_AFULL + g), (uint32_t)((u / NACC) & 1), abort_flag))) {
         if (lane == 0) fail();
         break;
       }
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       if constexpr (kTokenMajor) {
+        // this block's slot of every query of the tile, one query per thread of the group
+        int32_t* tbl = slotb + ((u / NACC) & 1) * (NACC * kTileQ) + g * kTileQ;
+        tbl[r] = slot_of(b);
+        asm volatile("bar.sync %0, %1;" ::"r"(2 + g), "n"(128) : "memory");
         // lane = token jb * B + quarter * 32 + lane; chunk cc holds queries cc * kQpc .. + kQpc - 1
         constexpr int kQpc = 32 / (HET > 0 ? HET : 1);
         const float* wsm = reinterpret_cast<const float*>(smem + L::W_OFF);
-        const int64_t tk = (jb0 + b) * B + quarter * 32 + lane;
+        const int64_t tk = (int64_t)b * B + quarter * 32 + lane;
 #pragma unroll 1
         for (int cc = 0; cc < kTileQ / 32; ++cc) {
           int sl[kQpc];
@@ -310,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int qq = 0; qq < kQpc; ++qq) {
             const int ql = cc * kQpc + qq;
             const int64_t qr = tq0 + ql;
-            sl[qq] = (qr >= t_lo && qr < t_hi) ? smap[b * kTileQ + ql] : -1;  // the same in every lane
+            sl[qq] = (qr >= t_lo && qr < t_hi) ? tbl[ql] : -1;  // the same in every lane
             any = any || sl[qq] >= 0;
           }
           if (!any) continue;  // warp-uniform
@@ -346,11 +400,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else {
-        // rows whose query kept block jb0 + b
-        const int slot = row_ok ? smap[b * kTileQ + qi] : -1;
+        // rows whose query kept block b
+        const int slot = slot_of(b);
         if (__any_sync(0xFFFFFFFFu, slot >= 0)) {
-          const int64_t j = jb0 + b;
-          const int64_t tok0 = j * B;
+          const int64_t tok0 = (int64_t)b * B;
           uint32_t* dst = krow_keys + (int64_t)(slot < 0 ? 0 : slot) * B;
           // lane 0 holds the warp's first query: a block wholly at or before it needs no causal test
           const bool whole = tok0 + B - 1 <= __shfl_sync(0xFFFFFFFFu, p, 0);
@@ -410,18 +463,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
           };
-          // 32 columns at a time, the load of the next chunk in flight while this one is converted
+          // 32 columns at a time
           const uint32_t a0 = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(g * B);
-          uint32_t va[32], vb[32];
-          tmem_ld32_issue(a0, va);
-          tmem_wait_ld(va);
-#pragma unroll
+#pragma unroll 1
           for (int cc = 0; cc < B / 32; ++cc) {
-            uint32_t(&cur)[32] = (cc & 1) ? vb : va;
-            uint32_t(&nxt)[32] = (cc & 1) ? va : vb;
-            if (cc + 1 < B / 32) tmem_ld32_issue(a0 + (uint32_t)((cc + 1) * 32), nxt);
-            chunk(cc, cur);
-            if (cc + 1 < B / 32) tmem_wait_ld(nxt);
+            uint32_t v[32];
+            tmem_ld32_issue(a0 + (uint32_t)(cc * 32), v);
+            tmem_wait_ld(v);
+            chunk(cc, v);
           }
         }
       }
@@ -443,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D, int B, int HET>
 cudaError_t launch_ts(const Shape& s, const void* q_idx, const void* k_idx, const int32_t* block_idx, int slots,
                       uint32_t* keys, int32_t* status, int64_t q0, int64_t nq, cudaStream_t st) {
-  using L = TsLayout<D, B>;
+  using L = TsLayout<D, B, HET>;
   CUtensorMap mq, mk;
   const int HE = s.HI > 0 ? s.HI : 1;
   const int QT = kTileQ / HE;
@@ -453,15 +502,14 @@ cudaError_t launch_ts(const Shape& s, const void* q_idx, const void* k_idx, cons
   cudaError_t e = ensure_smem((const void*)kern, L::SMEM);
   if (e != cudaSuccess) return e;
   const int q_tiles = (int)((s.n_q + QT - 1) / QT);
-  const int runs = (int)((s.n_blk + kRun - 1) / kRun);
   // tiles from the chunk's first tile to its last
   const int64_t first = (q0 / s.n_q) * q_tiles + (q0 % s.n_q) / QT;
   const int64_t lastq = q0 + nq - 1;
   const int64_t last = (lastq / s.n_q) * q_tiles + (lastq % s.n_q) / QT;
-  const int64_t grid = (last - first + 1) * runs;
+  const int64_t grid = last - first + 1;
   if (grid > 0x7FFFFFFFLL) return cudaErrorNotSupported;
-  kern<<<(unsigned)grid, kThreads, L::SMEM, st>>>(mq, mk, block_idx, slots, keys, status, s.n_q, s.n_kv, q_tiles,
-                                                  runs, q0, nq, s.w_idx, s.HI);
+  kern<<<(unsigned)grid, L::THREADS, L::SMEM, st>>>(mq, mk, block_idx, slots, keys, status, s.n_q, s.n_kv, q_tiles,
+                                                  grid, q0, nq, s.w_idx, s.HI);
   return cudaGetLastError();
 }
 
@@ -471,13 +519,14 @@ bool token_score_tc_eligible(const Shape& s, int slots) {
   // a query's indexer heads are consecutive rows of a warp: 1, 2, 4, 8 or 16 of them
   const bool heads_ok = s.HI == 0 || (s.HI <= 16 && (s.HI & (s.HI - 1)) == 0);
   return heads_ok && (s.d_idx == 64 || s.d_idx == 128) && (s.B == 32 || s.B == 64 || s.B == 128 || s.B == 256) &&
-         s.n_q >= kTileQ && slots < 32767 && s.n_query <= 0x7FFFFFFFLL &&
+         s.n_q >= kTileQ && s.n_blk <= kMaxBlocks && s.n_query <= 0x7FFFFFFFLL &&
          (int64_t)s.batch * s.n_kv <= 0x7FFFFFFFLL;
 }
 
 cudaError_t launch_token_score_tc(const Shape& s, const void* q_idx, const void* k_idx, const int32_t* block_idx,
                                   int slots, uint32_t* keys, int32_t* status, int64_t q0, int64_t nq, cudaStream_t st) {
   if (!token_score_tc_eligible(s, slots)) return cudaErrorNotSupported;
+  if (block_idx && slots > kListSlots) return cudaErrorNotSupported;  // the CUDA-core scorer takes long lists
   // B = 128 with at least HISA_TS_TM_MIN_HEADS indexer heads: token-major readout (a query's
   // heads in one thread, coalesced key stores)
   const int he = s.HI > 0 ? s.HI : 1;

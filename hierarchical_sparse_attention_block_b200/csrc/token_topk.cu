@@ -225,8 +225,8 @@ __global__ void __launch_bounds__(kScoreThreads)
 // One CTA per query; the row of keys, read from global memory, is staged in
 // shared memory and the first selection digit counted on the way in (three
 // sweeps of the row in all: staging, the candidate sweep and the emit sweep).
-// V = 4: the row length is a multiple of four (16-byte staging).
-template <int NT, int V>
+// V = 4: the row length is a multiple of four (16-byte staging).  SC: scores are written too.
+template <int NT, int V, bool SC>
 __global__ void __launch_bounds__(NT)
     token_select_staged_kernel(const uint32_t* __restrict__ keys, const int32_t* __restrict__ block_idx, int slots,
                                int32_t* __restrict__ token_idx, float* __restrict__ token_scores, int log2B, int k,
@@ -269,7 +269,7 @@ __global__ void __launch_bounds__(NT)
   float* osc = token_scores ? token_scores + qg * k : nullptr;
   const int K = staged_select<NT>(skeys, n, k, sm, [&](int rank, int i, uint32_t key) {
     out[rank] = sblk[i >> log2B] * B + (i & (B - 1));
-    if (osc) osc[rank] = key_score(key);
+    if constexpr (SC) osc[rank] = key_score(key);
   });
   for (int r = K + threadIdx.x; r < k; r += NT) {
     out[r] = -1;
@@ -380,10 +380,12 @@ cudaError_t launch_token_select(const Shape& s, const uint32_t* keys, const int3
   const size_t stat = wide ? sizeof(StagedSelectShared<kSelectThreadsWide>) : sizeof(StagedSelectShared<kSelectThreads>);
   const int64_t staged = n * 4 + (int64_t)slots * 4;
   if (n <= kSelectSmemKeys && staged + (int64_t)stat <= 227 * 1024) {
-    const bool v4 = (n & 3) == 0;
-    auto kern = wide ? (v4 ? token_select_staged_kernel<kSelectThreadsWide, 4>
-                           : token_select_staged_kernel<kSelectThreadsWide, 1>)
-                     : (v4 ? token_select_staged_kernel<kSelectThreads, 4> : token_select_staged_kernel<kSelectThreads, 1>);
+    const bool v4 = (n & 3) == 0, sc = token_scores != nullptr;
+#define HISA_SEL(NT) \
+  (v4 ? (sc ? token_select_staged_kernel<NT, 4, true> : token_select_staged_kernel<NT, 4, false>) \
+      : (sc ? token_select_staged_kernel<NT, 1, true> : token_select_staged_kernel<NT, 1, false>))
+    auto kern = wide ? HISA_SEL(kSelectThreadsWide) : HISA_SEL(kSelectThreads);
+#undef HISA_SEL
     cudaError_t e = ensure_smem((const void*)kern, (int)staged, (int)stat);
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)nq, nt, (int)staged, st>>>(keys, block_idx, slots, token_idx, token_scores, log2B, s.k, q0);
