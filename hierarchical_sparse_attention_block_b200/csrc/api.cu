@@ -607,14 +607,41 @@ hisa_status_t hisa_forward_host(const hisa_params_t* params, const void* q_idx, 
   return hisa::cuda_fail(se);
 }
 
+namespace hisa {
+namespace {
+
+// The flat indexer's window: 8192 candidate tokens (k rounded up to blocks if more), in blocks.
+int flat_window(const Shape& s) {
+  int64_t w = 8192 / s.B;
+  if (w < 1) w = 1;
+  if (w * s.B < s.k) w = (s.k + s.B - 1) / s.B;
+  if (w > s.n_blk) w = s.n_blk;
+  return (int)w;
+}
+
+// Bytes per query row processed at once: the window's keys and four k-entry arrays (two running
+// lists, ids and scores each).
+size_t flat_row_bytes(const Shape& s) {
+  return (size_t)flat_window(s) * s.B * sizeof(uint32_t) + 4 * (size_t)s.k * 4;
+}
+
+constexpr size_t kFlatCap = (size_t)8 << 30;
+
+}  // namespace
+}  // namespace hisa
+
 hisa_status_t hisa_flat_topk_workspace_size(const hisa_params_t* params, size_t* min_bytes, size_t* preferred_bytes) {
   Shape s;
   hisa_status_t rc = hisa::make_shape(params, true, false, &s);
   if (rc != HISA_OK) return rc;
   if (!min_bytes && !preferred_bytes) return HISA_ERR_INVALID_ARG;
-  if (s.n_blk > 50000 || s.n_blk * (int64_t)s.B > ((int64_t)1 << 30)) return HISA_ERR_UNSUPPORTED;
-  if (min_bytes) *min_bytes = hisa::token_keys_per_query(s, (int)s.n_blk);
-  if (preferred_bytes) *preferred_bytes = hisa::keys_preferred(s, (int)s.n_blk);
+  if (s.n_blk > 50000 || s.k >= 32768) return HISA_ERR_UNSUPPORTED;
+  const size_t per = hisa::flat_row_bytes(s) + 5 * hisa::kAlign;
+  size_t rows = hisa::kFlatCap / per;
+  if (rows < 1) rows = 1;
+  if (rows > (size_t)s.n_q) rows = (size_t)s.n_q;
+  if (min_bytes) *min_bytes = per;
+  if (preferred_bytes) *preferred_bytes = rows * per;
   return HISA_OK;
 }
 
@@ -629,9 +656,79 @@ hisa_status_t hisa_flat_topk(const hisa_params_t* params, const void* q_idx, con
   if (!hisa::aligned16(q_idx) || !hisa::aligned16(k_idx) || !hisa::aligned16(token_idx)) return HISA_ERR_INVALID_ARG;
   if (token_scores && !hisa::aligned16(token_scores)) return HISA_ERR_INVALID_ARG;
   if (!workspace || !hisa::aligned16(workspace)) return HISA_ERR_WORKSPACE;
-  if (s.n_blk > 50000 || s.n_blk * (int64_t)s.B > ((int64_t)1 << 30)) return HISA_ERR_UNSUPPORTED;
-  return hisa::run_token_stage(s, q_idx, k_idx, nullptr, (int)s.n_blk, token_idx, token_scores, nullptr, workspace,
-                               workspace_bytes, stream);
+  if (s.n_blk > 50000 || s.k >= 32768) return HISA_ERR_UNSUPPORTED;
+  const int W = hisa::flat_window(s);
+  const int64_t k = s.k, WB = (int64_t)W * s.B;
+  // rows per chunk: the window's keys, then running lists 0 and 1
+  const size_t per = hisa::flat_row_bytes(s) + 5 * hisa::kAlign;
+  int64_t R = (int64_t)(workspace_bytes / per);
+  if (R < 1) return HISA_ERR_WORKSPACE;
+  if (R > s.n_q) R = s.n_q;
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    uint8_t* p = base + off;
+    off += hisa::align_up(bytes);
+    return p;
+  };
+  uint32_t* keys = reinterpret_cast<uint32_t*>(take((size_t)R * WB * 4));
+  int32_t* ids[2];
+  float* sc[2];
+  for (int i = 0; i < 2; ++i) {
+    ids[i] = reinterpret_cast<int32_t*>(take((size_t)R * k * 4));
+    sc[i] = reinterpret_cast<float*>(take((size_t)R * k * 4));
+  }
+  // the select writes row q at out + q * k: shift a chunk buffer so that global row g0 lands first
+  auto at_row = [&](auto* buf, int64_t g0) {
+    return reinterpret_cast<decltype(buf)>(reinterpret_cast<uintptr_t>(buf) - (uintptr_t)(g0 * k * 4));
+  };
+  const int64_t off_kv = s.n_kv - s.n_q;  // position of query 0
+  // Window j covers blocks [j W, (j + 1) W); query i (position off_kv + i) takes part in windows
+  // 0 .. its own, and its list is final after that one: rows that end at window j write the output,
+  // the rest carry a running list (buffers cur / nxt in turn) to window j + 1.
+  auto first_row = [&](int64_t j, int64_t a) {  // first row of the chunk taking part in window j
+    const int64_t r = j * WB - off_kv;
+    return r > a ? r : a;
+  };
+  for (int64_t seq = 0; seq < s.batch; ++seq) {
+    for (int64_t a = 0; a < s.n_q; a += R) {
+      const int64_t b = a + R < s.n_q ? a + R : s.n_q;
+      const int64_t g0 = seq * s.n_q + a;  // global query of the chunk's row 0
+      int cur = 0, nxt = 1;
+      for (int64_t j = 0; j * W < s.n_blk; ++j) {
+        const int64_t qa = first_row(j, a);
+        if (qa >= b) break;
+        const int64_t qe = (j + 1) * W < s.n_blk ? (first_row(j + 1, a) < b ? first_row(j + 1, a) : b) : b;
+        // rows [qa, qe) end here, rows [qe, b) go on
+        const int64_t q0 = seq * s.n_q + qa;
+        const int blo = (int)(j * W);
+        cudaError_t e = hisa::launch_token_score(s, q_idx, k_idx, nullptr, W, keys, nullptr, q0, b - qa, stream, blo);
+        const uint32_t* keys_go = keys + (qe - qa) * WB;  // key rows of the rows that go on
+        if (j == 0) {
+          if (e == cudaSuccess && qe > qa)
+            e = hisa::launch_token_select(s, keys, nullptr, W, token_idx, token_scores, q0, qe - qa, stream, blo);
+          if (e == cudaSuccess && b > qe)
+            e = hisa::launch_token_select(s, keys_go, nullptr, W, at_row(ids[cur], g0), at_row(sc[cur], g0),
+                                          seq * s.n_q + qe, b - qe, stream, blo);
+        } else {
+          const int64_t ra = qa - a, re = qe - a, rb = b - a;  // chunk rows
+          const int64_t tok0 = (int64_t)blo * s.B;
+          if (e == cudaSuccess && re > ra)
+            e = hisa::launch_flat_select(keys, (int)WB, ids[cur] + ra * k, sc[cur] + ra * k, (int)k, tok0, re - ra,
+                                         token_idx + (g0 + ra) * k,
+                                         token_scores ? token_scores + (g0 + ra) * k : nullptr, stream);
+          if (e == cudaSuccess && rb > re)
+            e = hisa::launch_flat_select(keys_go, (int)WB, ids[cur] + re * k, sc[cur] + re * k, (int)k, tok0, rb - re,
+                                         ids[nxt] + re * k, sc[nxt] + re * k, stream);
+          const int t = cur;
+          cur = nxt;
+          nxt = t;
+        }
+        if (e != cudaSuccess) return hisa::cuda_fail(e);
+      }
+    }
+  }
+  return HISA_OK;
 }
 
 hisa_status_t hisa_block_candidates_workspace_size(const hisa_params_t* local, size_t* bytes) {

@@ -46,16 +46,27 @@ cudaError_t launch_block_topm(const Shape& s, const float* scores, int32_t* bloc
                               cudaStream_t st);
 
 // Steps 4-5 over queries [q0, q0 + nq) (global query ids).  `slots` is the
-// number of block slots per query: m with a block list, n_blk for the flat
-// indexer (block_idx == nullptr: slot r is block r).  keys: [nq][slots * B].
+// number of block slots per query: m with a block list; for the flat indexer
+// (block_idx == nullptr) a window of consecutive blocks, slot r being block
+// blk_lo + r.  keys: [nq][slots * B].
 cudaError_t launch_token_score(const Shape& s, const void* q_idx, const void* k_idx, const int32_t* block_idx,
-                               int slots, uint32_t* keys, int32_t* status, int64_t q0, int64_t nq, cudaStream_t st);
+                               int slots, uint32_t* keys, int32_t* status, int64_t q0, int64_t nq, cudaStream_t st,
+                               int blk_lo = 0);
 // Tensor-core version of launch_token_score for prefill (same key layout).
 bool token_score_tc_eligible(const Shape& s, int slots);
 cudaError_t launch_token_score_tc(const Shape& s, const void* q_idx, const void* k_idx, const int32_t* block_idx,
-                                  int slots, uint32_t* keys, int32_t* status, int64_t q0, int64_t nq, cudaStream_t st);
+                                  int slots, uint32_t* keys, int32_t* status, int64_t q0, int64_t nq, cudaStream_t st,
+                                  int blk_lo = 0);
+// Writes row q (global query id) of the result at token_idx[q * k] (token_scores likewise).
 cudaError_t launch_token_select(const Shape& s, const uint32_t* keys, const int32_t* block_idx, int slots,
-                                int32_t* token_idx, float* token_scores, int64_t q0, int64_t nq, cudaStream_t st);
+                                int32_t* token_idx, float* token_scores, int64_t q0, int64_t nq, cudaStream_t st,
+                                int blk_lo = 0);
+// The flat indexer's streaming top-k for one window after the first: per row r (rows of it), the
+// best k of the running list (run_ids / run_scores [rows][k], tokens below the window) and the
+// window's n keys (keys [rows][n], tokens tok0 ..), by (score desc, token asc), ascending.
+// out_scores may be null.
+cudaError_t launch_flat_select(const uint32_t* keys, int n, const int32_t* run_ids, const float* run_scores, int k,
+                               int64_t tok0, int64_t rows, int32_t* out_ids, float* out_scores, cudaStream_t st);
 
 // Step 6.  The kernel is picked from the shape and the workspace: the query-tile kernel when it
 // applies and `ws` holds its masks, else the gather kernels, with the token lists split across CTAs

@@ -101,7 +101,7 @@ __global__ void __launch_bounds__(TsLayout<D, B, HET>::THREADS, 1)
     token_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                           const int32_t* __restrict__ block_idx, int slots, uint32_t* __restrict__ keys,
                           int32_t* __restrict__ status, int64_t n_q, int64_t n_kv, int q_tiles, int64_t n_tiles,
-                          int64_t q0, int64_t nq, const float* __restrict__ w_idx, int HI) {
+                          int64_t q0, int64_t nq, const float* __restrict__ w_idx, int HI, int blk_lo) {
   using L = TsLayout<D, B, HET>;
   constexpr int S = L::STAGES;
   constexpr int NACC = L::NACC, kEpiWarps = L::EPI_WARPS, kWarpTma = L::WARP_TMA, kWarpMma = L::WARP_MMA;
@@ -222,8 +222,8 @@ __global__ void __launch_bounds__(TsLayout<D, B, HET>::THREADS, 1)
               if (in_range) mx = max(mx, b);
             }
           }
-        } else {  // blocks after the query's own block hold no candidate
-          for (int64_t r = c + 1; r < slots; ++r) {
+        } else {  // slots of the window after the query's own block hold no candidate
+          for (int64_t r = max((int64_t)0, c + 1 - blk_lo); r < slots; ++r) {
             uint4* z = reinterpret_cast<uint4*>(krow_keys + r * B);
             for (int i = 0; i < B / 4; ++i) z[i] = make_uint4(0, 0, 0, 0);
           }
@@ -231,9 +231,19 @@ __global__ void __launch_bounds__(TsLayout<D, B, HET>::THREADS, 1)
       }
       lists[cnt * kTileQ + tid] = 0xFFFF0000u;  // sentinel: above every block
     }
-    if (!block_idx)  // the flat indexer: every block up to the tile's last
-      for (int i = tid; i < nwords; i += kEpiWarps * 32)
-        bits[i] = (32 * i + 31 <= c_max) ? 0xFFFFFFFFu : (0xFFFFFFFFu >> (31 - (c_max & 31)));
+    if (!block_idx) {  // the flat indexer: the window's blocks up to the tile's last
+      const int hi = min(c_max, blk_lo + slots - 1);
+      for (int i = tid; i < nwords; i += kEpiWarps * 32) {
+        const int b0 = 32 * i;
+        uint32_t m = 0u;
+        if (b0 <= hi && b0 + 31 >= blk_lo) {
+          m = 0xFFFFFFFFu;
+          if (blk_lo > b0) m &= 0xFFFFFFFFu << (blk_lo - b0);
+          if (hi < b0 + 31) m &= 0xFFFFFFFFu >> (b0 + 31 - hi);
+        }
+        bits[i] = m;
+      }
+    }
     if constexpr (kTokenMajor) {
       float* wsm = reinterpret_cast<float*>(smem + L::W_OFF);
       if (tid < kTileQ) {
@@ -330,7 +340,7 @@ __global__ void __launch_bounds__(TsLayout<D, B, HET>::THREADS, 1)
     uint32_t ent = (lq_ok && block_idx) ? lists[lq] : 0xFFFF0000u;
     auto slot_of = [&](int b) -> int {
       if (!lq_ok) return -1;
-      if (!block_idx) return b <= lq_c ? b : -1;
+      if (!block_idx) return b <= lq_c ? b - blk_lo : -1;
       while ((int)(ent >> 16) < b) {
         ++cur;
         ent = lists[cur * kTileQ + lq];
@@ -491,7 +501,7 @@ __global__ void __launch_bounds__(TsLayout<D, B, HET>::THREADS, 1)
 
 template <int D, int B, int HET>
 cudaError_t launch_ts(const Shape& s, const void* q_idx, const void* k_idx, const int32_t* block_idx, int slots,
-                      uint32_t* keys, int32_t* status, int64_t q0, int64_t nq, cudaStream_t st) {
+                      uint32_t* keys, int32_t* status, int64_t q0, int64_t nq, cudaStream_t st, int blk_lo) {
   using L = TsLayout<D, B, HET>;
   CUtensorMap mq, mk;
   const int HE = s.HI > 0 ? s.HI : 1;
@@ -509,7 +519,7 @@ cudaError_t launch_ts(const Shape& s, const void* q_idx, const void* k_idx, cons
   const int64_t grid = last - first + 1;
   if (grid > 0x7FFFFFFFLL) return cudaErrorNotSupported;
   kern<<<(unsigned)grid, L::THREADS, L::SMEM, st>>>(mq, mk, block_idx, slots, keys, status, s.n_q, s.n_kv, q_tiles,
-                                                  grid, q0, nq, s.w_idx, s.HI);
+                                                  grid, q0, nq, s.w_idx, s.HI, blk_lo);
   return cudaGetLastError();
 }
 
@@ -524,7 +534,8 @@ bool token_score_tc_eligible(const Shape& s, int slots) {
 }
 
 cudaError_t launch_token_score_tc(const Shape& s, const void* q_idx, const void* k_idx, const int32_t* block_idx,
-                                  int slots, uint32_t* keys, int32_t* status, int64_t q0, int64_t nq, cudaStream_t st) {
+                                  int slots, uint32_t* keys, int32_t* status, int64_t q0, int64_t nq, cudaStream_t st,
+                                  int blk_lo) {
   if (!token_score_tc_eligible(s, slots)) return cudaErrorNotSupported;
   if (block_idx && slots > kListSlots) return cudaErrorNotSupported;  // the CUDA-core scorer takes long lists
   // B = 128 with at least HISA_TS_TM_MIN_HEADS indexer heads: token-major readout (a query's
@@ -532,13 +543,13 @@ cudaError_t launch_token_score_tc(const Shape& s, const void* q_idx, const void*
   const int he = s.HI > 0 ? s.HI : 1;
   if (s.B == 128 && he >= HISA_TS_TM_MIN_HEADS) {
 #define HISA_TS_TM(DD, HH) \
-  if (s.d_idx == DD && he == HH) return launch_ts<DD, 128, HH>(s, q_idx, k_idx, block_idx, slots, keys, status, q0, nq, st);
+  if (s.d_idx == DD && he == HH) return launch_ts<DD, 128, HH>(s, q_idx, k_idx, block_idx, slots, keys, status, q0, nq, st, blk_lo);
     HISA_TS_TM(64, 1) HISA_TS_TM(64, 2) HISA_TS_TM(64, 4) HISA_TS_TM(64, 8) HISA_TS_TM(64, 16)
     HISA_TS_TM(128, 1) HISA_TS_TM(128, 2) HISA_TS_TM(128, 4) HISA_TS_TM(128, 8) HISA_TS_TM(128, 16)
 #undef HISA_TS_TM
   }
 #define HISA_TS_CASE(DD, BB) \
-  if (s.d_idx == DD && s.B == BB) return launch_ts<DD, BB, 0>(s, q_idx, k_idx, block_idx, slots, keys, status, q0, nq, st);
+  if (s.d_idx == DD && s.B == BB) return launch_ts<DD, BB, 0>(s, q_idx, k_idx, block_idx, slots, keys, status, q0, nq, st, blk_lo);
   HISA_TS_CASE(64, 32) HISA_TS_CASE(64, 64) HISA_TS_CASE(64, 128) HISA_TS_CASE(64, 256)
   HISA_TS_CASE(128, 32) HISA_TS_CASE(128, 64) HISA_TS_CASE(128, 128) HISA_TS_CASE(128, 256)
 #undef HISA_TS_CASE

@@ -36,7 +36,7 @@ __global__ void __launch_bounds__(kScoreThreads)
     token_score_kernel(const uint16_t* __restrict__ q_idx, const uint16_t* __restrict__ k_idx,
                        const int32_t* __restrict__ block_idx, int slots, uint32_t* __restrict__ keys,
                        int32_t* __restrict__ status, int64_t n_q, int64_t n_kv, int B, int spc, int chunks,
-                       int64_t q0) {
+                       int64_t q0, int blk_lo) {
   constexpr int CPL = D / 64;  // 16-byte chunks per lane
   constexpr int U = 4;         // token rows in flight per lane group
   __shared__ int s_blk[kMaxSlotsPerCta];
@@ -71,8 +71,8 @@ __global__ void __launch_bounds__(kScoreThreads)
       ok = blk >= 0 && blk <= c && blk > mx;
       if (!ok && blk != -1 && lane == 0 && status) atomicOr(status, kStatusBadIndex);
     } else {
-      blk = r;
-      ok = r <= c;
+      blk = blk_lo + r;
+      ok = blk <= c;
     }
     if (lane == 0) {
       s_blk[rr] = ok ? blk : -1;
@@ -139,7 +139,7 @@ __global__ void __launch_bounds__(kScoreThreads)
     token_score_mh_kernel(const uint16_t* __restrict__ q_idx, const float* __restrict__ w_idx,
                           const uint16_t* __restrict__ k_idx, const int32_t* __restrict__ block_idx, int slots,
                           uint32_t* __restrict__ keys, int32_t* __restrict__ status, int64_t n_q, int64_t n_kv, int B,
-                          int spc, int chunks, int64_t q0, int HI) {
+                          int spc, int chunks, int64_t q0, int HI, int blk_lo) {
   constexpr int CPL = D / 64;  // 16-byte chunks per lane
   __shared__ int s_blk[kMaxSlotsPerCta];
   __shared__ int s_len[kMaxSlotsPerCta];
@@ -172,8 +172,8 @@ __global__ void __launch_bounds__(kScoreThreads)
       ok = blk >= 0 && blk <= c && blk > mx;
       if (!ok && blk != -1 && lane == 0 && status) atomicOr(status, kStatusBadIndex);
     } else {
-      blk = r;
-      ok = r <= c;
+      blk = blk_lo + r;
+      ok = blk <= c;
     }
     if (lane == 0) {
       s_blk[rr] = ok ? blk : -1;
@@ -230,7 +230,7 @@ template <int NT, int V, bool SC>
 __global__ void __launch_bounds__(NT)
     token_select_staged_kernel(const uint32_t* __restrict__ keys, const int32_t* __restrict__ block_idx, int slots,
                                int32_t* __restrict__ token_idx, float* __restrict__ token_scores, int log2B, int k,
-                               int64_t q0) {
+                               int64_t q0, int blk_lo) {
   __shared__ StagedSelectShared<NT> sm;
   extern __shared__ __align__(16) uint32_t dsm[];
   const int B = 1 << log2B;
@@ -241,7 +241,7 @@ __global__ void __launch_bounds__(NT)
   uint32_t* skeys = dsm;
   int32_t* sblk = reinterpret_cast<int32_t*>(dsm + n);
 
-  for (int r = threadIdx.x; r < slots; r += NT) sblk[r] = block_idx ? block_idx[qg * slots + r] : r;
+  for (int r = threadIdx.x; r < slots; r += NT) sblk[r] = block_idx ? block_idx[qg * slots + r] : blk_lo + r;
   for (int i = threadIdx.x; i < kWideBins / 4; i += NT)
     reinterpret_cast<uint4*>(sm.u.hist)[i] = make_uint4(0u, 0u, 0u, 0u);
   __syncthreads();
@@ -277,12 +277,67 @@ __global__ void __launch_bounds__(NT)
   }
 }
 
+// The flat indexer's streaming top-k, one window after the first: row r stages its running list
+// (k entries, ids run_ids[r], tokens of the earlier windows, ascending) ahead of the window's n
+// keys (tokens blk_lo * B ..), so the selection's lowest-position rule is the lowest-token rule,
+// and keeps the best k of both.
+template <int NT>
+__global__ void __launch_bounds__(NT)
+    flat_select_kernel(const uint32_t* __restrict__ keys, int n, const int32_t* __restrict__ run_ids,
+                       const float* __restrict__ run_sc, int k, int64_t tok0, int32_t* __restrict__ out_ids,
+                       float* __restrict__ out_sc) {
+  __shared__ StagedSelectShared<NT> sm;
+  extern __shared__ __align__(16) uint32_t dsm[];
+  const int64_t row = blockIdx.x;
+  const int32_t* ri = run_ids + row * k;
+  const float* rs = run_sc + row * k;
+  const uint32_t* wk = keys + row * (int64_t)n;
+  uint32_t* skeys = dsm;
+  for (int i = threadIdx.x; i < kWideBins / 4; i += NT)
+    reinterpret_cast<uint4*>(sm.u.hist)[i] = make_uint4(0u, 0u, 0u, 0u);
+  __syncthreads();
+  for (int i = threadIdx.x; i < k; i += NT) {
+    const uint32_t key = ri[i] >= 0 ? score_key(rs[i]) : 0u;
+    skeys[i] = key;
+    counts_first_digit(sm.u.hist, key);
+  }
+  if ((n & 3) == 0 && (k & 3) == 0) {
+    const uint4* src = reinterpret_cast<const uint4*>(wk);
+    uint4* dst = reinterpret_cast<uint4*>(skeys + k);
+    for (int i = threadIdx.x; i < n / 4; i += NT) {
+      const uint4 v = src[i];
+      dst[i] = v;
+      counts_first_digit(sm.u.hist, v.x);
+      counts_first_digit(sm.u.hist, v.y);
+      counts_first_digit(sm.u.hist, v.z);
+      counts_first_digit(sm.u.hist, v.w);
+    }
+  } else {
+    for (int i = threadIdx.x; i < n; i += NT) {
+      const uint32_t v = wk[i];
+      skeys[k + i] = v;
+      counts_first_digit(sm.u.hist, v);
+    }
+  }
+  __syncthreads();
+  int32_t* oi = out_ids + row * k;
+  float* os = out_sc ? out_sc + row * k : nullptr;
+  const int K = staged_select<NT>(skeys, n + k, k, sm, [&](int rank, int i, uint32_t key) {
+    oi[rank] = i < k ? ri[i] : (int32_t)(tok0 + (i - k));
+    if (os) os[rank] = key_score(key);
+  });
+  for (int r = K + threadIdx.x; r < k; r += NT) {
+    oi[r] = -1;
+    if (os) os[r] = __int_as_float(0x7FC00000);
+  }
+}
+
 // Rows too long for shared memory: the selection reads the keys from global memory on every pass.
 template <int NT>
 __global__ void __launch_bounds__(NT)
     token_select_kernel(const uint32_t* __restrict__ keys, const int32_t* __restrict__ block_idx, int slots,
                         int32_t* __restrict__ token_idx, float* __restrict__ token_scores, int log2B, int k,
-                        int64_t q0) {
+                        int64_t q0, int blk_lo) {
   __shared__ SelectShared<NT> sm;
   extern __shared__ __align__(16) uint32_t dsm[];
   const int B = 1 << log2B;
@@ -292,7 +347,7 @@ __global__ void __launch_bounds__(NT)
   const uint32_t* row = keys + lq * (int64_t)n;
   int32_t* sblk = reinterpret_cast<int32_t*>(dsm);
 
-  for (int r = threadIdx.x; r < slots; r += NT) sblk[r] = block_idx ? block_idx[qg * slots + r] : r;
+  for (int r = threadIdx.x; r < slots; r += NT) sblk[r] = block_idx ? block_idx[qg * slots + r] : blk_lo + r;
   __syncthreads();
   auto key = [&](int i) -> uint32_t { return row[i]; };
   const int nv = count_nonzero<NT>(key, n, sm);
@@ -316,11 +371,12 @@ __global__ void __launch_bounds__(NT)
 }  // namespace
 
 cudaError_t launch_token_score(const Shape& s, const void* q_idx, const void* k_idx, const int32_t* block_idx,
-                               int slots, uint32_t* keys, int32_t* status, int64_t q0, int64_t nq, cudaStream_t st) {
+                               int slots, uint32_t* keys, int32_t* status, int64_t q0, int64_t nq, cudaStream_t st,
+                               int blk_lo) {
   if (nq <= 0) return cudaSuccess;
   // Many queries per sequence: tensor-core tiles of 128 queries x one key block.
   if (token_score_tc_eligible(s, slots)) {
-    const cudaError_t e = launch_token_score_tc(s, q_idx, k_idx, block_idx, slots, keys, status, q0, nq, st);
+    const cudaError_t e = launch_token_score_tc(s, q_idx, k_idx, block_idx, slots, keys, status, q0, nq, st, blk_lo);
     if (e != cudaErrorNotSupported) return e;
   }
   int spc = 1024 / s.B;
@@ -336,15 +392,15 @@ cudaError_t launch_token_score(const Shape& s, const void* q_idx, const void* k_
     switch (s.d_idx) {
       case 64:
         token_score_mh_kernel<64><<<(unsigned)grid, kScoreThreads, smem, st>>>(
-            qp, s.w_idx, kp, block_idx, slots, keys, status, s.n_q, s.n_kv, s.B, spc, chunks, q0, s.HI);
+            qp, s.w_idx, kp, block_idx, slots, keys, status, s.n_q, s.n_kv, s.B, spc, chunks, q0, s.HI, blk_lo);
         break;
       case 128:
         token_score_mh_kernel<128><<<(unsigned)grid, kScoreThreads, smem, st>>>(
-            qp, s.w_idx, kp, block_idx, slots, keys, status, s.n_q, s.n_kv, s.B, spc, chunks, q0, s.HI);
+            qp, s.w_idx, kp, block_idx, slots, keys, status, s.n_q, s.n_kv, s.B, spc, chunks, q0, s.HI, blk_lo);
         break;
       case 256:
         token_score_mh_kernel<256><<<(unsigned)grid, kScoreThreads, smem, st>>>(
-            qp, s.w_idx, kp, block_idx, slots, keys, status, s.n_q, s.n_kv, s.B, spc, chunks, q0, s.HI);
+            qp, s.w_idx, kp, block_idx, slots, keys, status, s.n_q, s.n_kv, s.B, spc, chunks, q0, s.HI, blk_lo);
         break;
       default: return cudaErrorInvalidValue;
     }
@@ -353,15 +409,15 @@ cudaError_t launch_token_score(const Shape& s, const void* q_idx, const void* k_
   switch (s.d_idx) {
     case 64:
       token_score_kernel<64><<<(unsigned)grid, kScoreThreads, 0, st>>>(qp, kp, block_idx, slots, keys, status, s.n_q,
-                                                                       s.n_kv, s.B, spc, chunks, q0);
+                                                                       s.n_kv, s.B, spc, chunks, q0, blk_lo);
       break;
     case 128:
       token_score_kernel<128><<<(unsigned)grid, kScoreThreads, 0, st>>>(qp, kp, block_idx, slots, keys, status, s.n_q,
-                                                                        s.n_kv, s.B, spc, chunks, q0);
+                                                                        s.n_kv, s.B, spc, chunks, q0, blk_lo);
       break;
     case 256:
       token_score_kernel<256><<<(unsigned)grid, kScoreThreads, 0, st>>>(qp, kp, block_idx, slots, keys, status, s.n_q,
-                                                                        s.n_kv, s.B, spc, chunks, q0);
+                                                                        s.n_kv, s.B, spc, chunks, q0, blk_lo);
       break;
     default: return cudaErrorInvalidValue;
   }
@@ -369,7 +425,8 @@ cudaError_t launch_token_score(const Shape& s, const void* q_idx, const void* k_
 }
 
 cudaError_t launch_token_select(const Shape& s, const uint32_t* keys, const int32_t* block_idx, int slots,
-                                int32_t* token_idx, float* token_scores, int64_t q0, int64_t nq, cudaStream_t st) {
+                                int32_t* token_idx, float* token_scores, int64_t q0, int64_t nq, cudaStream_t st,
+                                int blk_lo) {
   if (nq <= 0) return cudaSuccess;
   const int64_t n = (int64_t)slots * s.B;
   int log2B = 0;
@@ -388,7 +445,8 @@ cudaError_t launch_token_select(const Shape& s, const uint32_t* keys, const int3
 #undef HISA_SEL
     cudaError_t e = ensure_smem((const void*)kern, (int)staged, (int)stat);
     if (e != cudaSuccess) return e;
-    kern<<<(unsigned)nq, nt, (int)staged, st>>>(keys, block_idx, slots, token_idx, token_scores, log2B, s.k, q0);
+    kern<<<(unsigned)nq, nt, (int)staged, st>>>(keys, block_idx, slots, token_idx, token_scores, log2B, s.k, q0,
+                                                 blk_lo);
     return cudaGetLastError();
   }
   const int smem = slots * 4;
@@ -397,7 +455,22 @@ cudaError_t launch_token_select(const Shape& s, const uint32_t* keys, const int3
   const int gstat = (int)(wide ? sizeof(SelectShared<kSelectThreadsWide>) : sizeof(SelectShared<kSelectThreads>));
   cudaError_t e = ensure_smem((const void*)kern, smem, gstat);
   if (e != cudaSuccess) return e;
-  kern<<<(unsigned)nq, nt, smem, st>>>(keys, block_idx, slots, token_idx, token_scores, log2B, s.k, q0);
+  kern<<<(unsigned)nq, nt, smem, st>>>(keys, block_idx, slots, token_idx, token_scores, log2B, s.k, q0, blk_lo);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_flat_select(const uint32_t* keys, int n, const int32_t* run_ids, const float* run_scores, int k,
+                               int64_t tok0, int64_t rows, int32_t* out_ids, float* out_scores, cudaStream_t st) {
+  if (rows <= 0) return cudaSuccess;
+  const int64_t smem = ((int64_t)n + k) * 4;
+  const int stat = (int)sizeof(StagedSelectShared<kSelectThreads>);
+  if (k < 1 || n < 1 || (int64_t)n + k >= 65536 || smem + stat > 227 * 1024 || rows > 0x7FFFFFFFLL)
+    return cudaErrorInvalidValue;
+  auto kern = flat_select_kernel<kSelectThreads>;
+  cudaError_t e = ensure_smem((const void*)kern, (int)smem, stat);
+  if (e != cudaSuccess) return e;
+  kern<<<(unsigned)rows, kSelectThreads, (int)smem, st>>>(keys, n, run_ids, run_scores, k, tok0, out_ids,
+                                                           out_scores);
   return cudaGetLastError();
 }
 

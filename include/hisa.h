@@ -224,7 +224,16 @@ hisa_status_t hisa_forward_cached(const hisa_params_t* params, const void* q_idx
 /* The flat token indexer the two-level one replaces ([IP] 1.1 item 1; [QB]
  * "兩步消除上下文索引瓶頸"): token_idx[s][i] = the min(k, p_i+1) best tokens
  * t <= p_i of the whole sequence.  Same output format as hisa_token_topk;
- * used as the speed comparator and for the degeneration check. */
+ * used as the speed comparator and for the degeneration check.  It runs the
+ * token stage's own kernels over windows of consecutive blocks (8192
+ * candidate tokens, or k rounded up to blocks, a window) and keeps a running
+ * top-k per query, selected again with each window's keys, so no query's
+ * whole row of candidates is ever held at once.  Workspace per query row
+ * processed at once: the window's keys plus four k-entry arrays; min_bytes holds one row,
+ * preferred_bytes all rows (up to 8 GiB), and any size in between is used in
+ * chunks of rows.  Errors: HISA_ERR_WORKSPACE when workspace_bytes is below
+ * min_bytes or the pointer is not 16-byte aligned; HISA_ERR_UNSUPPORTED for
+ * more than 50000 blocks or k of 32768 or more. */
 hisa_status_t hisa_flat_topk_workspace_size(const hisa_params_t* params, size_t* min_bytes,
                                             size_t* preferred_bytes);
 hisa_status_t hisa_flat_topk(const hisa_params_t* params, const void* q_idx, const float* idx_weights,

@@ -102,8 +102,11 @@ def test_workspace_checks_before_launch():
     mn, pref = hs.hisa_token_topk_workspace_size(p)
     assert mn == p.top_m * p.block * 4 and pref == mn * p.n_q
     assert lib.hisa_token_topk(ctypes.byref(p), a, None, a, a, a, None, None, a, mn - 4, None) == hs.HISA_ERR_WORKSPACE
+    # the flat indexer: one row = a window of min(8192 tokens, all 16 blocks) keys, four k-entry
+    # arrays and the alignment slack of its five buffers; preferred = every row
     fmin, fpref = hs.hisa_flat_topk_workspace_size(p)
-    assert fmin == 16 * 64 * 4
+    assert fmin == 16 * 64 * 4 + 4 * 128 * 4 + 5 * 256 and fpref == fmin * p.n_q
+    assert lib.hisa_flat_topk(ctypes.byref(p), a, None, a, a, None, a, fmin - 1, None) == hs.HISA_ERR_WORKSPACE
     need_f = hs.hisa_forward_workspace_size(p)
     assert lib.hisa_forward(ctypes.byref(p), a, None, a, a, a, a, a, None, None, None, None, a, need_f - 1,
                             None) == hs.HISA_ERR_WORKSPACE

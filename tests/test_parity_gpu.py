@@ -116,6 +116,29 @@ def test_flat_matches_oracle_and_degeneration(hs, oracle_lib, w):
     assert np.array_equal(got["token_idx"].cpu().numpy().reshape(n, w.top_k), flat)
 
 
+def test_flat_streaming_windows_prefill(hs, oracle_lib):
+    """The flat indexer over several 8192-token windows on the tensor-core scorer: a chunk whose
+    queries join at different windows (the sequence starts 3000 tokens before the first query),
+    window tops merged into the running top-k.  Sampled rows at window edges against the oracle's
+    flat top-k, indices and scores bit for bit."""
+    w = Workload("flat_windows", 1, 17000, 20000, 128, 128, 4, 700, 1, 1, 64)
+    inp = full_inputs(w)
+    dev = _dev(inp)
+    p = hs.params_of(w)
+    tok = torch.empty((1, w.n_q, w.top_k), dtype=torch.int32, device="cuda")
+    sc = torch.empty((1, w.n_q, w.top_k), dtype=torch.float32, device="cuda")
+    hs.hisa_flat_topk(p, dev["q_idx"], dev["k_idx"], tok, sc)
+    torch.cuda.synchronize()
+    tok = tok.cpu().numpy()[0]
+    sc = sc.cpu().numpy()[0]
+    off = w.n_kv - w.n_q
+    rows = [0, 1, 5191, 5192, 5193, 8000, 13384, 13385, 16999]  # positions 8191 / 8192 / 16383 / 16384 on
+    for i in rows:
+        want, k_eff, wsc = oracle_lib.flat_topk(inp["q_idx"][0, i], inp["k_idx"][0], off + i, w.top_k, scores=True)
+        assert np.array_equal(tok[i], want), (i, np.argwhere(tok[i] != want)[:5])
+        assert np.array_equal(sc[i, :k_eff], wsc[:k_eff].astype(np.float32)), i
+
+
 def test_device_generator_matches_host(hs):
     import synth.device as sd
     from synth.workloads import k_idx_rows
