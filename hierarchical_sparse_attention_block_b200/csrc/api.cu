@@ -379,7 +379,10 @@ namespace {
 // at least kHostChunk queries, at most kHostMaxChunks per sequence: chunk [i0, i1) needs the K/V
 // rows [0, n_kv - n_q + i1) only, so each chunk copies just the rows the earlier ones did not.
 // Short sequences (decode) go in up to kHostGroups groups of whole sequences.
-constexpr int64_t kHostChunk = 8192;
+#ifndef HISA_HOST_CHUNK
+#define HISA_HOST_CHUNK 8192
+#endif
+constexpr int64_t kHostChunk = HISA_HOST_CHUNK;
 constexpr int64_t kHostMaxChunks = 16;
 constexpr int kHostGroups = 8;
 
@@ -418,7 +421,7 @@ Shape unit_shape(const Shape& s, const HostUnit& u) {
 
 struct HostFwdLayout {
   FwdLayout f;
-  size_t part, q_idx, w, k_idx, q, k, v, o, lse, total;
+  size_t part[2], q_idx, w, k_idx, q, k, v, o, lse, total;
 };
 
 HostFwdLayout host_fwd_layout(const Shape& s) {
@@ -436,7 +439,8 @@ HostFwdLayout host_fwd_layout(const Shape& s) {
     return at;
   };
   const int64_t he = s.HI > 0 ? s.HI : 1;
-  L.part = take(part);
+  L.part[0] = take(part);  // the attention workspace of even units and of odd units
+  L.part[1] = take(part);
   L.q_idx = take((size_t)s.n_query * he * s.d_idx * 2);
   L.w = take(s.HI > 0 ? (size_t)s.n_query * s.HI * sizeof(float) : 0);
   L.k_idx = take((size_t)s.batch * s.n_kv * s.d_idx * 2);
@@ -514,6 +518,20 @@ hisa_status_t hisa_forward_host(const hisa_params_t* params, const void* q_idx, 
   const bool overlap = copy_stream != nullptr && copy_stream != stream;
   cudaStream_t cs = overlap ? copy_stream : stream;
   EventSet events;
+  // With copies on their own stream, units alternate between `stream` and a second compute stream
+  // of the call, each with its own workspace part, so that a unit starts on the SMs the previous
+  // unit's last wave leaves idle.
+  cudaStream_t s2 = nullptr;
+  if (overlap && cudaStreamCreateWithFlags(&s2, cudaStreamNonBlocking) != cudaSuccess) {
+    (void)cudaGetLastError();
+    s2 = nullptr;
+  }
+  struct StreamGuard {
+    cudaStream_t st;
+    ~StreamGuard() {
+      if (st) cudaStreamDestroy(st);
+    }
+  } s2_guard{s2};
   // Everything enqueued (on success or after an error) completes before the call returns, so
   // the host buffers and the events are free afterwards.
   auto enqueue = [&]() -> hisa_status_t {
@@ -529,13 +547,18 @@ hisa_status_t hisa_forward_host(const hisa_params_t* params, const void* q_idx, 
         return hisa::cuda_fail(e);
     }
 
-    // Indexer inputs first, then steps 1-5 on stream while the attention inputs stream in.
+    // Indexer inputs first (ahead of the attention inputs on the copy stream, so that they have
+    // the link to themselves), then steps 1-5 on stream while the attention inputs stream in.
     const int64_t he = s.HI > 0 ? s.HI : 1;
     const size_t qrow = (size_t)s.H * s.d * 2, kvrow = (size_t)s.Hkv * s.d * 2;
-    ok(cudaMemcpyAsync(d_q_idx, q_idx, (size_t)s.n_query * he * s.d_idx * 2, cudaMemcpyHostToDevice, stream));
+    ok(cudaMemcpyAsync(d_q_idx, q_idx, (size_t)s.n_query * he * s.d_idx * 2, cudaMemcpyHostToDevice, cs));
     if (d_w) ok(cudaMemcpyAsync(d_w, idx_weights, (size_t)s.n_query * s.HI * sizeof(float), cudaMemcpyHostToDevice,
-                                stream));
-    ok(cudaMemcpyAsync(d_k_idx, k_idx, (size_t)s.batch * s.n_kv * s.d_idx * 2, cudaMemcpyHostToDevice, stream));
+                                cs));
+    ok(cudaMemcpyAsync(d_k_idx, k_idx, (size_t)s.batch * s.n_kv * s.d_idx * 2, cudaMemcpyHostToDevice, cs));
+    if (overlap) {
+      cudaEvent_t idx_in;
+      if (ok(events.make(&idx_in)) && ok(cudaEventRecord(idx_in, cs))) ok(cudaStreamWaitEvent(stream, idx_in, 0));
+    }
     if (e != cudaSuccess) return hisa::cuda_fail(e);
     if (!ok(hisa::launch_block_pool(s, d_k_idx, 0, s.n_blk, bk, stream))) return hisa::cuda_fail(e);
     rc = hisa::run_block_stage(s, d_q_idx, bk, blk, nullptr, dev_status, ws + L.f.blk_stage, stream);
@@ -566,19 +589,32 @@ hisa_status_t hisa_forward_host(const hisa_params_t* params, const void* q_idx, 
     }
     if (e != cudaSuccess) return hisa::cuda_fail(e);
 
-    // Step 6 per unit, as soon as its rows are in.
+    // Step 6 per unit, as soon as its rows are in; odd units on the second compute stream (after
+    // the token stage, and after the unit two before it, which used the same workspace part).
+    if (s2) {
+      cudaEvent_t idx_done;
+      if (!ok(events.make(&idx_done)) || !ok(cudaEventRecord(idx_done, stream)) ||
+          !ok(cudaStreamWaitEvent(s2, idx_done, 0)))
+        return hisa::cuda_fail(e);
+    }
     for (size_t j = 0; j < units.size(); ++j) {
       const HostUnit& u = units[j];
       const Shape c = unit_shape(s, u);
-      if (overlap && !ok(cudaStreamWaitEvent(stream, in[j], 0))) return hisa::cuda_fail(e);
+      const int part = s2 ? (int)(j & 1) : 0;
+      cudaStream_t us = part ? s2 : stream;
+      if (overlap && !ok(cudaStreamWaitEvent(us, in[j], 0))) return hisa::cuda_fail(e);
       const size_t q0 = (size_t)u.s0 * s.n_q + u.i0;  // first query row of the unit
       const size_t kv_off = (size_t)u.s0 * s.n_kv * kvrow;
       if (!ok(hisa::launch_sparse_attn(c, d_q + q0 * qrow, d_k + kv_off, d_v + kv_off, tok + q0 * s.k, d_o + q0 * qrow,
-                                       d_lse + q0 * s.H, dev_status, ws + L.part, hisa::attn_workspace_bytes(c),
-                                       stream)))
+                                       d_lse + q0 * s.H, dev_status, ws + L.part[part], hisa::attn_workspace_bytes(c),
+                                       us)))
         return hisa::cuda_fail(e);
-      if (overlap && ok(events.make(&done[j]))) ok(cudaEventRecord(done[j], stream));
+      if (overlap && ok(events.make(&done[j]))) ok(cudaEventRecord(done[j], us));
       if (e != cudaSuccess) return hisa::cuda_fail(e);
+    }
+    if (s2 && units.size() > 1) {  // stream waits for the second stream's last unit
+      const size_t last_odd = ((units.size() - 1) & 1) ? units.size() - 1 : units.size() - 2;
+      if (!ok(cudaStreamWaitEvent(stream, done[last_odd], 0))) return hisa::cuda_fail(e);
     }
 
     // O and LSE of each unit back to the host once its attention is done.
@@ -601,6 +637,7 @@ hisa_status_t hisa_forward_host(const hisa_params_t* params, const void* q_idx, 
     return hisa::cuda_fail(e);
   };
   const hisa_status_t st = enqueue();
+  if (s2) (void)cudaStreamSynchronize(s2);
   if (overlap) (void)cudaStreamSynchronize(cs);
   const cudaError_t se = cudaStreamSynchronize(stream);
   if (st != HISA_OK) return st;

@@ -194,11 +194,16 @@ hisa_status_t hisa_forward(const hisa_params_t* params, const void* q_idx, const
  * each sequence (a chunk of queries [i0, i1) needs the K/V rows up to its last
  * position only); attention of a chunk starts as soon as its rows have
  * arrived, and its O/LSE rows go back on copy_stream while the next chunk
- * runs.  The selections equal hisa_forward's on the same inputs, and so do o
+ * runs.  With a copy_stream, chunks alternate between stream and a second
+ * compute stream the call creates (each with its own part of the workspace),
+ * so that a chunk starts on the SMs the previous chunk's last wave leaves
+ * idle.  The selections equal hisa_forward's on the same inputs, and so do o
  * and lse bit for bit, except for a chunk or group with so few queries that
  * its token lists are split across CTAs differently (then they differ by the
- * rounding of the split merge).  copy_stream (nullable, or equal to stream)
- * runs the copies; without one everything is serialised on stream.  The call
+ * rounding of the split merge), and when a head's V values reach 2^15 (the
+ * fp16 scale of V then follows the chunk's rows, not all of them).
+ * copy_stream (nullable, or equal to stream) runs the copies; without one
+ * everything is serialised on stream.  The call
  * is synchronous: it returns when o and lse are in host memory (it
  * synchronises stream), so it cannot be captured in a CUDA graph.  Returns
  * HISA_ERR_INVALID_ARG when a host argument is device memory. */
