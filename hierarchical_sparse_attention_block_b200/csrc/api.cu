@@ -676,7 +676,7 @@ hisa_status_t hisa_flat_topk_workspace_size(const hisa_params_t* params, size_t*
   const size_t per = hisa::flat_row_bytes(s) + 5 * hisa::kAlign;
   size_t rows = hisa::kFlatCap / per;
   if (rows < 1) rows = 1;
-  if (rows > (size_t)s.n_q) rows = (size_t)s.n_q;
+  if (rows > (size_t)s.n_query) rows = (size_t)s.n_query;
   if (min_bytes) *min_bytes = per;
   if (preferred_bytes) *preferred_bytes = rows * per;
   return HISA_OK;
@@ -700,7 +700,7 @@ hisa_status_t hisa_flat_topk(const hisa_params_t* params, const void* q_idx, con
   const size_t per = hisa::flat_row_bytes(s) + 5 * hisa::kAlign;
   int64_t R = (int64_t)(workspace_bytes / per);
   if (R < 1) return HISA_ERR_WORKSPACE;
-  if (R > s.n_q) R = s.n_q;
+  if (R > s.n_query) R = s.n_query;
   uint8_t* base = static_cast<uint8_t*>(workspace);
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -727,28 +727,35 @@ hisa_status_t hisa_flat_topk(const hisa_params_t* params, const void* q_idx, con
     const int64_t r = j * WB - off_kv;
     return r > a ? r : a;
   };
-  for (int64_t seq = 0; seq < s.batch; ++seq) {
-    for (int64_t a = 0; a < s.n_q; a += R) {
-      const int64_t b = a + R < s.n_q ? a + R : s.n_q;
-      const int64_t g0 = seq * s.n_q + a;  // global query of the chunk's row 0
+  // When every query sees every window (decode; or sequences whose first query lies past the last
+  // window's start), whole sequences share each window's launches: G of them per group.
+  const int64_t n_win = (s.n_blk + W - 1) / W;
+  const bool all_see = (n_win - 1) * WB <= off_kv;
+  const int64_t G = (all_see && R >= s.n_q) ? R / s.n_q : 1;
+  for (int64_t seq0 = 0; seq0 < s.batch; seq0 += G) {
+    const int64_t nseq = G < s.batch - seq0 ? G : s.batch - seq0;
+    for (int64_t a = 0; a < s.n_q; a += (nseq > 1 ? s.n_q : R)) {
+      const int64_t b = nseq > 1 ? s.n_q : (a + R < s.n_q ? a + R : s.n_q);
+      const int64_t g0 = seq0 * s.n_q + a;  // global query of the chunk's row 0
       int cur = 0, nxt = 1;
-      for (int64_t j = 0; j * W < s.n_blk; ++j) {
+      for (int64_t j = 0; j < n_win; ++j) {
         const int64_t qa = first_row(j, a);
         if (qa >= b) break;
-        const int64_t qe = (j + 1) * W < s.n_blk ? (first_row(j + 1, a) < b ? first_row(j + 1, a) : b) : b;
-        // rows [qa, qe) end here, rows [qe, b) go on
-        const int64_t q0 = seq * s.n_q + qa;
+        const int64_t qe = j + 1 < n_win ? (first_row(j + 1, a) < b ? first_row(j + 1, a) : b) : b;
+        // per sequence, rows [qa, qe) end here and rows [qe, b) go on; as chunk rows (with several
+        // sequences, qa = a = 0 and qe is 0 or n_q, so the ranges cover whole sequences)
+        const int64_t ra = (qa - a) * nseq, re = (qe - a) * nseq, rb = (b - a) * nseq;
         const int blo = (int)(j * W);
-        cudaError_t e = hisa::launch_token_score(s, q_idx, k_idx, nullptr, W, keys, nullptr, q0, b - qa, stream, blo);
-        const uint32_t* keys_go = keys + (qe - qa) * WB;  // key rows of the rows that go on
+        cudaError_t e =
+            hisa::launch_token_score(s, q_idx, k_idx, nullptr, W, keys, nullptr, g0 + ra, rb - ra, stream, blo);
+        const uint32_t* keys_go = keys + (re - ra) * WB;  // key rows of the rows that go on
         if (j == 0) {
-          if (e == cudaSuccess && qe > qa)
-            e = hisa::launch_token_select(s, keys, nullptr, W, token_idx, token_scores, q0, qe - qa, stream, blo);
-          if (e == cudaSuccess && b > qe)
-            e = hisa::launch_token_select(s, keys_go, nullptr, W, at_row(ids[cur], g0), at_row(sc[cur], g0),
-                                          seq * s.n_q + qe, b - qe, stream, blo);
+          if (e == cudaSuccess && re > ra)
+            e = hisa::launch_token_select(s, keys, nullptr, W, token_idx, token_scores, g0 + ra, re - ra, stream, blo);
+          if (e == cudaSuccess && rb > re)
+            e = hisa::launch_token_select(s, keys_go, nullptr, W, at_row(ids[cur], g0), at_row(sc[cur], g0), g0 + re,
+                                          rb - re, stream, blo);
         } else {
-          const int64_t ra = qa - a, re = qe - a, rb = b - a;  // chunk rows
           const int64_t tok0 = (int64_t)blo * s.B;
           if (e == cudaSuccess && re > ra)
             e = hisa::launch_flat_select(keys, (int)WB, ids[cur] + ra * k, sc[cur] + ra * k, (int)k, tok0, re - ra,

@@ -139,6 +139,25 @@ def test_flat_streaming_windows_prefill(hs, oracle_lib):
         assert np.array_equal(sc[i, :k_eff], wsc[:k_eff].astype(np.float32)), i
 
 
+def test_flat_streaming_windows_decode_batch(hs, oracle_lib):
+    """Decode shape (one query per sequence, each seeing every window): whole sequences share each
+    window's launches.  Every sequence's row against the oracle's flat top-k."""
+    w = Workload("flat_decode", 5, 1, 30000, 64, 64, 4, 300, 1, 1, 64)
+    inp = full_inputs(w)
+    dev = _dev(inp)
+    p = hs.params_of(w)
+    tok = torch.empty((w.batch, 1, w.top_k), dtype=torch.int32, device="cuda")
+    sc = torch.empty((w.batch, 1, w.top_k), dtype=torch.float32, device="cuda")
+    hs.hisa_flat_topk(p, dev["q_idx"], dev["k_idx"], tok, sc)
+    torch.cuda.synchronize()
+    tok = tok.cpu().numpy()
+    sc = sc.cpu().numpy()
+    for b in range(w.batch):
+        want, k_eff, wsc = oracle_lib.flat_topk(inp["q_idx"][b, 0], inp["k_idx"][b], w.n_kv - 1, w.top_k, scores=True)
+        assert np.array_equal(tok[b, 0], want), (b, np.argwhere(tok[b, 0] != want)[:5])
+        assert np.array_equal(sc[b, 0, :k_eff], wsc[:k_eff].astype(np.float32)), b
+
+
 def test_device_generator_matches_host(hs):
     import synth.device as sd
     from synth.workloads import k_idx_rows
