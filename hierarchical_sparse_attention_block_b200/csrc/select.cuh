@@ -332,11 +332,15 @@ __device__ void narrow_digit(Visit visit, int shift, uint32_t& prefix, uint32_t&
 }
 
 // Selects the best min(k, keys >= 2^21) keys of skeys[0, n) (n < 65536) and
-// hands them out in ascending position order: put(rank, position, key).  On
+// hands them out in ascending position order: store(rank, ident(position, key),
+// key) -- ident runs on every lane of a group whose position lies in the row,
+// store only on the taken ones (a lone guarded store, so that no lane diverges
+// around a lookup).  On
 // entry sm.u.hist holds the first-digit counts of all n keys and the threads
 // are synchronised.  All NT threads call; returns the number taken.
-template <int NT, class Put>
-__device__ int staged_select(const uint32_t* skeys, int n, int k, StagedSelectShared<NT>& sm, Put put) {
+template <int NT, class Ident, class Store>
+__device__ int staged_select(const uint32_t* skeys, int n, int k, StagedSelectShared<NT>& sm, Ident ident,
+                             Store store) {
   using SS = StagedSelectShared<NT>;
   constexpr int NW = SS::NW, SEG = SS::SEG;
   constexpr int U = 4;  // groups of 32 positions per step
@@ -475,7 +479,10 @@ __device__ int staged_select(const uint32_t* skeys, int n, int k, StagedSelectSh
         eq_seen += __popc(be);
       }
       const uint32_t bs = __ballot_sync(0xFFFFFFFFu, sel);
-      if (sel) put(rank + __popc(bs & below), i, kk[j]);
+      int32_t id = 0;
+      if (in) id = ident(i, kk[j]);  // positions past the row have no identity (nor a slot)
+      const int o = rank + __popc(bs & below);
+      if (sel) store(o, id, kk[j]);
       rank += __popc(bs);
     }
   };

@@ -267,10 +267,12 @@ __global__ void __launch_bounds__(NT)
   __syncthreads();
   int32_t* out = token_idx + qg * k;
   float* osc = token_scores ? token_scores + qg * k : nullptr;
-  const int K = staged_select<NT>(skeys, n, k, sm, [&](int rank, int i, uint32_t key) {
-    out[rank] = sblk[i >> log2B] * B + (i & (B - 1));
-    if constexpr (SC) osc[rank] = key_score(key);
-  });
+  const int K = staged_select<NT>(
+      skeys, n, k, sm, [&](int i, uint32_t) { return sblk[i >> log2B] * B + (i & (B - 1)); },
+      [&](int rank, int32_t id, uint32_t key) {
+        out[rank] = id;
+        if constexpr (SC) osc[rank] = key_score(key);
+      });
   for (int r = K + threadIdx.x; r < k; r += NT) {
     out[r] = -1;
     if (osc) osc[r] = __int_as_float(0x7FC00000);
@@ -322,10 +324,12 @@ __global__ void __launch_bounds__(NT)
   __syncthreads();
   int32_t* oi = out_ids + row * k;
   float* os = out_sc ? out_sc + row * k : nullptr;
-  const int K = staged_select<NT>(skeys, n + k, k, sm, [&](int rank, int i, uint32_t key) {
-    oi[rank] = i < k ? ri[i] : (int32_t)(tok0 + (i - k));
-    if (os) os[rank] = key_score(key);
-  });
+  const int K = staged_select<NT>(
+      skeys, n + k, k, sm, [&](int i, uint32_t) { return i < k ? ri[i] : (int32_t)(tok0 + (i - k)); },
+      [&](int rank, int32_t id, uint32_t key) {
+        oi[rank] = id;
+        if (os) os[rank] = key_score(key);
+      });
   for (int r = K + threadIdx.x; r < k; r += NT) {
     oi[r] = -1;
     if (os) os[r] = __int_as_float(0x7FC00000);
