@@ -134,7 +134,9 @@ hisa_status_t hisa_block_topm(const hisa_params_t* params, const void* q_idx, co
 
 /* Steps 4-5 -- [IP] 1.2.2 items 1-2; [QB] "塊內精挑字符".
  * token_idx[s][i][0..k): the min(k, candidates) best tokens t <= p_i of the
- * blocks in block_idx[s][i], ascending, -1 padded.  token_scores (nullable)
+ * blocks in block_idx[s][i], ascending, -1 padded (a token whose score is a
+ * NaN of negative sign with one of the largest payloads -- no arithmetic
+ * produces one -- counts as no candidate).  token_scores (nullable)
  * [b][n_q][k] fp32: their indexer scores (NaN for padding).  dev_status
  * (nullable) int32 on the device, see conventions.  Any workspace of at least
  * the reported minimum works; more lets more queries run per launch. */
