@@ -383,7 +383,11 @@ cudaError_t launch_token_score(const Shape& s, const void* q_idx, const void* k_
     const cudaError_t e = launch_token_score_tc(s, q_idx, k_idx, block_idx, slots, keys, status, q0, nq, st, blk_lo);
     if (e != cudaErrorNotSupported) return e;
   }
+  // Up to 1024 tokens per CTA; with few queries (decode) fewer, so that the grid has about four
+  // CTAs per SM to hide the gathers' latency.
   int spc = 1024 / s.B;
+  const int64_t want = (nq * slots + 4 * 148 - 1) / (4 * 148);  // slots per CTA for ~4 waves
+  if (want < spc) spc = (int)want;
   spc = spc < 1 ? 1 : (spc > kMaxSlotsPerCta ? kMaxSlotsPerCta : spc);
   if (spc > slots) spc = slots;
   const int chunks = (slots + spc - 1) / spc;
